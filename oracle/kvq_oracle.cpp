@@ -31,6 +31,7 @@
 //    code = clamp(rint((x - z) * (1/s)), 0, qmax), rint = round-half-even.
 //    z is clamped to >= -65504 and s to <= 65504 (fp16 finite range).
 //  * s == 0 (constant group whose value is fp16-representable): codes are 0.
+//  * signed zeros: the min and max of a set are taken as +0 when they are zero.
 //  * fp32 inputs are rounded to bf16 (round-to-nearest-even) at entry.
 //  * q head h reads KV head h / (Hq/Hkv); softmax scale 1/sqrt(D); no mask.
 //  * empty sequence: output 0.
@@ -125,6 +126,10 @@ void quantize_set(const float* x, int n, int bits, uint8_t* codes,
   const int qmax = (1 << bits) - 1;
   float mn = x[0], mx = x[0];
   for (int i = 1; i < n; ++i) { mn = std::min(mn, x[i]); mx = std::max(mx, x[i]); }
+  // A set whose minimum (or maximum) is zero may hold both -0 and +0; which one
+  // the min/max returns depends on order. Adding +0 makes either one +0.
+  mn = mn + 0.0f;
+  mx = mx + 0.0f;
   uint16_t zb = f32_to_f16_directed(mn, /*up=*/false);
   float z = (float)f16_value(zb);
   if (z < -65504.0f) { z = -65504.0f; zb = f16_encode_exact(-65504.0, false); }

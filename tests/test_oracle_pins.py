@@ -230,6 +230,16 @@ def test_quantizer_constant_channel_exact(oracle, bits):
             assert np.all(np.abs(codes * s + z - xv) <= s / 2 + abs(xv) * 2 ** -22)
 
 
+def test_quantizer_signed_zero_minimum(oracle):
+    # {-0, +0, 1}: the zero point is +0 whichever zero comes first
+    for x in ([-0.0, 0.0, 1.0], [0.0, -0.0, 1.0], [1.0, -0.0, 0.0]):
+        codes, sb, zb = oracle.quantize(np.array(x * 11, dtype=np.float32)[:32], 4)
+        assert zb == 0x0000
+        assert list(codes[:3]) == [0 if v == 0 else 15 for v in x]
+    codes, sb, zb = oracle.quantize(np.array([-0.0] * 32, dtype=np.float32), 2)
+    assert zb == 0x0000 and sb == 0x0000
+
+
 def test_quantizer_two_level_set(oracle):
     # {a, b} with a < b, both fp16-representable: z = a, s = ru((b-a)/qmax),
     # a -> code 0, b -> qmax.
