@@ -1,0 +1,374 @@
+"""Benchmark of the mixed-precision KV decode step on B200.
+
+One step = for every layer of the stack: append one new token per sequence
+(kvq_append) and decode attention for every query head (kvq_decode_attn), over
+a cache prefilled to the workload's context. Default workload: the
+Llama-3.1-8B-shaped uniform K4V4 stack (32 layers, 32 query / 8 KV heads,
+head_dim 128, batch 16, context 4096).
+
+value = algorithmic HBM bytes per step (packed codes, fp16 scales/zeros, bf16
+window of every layer at the step's context) / device time per step, in GB/s.
+The cache (2.5 GB) is far larger than the 126 MB L2, so no flush is needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from layer_wise_mixed_kvq_b200 import replicas, synth  # noqa: E402
+
+METRIC = "quantized-KV decode attention HBM GB/s (% of B200 peak) and decode steps/s"
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default="llama_k4v4", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "layer_wise_mixed_kvq_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("kvq_decode") and name.endswith(".cu"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(workload):
+    """dram bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source."""
+    path = os.path.join(PROFILES, "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------- clocks --
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------- CPU oracle --
+def cpu_baseline(w, seconds):
+    """The oracle, as it stands, timed on this host on a bounded sample of the
+    workload: whole layers (every KV head) of single sequences at the
+    workload's context, prefill appends untimed, decode attention timed."""
+    import oracle
+    oracle.build()
+    done_bytes, t_attn, samples = 0, 0.0, 0
+    layer = 0
+    ctx = int(synth.context_lengths(w, 1)[0])
+    while t_attn < seconds and samples < 64:
+        pair = w.layer_map[layer % w.n_layers]
+        L = oracle.OracleLayer(pair[0], pair[1], 1, w.n_kv_heads, w.head_dim)
+        K, V = synth.kv_tokens(w, layer, ctx + 1)
+        L.append(K, V, [ctx + 1])
+        Q = synth.queries(w, layer, batch=1)
+        t0 = time.perf_counter()
+        L.attend(Q)
+        t_attn += time.perf_counter() - t0
+        T = ctx + 1
+        P, W = T // 32, T % 32
+        page = oracle.page_bytes(pair[0], pair[1], w.head_dim)
+        done_bytes += w.n_kv_heads * (P * page + W * w.head_dim * 4)
+        samples += 1
+        layer += 1
+    gbs = done_bytes / t_attn / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{samples} single-sequence layer(s) of {w.name} at context {ctx + 1}, all "
+                      f"{w.n_q_heads} query heads, fp64 attention; {t_attn:.1f} s of attention",
+            "decode_layers_per_s": samples / t_attn}
+
+
+def run_reference(args, w):
+    rank, world, _ = replicas.world()
+    if rank != 0:
+        return 0
+    cb = cpu_baseline(w, args.cpu_seconds / 2)
+    # one "step" = one full layer stack for one sequence, bounded per step
+    per_layer_s = 1.0 / cb["decode_layers_per_s"]
+    bytes_per_layer = cb["value"] * 1e9 * per_layer_s
+    value = cb["value"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_layer_s * w.n_layers * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": 1, "context": w.context, "layers": w.n_layers,
+                   "note": "CPU oracle on a bounded sample (single sequence per layer)"},
+        "cpu_baseline": {k: cb[k] for k in ("kind", "cores", "sample")} | {"value": value, "unit": "GB/s"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "bytes_per_layer": bytes_per_layer,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU --
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = replicas.world()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    from layer_wise_mixed_kvq_b200 import kvq
+
+    B, Hq, Hkv, D, NL = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.n_layers
+    lens = synth.context_lengths(w)
+    total_steps = args.warmup + args.steps
+    max_tokens = int(lens.max()) + total_steps + 32  # + the end-to-end steps
+    cache = kvq.kvq_cache_create(list(w.layer_map), Hq, Hkv, D, B, max_tokens)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed * 1000 + rank)
+
+    # prefill every layer (timed separately: append tokens/s)
+    pre_ms = 0.0
+    for layer in range(NL):
+        K, V = synth.torch_kv_tokens(w, layer, int(lens.sum()), dev, gen)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvq.kvq_append(cache, layer, K, V, [int(x) for x in lens])
+        e1.record()
+        torch.cuda.synchronize()
+        pre_ms += e0.elapsed_time(e1)
+        del K, V
+    prefill_tokens = int(lens.sum()) * NL
+
+    # per-step inputs resident in HBM
+    steps_K, steps_V, steps_Q = [], [], []
+    for s in range(total_steps):
+        kl, vl, ql = [], [], []
+        for layer in range(NL):
+            k1, v1 = synth.torch_kv_tokens(w, layer, B, dev, gen)
+            kl.append(k1)
+            vl.append(v1)
+            ql.append(torch.randn((B, Hq, D), device=dev, generator=gen).to(torch.bfloat16))
+        steps_K.append(kl)
+        steps_V.append(vl)
+        steps_Q.append(ql)
+    outs = [torch.empty((B, Hq, D), device=dev, dtype=torch.float32) for _ in range(NL)]
+    ones = [1] * B
+    stream = torch.cuda.current_stream()
+
+    def step(s, events=None):
+        for layer in range(NL):
+            kvq.kvq_append(cache, layer, steps_K[s][layer], steps_V[s][layer], ones, stream)
+            if events is not None:
+                events[layer][0].record(stream)
+            kvq.kvq_decode_attn(cache, layer, steps_Q[s][layer], outs[layer], stream)
+            if events is not None:
+                events[layer][1].record(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    def step_bytes():
+        return sum(kvq.kvq_bytes(cache, layer, B, True) for layer in range(NL))
+
+    bytes_before = step_bytes()
+    launches0 = kvq.kvq_launch_count(cache)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(NL)]
+          for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        replicas.barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for s in range(args.steps):
+            step(args.warmup + s, ev[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        replicas.barrier()
+    launches = kvq.kvq_launch_count(cache) - launches0
+    bytes_after = step_bytes()
+    # the step at context c reads the cache after its own append
+    bytes_per_step = (bytes_before + bytes_after) / 2.0
+    local_ms = t0.elapsed_time(t1)
+    attn_ms = [ev[s][l][0].elapsed_time(ev[s][l][1]) for s in range(args.steps) for l in range(NL)]
+    total_bytes, max_ms, _ = replicas.aggregate(bytes_per_step * args.steps, local_ms)
+    ms_per_step = max_ms / args.steps
+    value = total_bytes / (max_ms / 1e3) / 1e9
+    attn_avg_ms = float(np.mean(attn_ms))
+    attn_gbs = (bytes_per_step / NL) / (attn_avg_ms / 1e3) / 1e9
+    peak, peak_kind = peaks()
+
+    # ---- end to end through the public API with host buffers ----
+    e2e_steps = max(3, min(args.steps, 20))
+    hK = [[t.cpu().pin_memory() for t in steps_K[s % total_steps]] for s in range(e2e_steps)]
+    hV = [[t.cpu().pin_memory() for t in steps_V[s % total_steps]] for s in range(e2e_steps)]
+    hQ = [[t.cpu().pin_memory() for t in steps_Q[s % total_steps]] for s in range(e2e_steps)]
+    hO = [torch.empty((B, Hq, D), dtype=torch.float32).pin_memory() for _ in range(NL)]
+    dK = [torch.empty_like(t) for t in steps_K[0]]
+    dV = [torch.empty_like(t) for t in steps_V[0]]
+    dQ = [torch.empty_like(t) for t in steps_Q[0]]
+    h2d = sum(t.numel() * t.element_size() for t in hK[0] + hV[0] + hQ[0])
+    d2h = sum(t.numel() * t.element_size() for t in hO)
+    e2e_bytes0 = step_bytes()
+    replicas.barrier()
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(e2e_steps):
+        for layer in range(NL):
+            dK[layer].copy_(hK[s][layer], non_blocking=True)
+            dV[layer].copy_(hV[s][layer], non_blocking=True)
+            dQ[layer].copy_(hQ[s][layer], non_blocking=True)
+            kvq.kvq_append(cache, layer, dK[layer], dV[layer], ones, stream)
+            kvq.kvq_decode_attn(cache, layer, dQ[layer], outs[layer], stream)
+            hO[layer].copy_(outs[layer], non_blocking=True)
+    b_.record(stream)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    e2e_local = a.elapsed_time(b_)
+    e2e_bytes = (e2e_bytes0 + step_bytes()) / 2.0
+    e2e_total, e2e_max, _ = replicas.aggregate(e2e_bytes * e2e_steps, e2e_local)
+    e2e_value = e2e_total / (e2e_max / 1e3) / 1e9
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w, args.cpu_seconds)
+        cb.pop("decode_layers_per_s", None)
+
+    traffic = traffic_from_profile(w.name)
+    clocks = clk.summary()
+    result = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4/int2/int8 codes + bf16, fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": w.name, "layers": NL, "layer_map_equiv_bits": kvq.kvq_equiv_bits(list(w.layer_map)),
+                   "batch": B, "n_q_heads": Hq, "n_kv_heads": Hkv, "head_dim": D,
+                   "context": int(lens.max()), "parallelism": f"replicas x{world}",
+                   "l2": "cache larger than L2 (no flush)"},
+        "pct_of_peak": value / peak,
+        "decode_steps_per_s": 1e3 / ms_per_step,
+        "tokens_per_s": B * world * 1e3 / ms_per_step,
+        "append_prefill_tokens_per_s": prefill_tokens / (pre_ms / 1e3),
+        "bytes_per_step": bytes_per_step,
+        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": attn_gbs / peak, "traffic": traffic,
+                     "kernel": "decode attention (kvq_decode_attn), mean over launches in the timed region",
+                     "peak_kind": peak_kind, "avg_launch_us": attn_avg_ms * 1e3},
+        "cpu_baseline": cb,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "ms_per_step": e2e_max / e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    kvq.kvq_cache_destroy(cache)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        print("warmup must be >= 3", file=sys.stderr)
+        return 2
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

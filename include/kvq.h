@@ -1,0 +1,198 @@
+/*
+ * kvq.h -- C ABI of libkvq: decode attention over a KV cache whose precision
+ * pair (key bits, value bits) is set per layer by an offline-searched layer map.
+ *
+ * The method is KVTuner ("KVTuner: Sensitivity-Aware Layer-wise Mixed Precision
+ * KV Cache Quantization", arXiv 2502.04420). The pages this library follows:
+ *   [facts]  llms-explorer.com, "Mixed-precision KV-cache quantization
+ *            per-layer sensitivity" -- facts list (per-layer pairs applied at
+ *            inference with no online decision; keys per-channel asymmetric,
+ *            values per-token asymmetric; 3.25-bit / 4.0-bit maps).
+ *   [abs]    mlsanity.com, arXiv 2502.04420 abstract (layer-wise precision pairs,
+ *            offline-searched configurations used during online inference).
+ *   [qa]     machinoai.in Q&A on mixed BF16/FP8 KV, section 2 (byte accounting,
+ *            sensitive layers kept in BF16).
+ *   [rebut]  paperhub.cn OpenReview rebuttal: "Computational cost" (only newly
+ *            generated tokens are quantized online), "Baseline Implementation"
+ *            (FlashAttention-style decode kernels over int8 / mixed K-V
+ *            precision), "New GQA efficiency results" (GQA), and the per-layer
+ *            K4V8 facts for layers 0, 1, 2, 31 of Llama-3.1-8B-Instruct.
+ *
+ * Fixed by this library where the pages are silent: key groups of 32 tokens
+ * (one fp16 scale and zero per channel per group), one fp16 scale and zero per
+ * value token, and a bf16 window holding the most recent (T mod 32) tokens that
+ * are not yet quantized.
+ *
+ * Conventions for every call:
+ *  - Device pointers are plain CUDA device addresses (e.g. a torch tensor's
+ *    data_ptr()); `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *    default stream). Calls only enqueue work: none synchronises the device
+ *    except kvq_export_layer and kvq_sync.
+ *  - The caller owns Q, K, V, out and the stream. The library owns the cache
+ *    metadata and, unless a device pool is passed to kvq_cache_create, the
+ *    device memory of the cache.
+ *  - Errors are returned as kvq_status; no exception crosses the ABI. Invalid
+ *    arguments and capacity overflow are detected on the host before any launch
+ *    and leave the cache unchanged. kvq_last_error() gives a message for the
+ *    last failing call on the calling thread.
+ *  - Sequence lengths are mirrored on the host; no call reads them back.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kvq_cache kvq_cache;
+
+/* One layer's precision pair: k_bits, v_bits in {2, 4, 8}, or {16, 16} for a
+ * layer kept in bf16 ([qa] section 2: sensitive layers stay BF16; [facts]:
+ * vLLM-style skip layers). Mixed bf16/int pairs are rejected. */
+typedef struct {
+  uint8_t k_bits;
+  uint8_t v_bits;
+} kvq_pair;
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_EINVAL = 1,    /* bad argument: null/misaligned pointer, bad layer, bad pair, bad shape */
+  KVQ_ECAPACITY = 2, /* append would exceed max_tokens or max_batch */
+  KVQ_ENOMEM = 3,    /* device allocation failed or the given pool is too small */
+  KVQ_ECUDA = 4      /* a CUDA call failed (message in kvq_last_error) */
+} kvq_status;
+
+typedef enum {
+  KVQ_BF16 = 0, /* bfloat16 */
+  KVQ_F32 = 1   /* float32; rounded to bf16 (round-to-nearest-even) on entry */
+} kvq_dtype;
+
+/*
+ * Storage format (per layer, per sequence b, per KV head h).
+ * Tokens [0, 32*floor(T/32)) live in full 32-token pages; the remaining
+ * W = T mod 32 tokens live in a bf16 window [2][32][head_dim] (keys, values;
+ * row = slot = token mod 32). A page is 16-byte aligned and holds
+ *   quantized pair: [K codes 4*D*k_bits B][V codes 4*D*v_bits B]
+ *                   [K scale D x fp16][K zero D x fp16][V scale 32 x fp16][V zero 32 x fp16]
+ *   bf16 layer:     [K 64*D B][V 64*D B]
+ * Code blocks are stored as 16x16 tiles f = 2*dt + tt (dt: 16-channel tile,
+ * tt: 16-token tile) laid out so that lane l = 4g + t of a warp reads its eight
+ * elements of every tile as contiguous 16-byte vectors: element e = 2p + j of
+ * tile f sits at row g + 8*(p & 1), column 2t + j + 8*(p >> 1), rows being
+ * tokens for keys and channels for values. Lane word w of lane l lives at byte
+ * ((w/4)*32 + l)*16 + (w%4)*4; 8-bit tiles take two words (element e in byte e),
+ * 4-bit tiles one word (nibble (e>>1) + 4*(e&1)), two 2-bit tiles share a word
+ * (slot 4u + (e>>1) + 8*(e&1) for tile 2w+u), bf16 tiles four words (half e).
+ * Key scale/zero entry i holds channel 16*dt + 2t + (j&1) + 8*(j>>1) with
+ * t = i/(D/4), dt = (i%(D/4))/4, j = i%4.
+ */
+
+/* Bytes of one 32-token page of `pair` at head_dim D (0 if invalid). */
+int64_t kvq_page_bytes(kvq_pair pair, int head_dim);
+
+/* Equivalent bitwidth of a layer map: the mean over layers of
+ * (k_bits + v_bits)/2, bf16 layers counting 16 ([facts], [abs]: 3.25-bit and
+ * 4.0-bit maps). Scales and zero points are not counted. Returns -1.0 on an
+ * invalid map. Host only, pure. */
+double kvq_equiv_bits(const kvq_pair* layer_map, int n_layers);
+
+/* Device bytes kvq_cache_create needs for these dimensions (0 if invalid).
+ * Use it to size a caller-owned pool. */
+size_t kvq_cache_pool_bytes(const kvq_pair* layer_map, int n_layers, int n_q_heads, int n_kv_heads,
+                            int head_dim, int max_batch, int64_t max_tokens);
+
+/* Create a cache for `n_layers` layers with the given per-layer pairs
+ * ([facts]: the per-layer configuration is searched offline and applied at
+ * inference with no online decision). n_q_heads must be a multiple of
+ * n_kv_heads with n_q_heads/n_kv_heads in [1, 8] (GQA, [rebut] "New GQA
+ * efficiency results"); head_dim in {64, 128}; max_batch in [1, 1024];
+ * max_tokens >= 1 per sequence.
+ * device_pool/pool_bytes: a caller-owned, 256-byte-aligned device buffer of at
+ * least kvq_cache_pool_bytes(...) bytes, or NULL/0 for the library to allocate
+ * with cudaMalloc. Uses the current CUDA device. The new cache holds empty
+ * sequences. On error *out is set to NULL. */
+kvq_status kvq_cache_create(const kvq_pair* layer_map, int n_layers, int n_q_heads, int n_kv_heads,
+                            int head_dim, int max_batch, int64_t max_tokens, void* device_pool,
+                            size_t pool_bytes, kvq_cache** out);
+
+/* Release the cache (synchronises the device first). NULL is a no-op. */
+void kvq_cache_destroy(kvq_cache* cache);
+
+/* Empty every sequence of every layer (enqueued on `stream`). */
+kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
+
+/* Append n_new[b] tokens to sequence b of `layer`, for b < batch ([rebut]
+ * "Computational cost": only the newly generated keys and values are quantized
+ * online, with the layer's calibrated pair).
+ *   K, V: device, [sum(n_new), n_kv_heads, head_dim] in `dtype`, sequences packed
+ *         in order b = 0..batch-1, 16-byte aligned.
+ *   n_new: host array [batch], each >= 0.
+ * Tokens enter the bf16 window; every time a sequence's window reaches 32
+ * tokens they are quantized as one group -- keys per channel over the 32
+ * tokens, values per token over head_dim ([facts]: per-channel asymmetric keys,
+ * per-token asymmetric values) -- bit-packed into the next page, and the window
+ * is emptied. The stored result does not depend on how tokens are split across
+ * calls. Quantizer: z = fp16 round-down(min), s = fp16 round-up((max - z)/qmax),
+ * code = clamp(rint((x - z) * (1/s)), 0, 2^bits - 1); all fp32 steps are single
+ * IEEE operations; z is clamped to >= -65504 and s to <= 65504; s = 0 gives
+ * all-zero codes. Inputs must be finite.
+ * Errors: KVQ_EINVAL (bad layer, batch, pointer, dtype), KVQ_ECAPACITY (some
+ * sequence would pass max_tokens); the cache is unchanged on error. */
+kvq_status kvq_append(kvq_cache* cache, int layer, const void* K, const void* V, kvq_dtype dtype,
+                      const int32_t* n_new, int batch, void* stream);
+
+/* Decode attention of `layer` for sequences b < batch ([rebut] "Baseline
+ * Implementation": FlashAttention-style decoding over the quantized cache):
+ *   out[b, hq, :] = sum_t softmax_t(q . k_t / sqrt(D)) v_t over every token
+ *   appended so far, keys/values dequantized as code*s + z (window tokens
+ *   exact bf16), q head hq reading KV head hq / (n_q_heads/n_kv_heads).
+ *   Q:   device bf16 [batch, n_q_heads, head_dim], 16-byte aligned.
+ *   out: device fp32 [batch, n_q_heads, head_dim], 16-byte aligned.
+ * An empty sequence gives zeros. One kernel launch: the sequence is split
+ * across CTAs and the last CTA of each (sequence, KV head) merges the partial
+ * softmax states. Errors: KVQ_EINVAL. */
+kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch, float* out,
+                           void* stream);
+
+/* Pages per split-K CTA for kvq_decode_attn: 0 = automatic (default). Changing
+ * it changes only the rounding order of the result. */
+kvq_status kvq_set_split_pages(kvq_cache* cache, int pages_per_split);
+
+/* Tokens currently held by sequence `seq` of `layer` (host mirror), -1 if invalid. */
+int64_t kvq_seq_len(const kvq_cache* cache, int layer, int seq);
+
+/* Bytes the decode attention of `layer` reads for sequences b < batch at their
+ * current lengths: packed codes, plus (include_metadata != 0) fp16 scales/zeros
+ * and the bf16 window. -1 if invalid. */
+int64_t kvq_bytes(const kvq_cache* cache, int layer, int batch, int include_metadata);
+
+/* Size of kvq_export_layer's output for sequences b < batch, -1 if invalid. */
+int64_t kvq_export_bytes(const kvq_cache* cache, int layer, int batch);
+
+/* Copy `layer`'s stored state to host memory (synchronises the device): for
+ * b < batch, for each KV head: the full pages (raw, format above), then the
+ * window keys [W][D] bf16, then the window values [W][D] bf16. `bytes` must be
+ * at least kvq_export_bytes(cache, layer, batch). */
+kvq_status kvq_export_layer(const kvq_cache* cache, int layer, int batch, void* host_dst,
+                            size_t bytes);
+
+/* Wait for the cache's work and report any asynchronous CUDA error. */
+kvq_status kvq_sync(kvq_cache* cache);
+
+/* Number of kernels the library has launched on this cache so far. */
+int64_t kvq_launch_count(const kvq_cache* cache);
+
+/* Message describing the last failing call on this thread ("" if none). */
+const char* kvq_last_error(void);
+
+/* Name of a status code. */
+const char* kvq_status_string(kvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,451 @@
+// kvq_api.cu -- the C ABI of libkvq: argument checks, device memory layout,
+// host mirror of sequence lengths, and the layer-map dispatcher that picks the
+// kernel instance of each layer's (key bits, value bits) pair.
+//
+// The layer map is fixed at creation: KVTuner applies its offline-searched
+// per-layer configuration at inference with no online decision (llms-explorer
+// facts page; arXiv 2502.04420 abstract), so dispatch is a table lookup.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "kvq_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvq_status fail(kvq_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+kvq_status cuda_fail(cudaError_t e, const char* what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return KVQ_ECUDA;
+}
+
+bool valid_pair(kvq_pair p) {
+  auto ok = [](int b) { return b == 2 || b == 4 || b == 8; };
+  return (p.k_bits == 16 && p.v_bits == 16) || (ok(p.k_bits) && ok(p.v_bits));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Geometry {
+  int64_t max_pages = 0;
+  std::vector<size_t> page_region, window_region;
+  size_t len_region = 0, partial_region = 0, merge_region = 0, append_region = 0, plan_region = 0;
+  int64_t partial_slots = 0;
+  size_t total = 0;
+};
+
+// Split-K partial slots: enough for every (sequence, head) to take 2 splits, and
+// at least 16 per SM of a 148-SM part.
+int64_t partial_slots_for(int max_batch, int n_kv_heads) {
+  return std::max<int64_t>((int64_t)max_batch * n_kv_heads * 2, 148LL * 16);
+}
+
+bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_heads, int head_dim,
+                   int max_batch, int64_t max_tokens, Geometry& g, std::string& why) {
+  if (!map || n_layers <= 0) { why = "layer_map is null or n_layers <= 0"; return false; }
+  for (int l = 0; l < n_layers; ++l)
+    if (!valid_pair(map[l])) {
+      why = "layer " + std::to_string(l) + " has an unsupported pair (k_bits, v_bits) = (" +
+            std::to_string(map[l].k_bits) + ", " + std::to_string(map[l].v_bits) + ")";
+      return false;
+    }
+  if (head_dim != 64 && head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
+  if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads != 0 ||
+      n_q_heads / n_kv_heads > kvq::kMaxGqa) {
+    why = "n_q_heads must be a positive multiple of n_kv_heads with at most 8 query heads per KV head";
+    return false;
+  }
+  if (max_batch <= 0 || max_batch > kvq::kMaxBatch) { why = "max_batch must be in [1, 1024]"; return false; }
+  if (max_tokens <= 0 || max_tokens > (int64_t)1 << 30) { why = "max_tokens must be in [1, 2^30]"; return false; }
+  g.max_pages = max_tokens / kvq::kPageTokens;
+  size_t total = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    size_t pb = (size_t)kvq::page_bytes_of(map[l].k_bits, map[l].v_bits, head_dim);
+    size_t pr = round_up((size_t)max_batch * n_kv_heads * std::max<int64_t>(g.max_pages, 1) * pb);
+    size_t wr = round_up((size_t)max_batch * n_kv_heads * 2 * kvq::kPageTokens * head_dim * 2);
+    g.page_region.push_back(pr);
+    g.window_region.push_back(wr);
+    total += pr + wr + round_up((size_t)max_batch * 4);
+  }
+  g.len_region = round_up((size_t)max_batch * 4);
+  g.partial_slots = partial_slots_for(max_batch, n_kv_heads);
+  int G = n_q_heads / n_kv_heads;
+  g.partial_region = round_up((size_t)g.partial_slots * G * (head_dim + 2) * 4);
+  g.merge_region = round_up((size_t)max_batch * n_kv_heads * 4);
+  g.append_region = round_up((size_t)max_batch * 4);
+  g.plan_region = round_up((size_t)max_batch * 4 * 4);
+  total += g.partial_region + g.merge_region + g.append_region + g.plan_region;
+  g.total = total;
+  return true;
+}
+
+kvq_status check_cache(const kvq_cache* c, int layer) {
+  if (!c) return fail(KVQ_EINVAL, "cache is null");
+  if (layer < 0 || layer >= c->n_layers) return fail(KVQ_EINVAL, "layer index out of range");
+  return KVQ_OK;
+}
+
+// Pages per split-K CTA: enough CTAs to cover the GPU about 4 times over, at
+// least 2 pages per CTA, and no more splits per (b, h) than the partial buffer
+// holds.
+int choose_chunk(const kvq_cache* c, int64_t total_pages, int64_t max_p, int batch) {
+  int64_t target_ctas = (int64_t)c->sm_count * 4;
+  int64_t chunk = std::max<int64_t>(2, (total_pages + target_ctas - 1) / std::max<int64_t>(target_ctas, 1));
+  int64_t stride = c->partial_slots / ((int64_t)batch * c->n_kv_heads);
+  if (stride < 1) stride = 1;
+  chunk = std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
+  return (int)std::max<int64_t>(chunk, 1);
+}
+
+}  // namespace
+
+namespace kvq {
+cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  return launch_decode_simt(kb, vb, D, p, grid, s);
+}
+}  // namespace kvq
+
+extern "C" {
+
+const char* kvq_last_error(void) { return g_last_error.c_str(); }
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "KVQ_OK";
+    case KVQ_EINVAL: return "KVQ_EINVAL";
+    case KVQ_ECAPACITY: return "KVQ_ECAPACITY";
+    case KVQ_ENOMEM: return "KVQ_ENOMEM";
+    case KVQ_ECUDA: return "KVQ_ECUDA";
+  }
+  return "KVQ_UNKNOWN";
+}
+
+int64_t kvq_page_bytes(kvq_pair pair, int head_dim) {
+  if (!valid_pair(pair) || (head_dim != 64 && head_dim != 128)) return 0;
+  return kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim);
+}
+
+double kvq_equiv_bits(const kvq_pair* map, int n_layers) {
+  if (!map || n_layers <= 0) return -1.0;
+  double sum = 0.0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (!valid_pair(map[l])) return -1.0;
+    sum += 0.5 * ((double)map[l].k_bits + (double)map[l].v_bits);
+  }
+  return sum / n_layers;
+}
+
+size_t kvq_cache_pool_bytes(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_heads,
+                            int head_dim, int max_batch, int64_t max_tokens) {
+  Geometry g;
+  std::string why;
+  if (!make_geometry(map, n_layers, n_q_heads, n_kv_heads, head_dim, max_batch, max_tokens, g, why)) return 0;
+  return g.total;
+}
+
+kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_heads,
+                            int head_dim, int max_batch, int64_t max_tokens, void* device_pool,
+                            size_t pool_bytes, kvq_cache** out) {
+  if (!out) return fail(KVQ_EINVAL, "out is null");
+  *out = nullptr;
+  Geometry g;
+  std::string why;
+  if (!make_geometry(map, n_layers, n_q_heads, n_kv_heads, head_dim, max_batch, max_tokens, g, why))
+    return fail(KVQ_EINVAL, why);
+  if (device_pool && (reinterpret_cast<uintptr_t>(device_pool) % kAlign) != 0)
+    return fail(KVQ_EINVAL, "device_pool must be 256-byte aligned");
+  if (device_pool && pool_bytes < g.total)
+    return fail(KVQ_ENOMEM, "device_pool is smaller than kvq_cache_pool_bytes()");
+
+  kvq_cache* c = new kvq_cache();
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e != cudaSuccess) { delete c; return cuda_fail(e, "cudaGetDevice"); }
+  cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
+  c->n_layers = n_layers;
+  c->n_q_heads = n_q_heads;
+  c->n_kv_heads = n_kv_heads;
+  c->head_dim = head_dim;
+  c->max_batch = max_batch;
+  c->max_tokens = max_tokens;
+  c->max_pages = g.max_pages;
+  c->partial_slots = g.partial_slots;
+
+  if (device_pool) {
+    c->pool = device_pool;
+    c->pool_bytes = pool_bytes;
+  } else {
+    e = cudaMalloc(&c->pool, g.total);
+    if (e != cudaSuccess) {
+      delete c;
+      cudaGetLastError();
+      return fail(KVQ_ENOMEM, std::string("cudaMalloc of the cache pool failed: ") + cudaGetErrorString(e));
+    }
+    c->owns_pool = true;
+    c->pool_bytes = g.total;
+  }
+  uint8_t* p = static_cast<uint8_t*>(c->pool);
+  c->layers.resize(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    kvq::LayerState& L = c->layers[l];
+    L.kb = map[l].k_bits;
+    L.vb = map[l].v_bits;
+    L.page_bytes = kvq::page_bytes_of(L.kb, L.vb, head_dim);
+    L.pages = p;
+    p += g.page_region[l];
+    L.window = reinterpret_cast<__nv_bfloat16*>(p);
+    p += g.window_region[l];
+    L.len = reinterpret_cast<int32_t*>(p);
+    p += g.len_region;
+    L.host_len.assign(max_batch, 0);
+  }
+  c->partials = reinterpret_cast<float*>(p);
+  p += g.partial_region;
+  c->merge_ctr = reinterpret_cast<int32_t*>(p);
+  p += g.merge_region;
+  c->append_ctr = reinterpret_cast<int32_t*>(p);
+  p += g.append_region;
+  c->plan_dev = reinterpret_cast<int32_t*>(p);
+  p += g.plan_region;
+
+  e = cudaMallocHost(&c->plan_host, (size_t)max_batch * 4 * sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->plan_done, cudaEventDisableTiming);
+  // lengths and counters start at zero; pages and windows need no initialisation
+  for (int l = 0; l < n_layers && e == cudaSuccess; ++l)
+    e = cudaMemset(c->layers[l].len, 0, (size_t)max_batch * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->merge_ctr, 0, (size_t)max_batch * n_kv_heads * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->append_ctr, 0, (size_t)max_batch * 4);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    kvq_status st = cuda_fail(e, "cache initialisation");
+    kvq_cache_destroy(c);
+    return st;
+  }
+  *out = c;
+  return KVQ_OK;
+}
+
+void kvq_cache_destroy(kvq_cache* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  if (c->plan_done) cudaEventDestroy(c->plan_done);
+  if (c->plan_host) cudaFreeHost(c->plan_host);
+  if (c->owns_pool && c->pool) cudaFree(c->pool);
+  delete c;
+}
+
+kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
+  if (!c) return fail(KVQ_EINVAL, "cache is null");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (auto& L : c->layers) {
+    cudaError_t e = cudaMemsetAsync(L.len, 0, (size_t)c->max_batch * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    std::fill(L.host_len.begin(), L.host_len.end(), 0);
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_split_pages(kvq_cache* c, int pages_per_split) {
+  if (!c) return fail(KVQ_EINVAL, "cache is null");
+  if (pages_per_split < 0) return fail(KVQ_EINVAL, "pages_per_split must be >= 0");
+  c->split_pages = pages_per_split;
+  return KVQ_OK;
+}
+
+kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq_dtype dtype,
+                      const int32_t* n_new, int batch, void* stream) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (dtype != KVQ_BF16 && dtype != KVQ_F32) return fail(KVQ_EINVAL, "dtype must be KVQ_BF16 or KVQ_F32");
+  if (!n_new) return fail(KVQ_EINVAL, "n_new is null");
+  if (batch <= 0) return fail(KVQ_EINVAL, "batch must be positive");
+  if (batch > c->max_batch) return fail(KVQ_ECAPACITY, "batch exceeds max_batch");
+  kvq::LayerState& L = c->layers[layer];
+  int64_t total = 0;
+  bool all_one = true;
+  int max_items = 1;
+  for (int b = 0; b < batch; ++b) {
+    if (n_new[b] < 0) return fail(KVQ_EINVAL, "n_new entries must be >= 0");
+    if (L.host_len[b] + n_new[b] > c->max_tokens)
+      return fail(KVQ_ECAPACITY, "append would exceed max_tokens for sequence " + std::to_string(b));
+    total += n_new[b];
+    all_one = all_one && (n_new[b] == 1);
+    int64_t T0 = L.host_len[b], T1 = T0 + n_new[b];
+    max_items = (int)std::max<int64_t>(max_items, T1 / kvq::kPageTokens - T0 / kvq::kPageTokens);
+  }
+  if (total == 0) return KVQ_OK;
+  if (!K || !V) return fail(KVQ_EINVAL, "K or V is null");
+  if (!aligned16(K) || !aligned16(V)) return fail(KVQ_EINVAL, "K and V must be 16-byte aligned");
+  if (total > INT32_MAX) return fail(KVQ_EINVAL, "too many tokens in one call");
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kvq::AppendParams p{};
+  p.pages = L.pages;
+  p.window = L.window;
+  p.len = L.len;
+  p.ctr = c->append_ctr;
+  p.K = K;
+  p.V = V;
+  p.page_bytes = L.page_bytes;
+  p.max_pages = (int)c->max_pages;
+  p.n_kv_heads = c->n_kv_heads;
+  p.plan = nullptr;
+  if (!all_one) {
+    // multi-token append: per-sequence plan (start, count, row offset, items)
+    if (c->plan_pending) {
+      cudaError_t e = cudaEventSynchronize(c->plan_done);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    }
+    int64_t off = 0;
+    for (int b = 0; b < batch; ++b) {
+      int64_t T0 = L.host_len[b], T1 = T0 + n_new[b];
+      c->plan_host[4 * b + 0] = (int32_t)T0;
+      c->plan_host[4 * b + 1] = n_new[b];
+      c->plan_host[4 * b + 2] = (int32_t)off;
+      c->plan_host[4 * b + 3] = (int32_t)std::max<int64_t>(1, T1 / kvq::kPageTokens - T0 / kvq::kPageTokens);
+      off += n_new[b];
+    }
+    cudaError_t e = cudaMemcpyAsync(c->plan_dev, c->plan_host, (size_t)batch * 16, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(plan)");
+    e = cudaEventRecord(c->plan_done, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    c->plan_pending = true;
+    p.plan = c->plan_dev;
+  }
+  dim3 grid(all_one ? 1 : max_items, c->n_kv_heads, batch);
+  cudaError_t e = kvq::launch_append(L.kb, L.vb, c->head_dim, dtype, p, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+  c->launches += 1;
+  for (int b = 0; b < batch; ++b) L.host_len[b] += n_new[b];
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, float* out, void* stream) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (batch <= 0 || batch > c->max_batch) return fail(KVQ_EINVAL, "batch must be in [1, max_batch]");
+  if (!Q || !out) return fail(KVQ_EINVAL, "Q or out is null");
+  if (!aligned16(Q) || !aligned16(out)) return fail(KVQ_EINVAL, "Q and out must be 16-byte aligned");
+  const kvq::LayerState& L = c->layers[layer];
+  int64_t total_pages = 0, max_p = 0;
+  for (int b = 0; b < batch; ++b) {
+    int64_t P = L.host_len[b] / kvq::kPageTokens;
+    total_pages += P;
+    max_p = std::max(max_p, P);
+  }
+  total_pages *= c->n_kv_heads;
+  int chunk = c->split_pages > 0 ? c->split_pages : choose_chunk(c, total_pages, max_p, batch);
+  int64_t stride = c->partial_slots / ((int64_t)batch * c->n_kv_heads);
+  if (stride < 1) return fail(KVQ_EINVAL, "batch too large for the split-K buffer");
+  // never more splits than the partial buffer holds
+  chunk = (int)std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
+  int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
+
+  kvq::DecodeParams p{};
+  p.pages = L.pages;
+  p.window = L.window;
+  p.len = L.len;
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.out = out;
+  p.partials = c->partials;
+  p.ctr = c->merge_ctr;
+  p.page_bytes = L.page_bytes;
+  p.max_pages = (int)c->max_pages;
+  p.n_kv_heads = c->n_kv_heads;
+  p.gqa = c->n_q_heads / c->n_kv_heads;
+  p.chunk = chunk;
+  p.splits_stride = (int)stride;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
+  dim3 grid(splits, c->n_kv_heads, batch);
+  cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  c->launches += 1;
+  return KVQ_OK;
+}
+
+int64_t kvq_seq_len(const kvq_cache* c, int layer, int seq) {
+  if (!c || layer < 0 || layer >= c->n_layers || seq < 0 || seq >= c->max_batch) return -1;
+  return c->layers[layer].host_len[seq];
+}
+
+int64_t kvq_bytes(const kvq_cache* c, int layer, int batch, int include_metadata) {
+  if (!c || layer < 0 || layer >= c->n_layers || batch <= 0 || batch > c->max_batch) return -1;
+  const kvq::LayerState& L = c->layers[layer];
+  const int D = c->head_dim;
+  int64_t total = 0;
+  for (int b = 0; b < batch; ++b) {
+    int64_t T = L.host_len[b], P = T / kvq::kPageTokens, W = T % kvq::kPageTokens;
+    int64_t codes = kvq::code_block_bytes(L.kb, D) + kvq::code_block_bytes(L.vb, D);
+    total += P * (include_metadata ? L.page_bytes : codes);
+    if (include_metadata) total += W * D * 2 * 2;
+  }
+  return total * c->n_kv_heads;
+}
+
+int64_t kvq_export_bytes(const kvq_cache* c, int layer, int batch) {
+  if (!c || layer < 0 || layer >= c->n_layers || batch <= 0 || batch > c->max_batch) return -1;
+  const kvq::LayerState& L = c->layers[layer];
+  int64_t total = 0;
+  for (int b = 0; b < batch; ++b) {
+    int64_t T = L.host_len[b];
+    total += (T / kvq::kPageTokens) * L.page_bytes + (T % kvq::kPageTokens) * c->head_dim * 2 * 2;
+  }
+  return total * c->n_kv_heads;
+}
+
+kvq_status kvq_export_layer(const kvq_cache* c, int layer, int batch, void* host_dst, size_t bytes) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  int64_t need = kvq_export_bytes(c, layer, batch);
+  if (need < 0) return fail(KVQ_EINVAL, "bad batch");
+  if (!host_dst || bytes < (size_t)need) return fail(KVQ_EINVAL, "host_dst is null or too small");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  const kvq::LayerState& L = c->layers[layer];
+  const int D = c->head_dim, H = c->n_kv_heads;
+  uint8_t* dst = static_cast<uint8_t*>(host_dst);
+  for (int b = 0; b < batch; ++b)
+    for (int h = 0; h < H; ++h) {
+      int64_t T = L.host_len[b], P = T / kvq::kPageTokens, W = T % kvq::kPageTokens;
+      const uint8_t* pg = L.pages + ((int64_t)(b * H + h) * c->max_pages) * L.page_bytes;
+      if (P) {
+        e = cudaMemcpy(dst, pg, (size_t)(P * L.page_bytes), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(pages)");
+        dst += P * L.page_bytes;
+      }
+      const __nv_bfloat16* win = L.window + ((int64_t)(b * H + h) * 2) * kvq::kPageTokens * D;
+      if (W) {
+        e = cudaMemcpy(dst, win, (size_t)(W * D * 2), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(window K)");
+        dst += W * D * 2;
+        e = cudaMemcpy(dst, win + kvq::kPageTokens * D, (size_t)(W * D * 2), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(window V)");
+        dst += W * D * 2;
+      }
+    }
+  return KVQ_OK;
+}
+
+kvq_status kvq_sync(kvq_cache* c) {
+  if (!c) return fail(KVQ_EINVAL, "cache is null");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetLastError");
+  return KVQ_OK;
+}
+
+int64_t kvq_launch_count(const kvq_cache* c) { return c ? c->launches : -1; }
+
+}  // extern "C"

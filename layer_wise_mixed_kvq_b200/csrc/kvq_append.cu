@@ -1,0 +1,325 @@
+// kvq_append.cu -- append new tokens to a layer's cache: bf16 window, and on
+// every 32nd token a quantize + bit-pack flush into the next page.
+//
+// KVTuner OpenReview rebuttal, "Computational cost": only the newly generated
+// keys and values are quantized online, with the layer's calibrated precision
+// pair. Keys are quantized per channel and values per token, both asymmetric
+// (llms-explorer facts page; rebuttal "key per-channel-asym and value
+// per-token-asym"). The group size (32 tokens) and the fp16 scale/zero format
+// are this library's choices.
+//
+// Grid (items, n_kv_heads, batch), 128 threads. Work item i of (b, h) quantizes
+// group floor(T0/32) + i when that group completes during this call; item 0
+// also rewrites the window afterwards (it is the only item reading old window
+// tokens). With no completed group, item 0 only writes the window.
+//
+// Quantizer (bit-exact contract with the CPU oracle; every fp32 step is a
+// single IEEE operation, the __f*_rn intrinsics are never contracted):
+//   mn, mx = min, max (signed zeros canonicalised to +0)
+//   z = fp16_round_down(mn) clamped to >= -65504
+//   s = fp16_round_up((mx - z) / qmax) clamped to <= 65504
+//   code = s == 0 ? 0 : clamp(rint((x - z) * (1/s)), 0, qmax)
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kThreads = 128;
+
+struct QParams {
+  float z, r;
+  __half s_h, z_h;
+  bool zero_scale;
+};
+
+__device__ __forceinline__ QParams make_qparams(float mn, float mx, int qmax) {
+  QParams q;
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  float z = __half2float(__float2half_rd(mn));
+  z = fmaxf(z, -65504.0f);
+  float d = __fsub_rn(mx, z);
+  float ratio = __fdiv_rn(d, (float)qmax);
+  float s = __half2float(__float2half_ru(ratio));
+  s = fminf(s, 65504.0f);
+  q.z = z;
+  q.s_h = __float2half_rn(s);   // exact: s is an fp16 value
+  q.z_h = __float2half_rn(z);
+  q.zero_scale = (s == 0.0f);
+  q.r = q.zero_scale ? 0.0f : __fdiv_rn(1.0f, s);
+  return q;
+}
+
+__device__ __forceinline__ uint32_t quant_code(float x, const QParams& q, int qmax) {
+  if (q.zero_scale) return 0u;
+  float y = __fmul_rn(__fsub_rn(x, q.z), q.r);
+  int c = __float2int_rn(y);
+  c = c < 0 ? 0 : (c > qmax ? qmax : c);
+  return (uint32_t)c;
+}
+
+// Element e of tile f for lane l: (token, channel) it stores.
+__device__ __forceinline__ void tile_elem(int f, int lane, int e, bool is_value, int& tok, int& dim) {
+  int dt = f >> 1, tt = f & 1;
+  int g = lane >> 2, t = lane & 3;
+  int p = e >> 1, j = e & 1;
+  int row = g + 8 * (p & 1);
+  int col = 2 * t + j + 8 * (p >> 1);
+  if (is_value) { dim = 16 * dt + row; tok = 16 * tt + col; }
+  else          { tok = 16 * tt + row; dim = 16 * dt + col; }
+}
+
+// Lane word w of lane `lane` for a block of `BITS`-bit elements read from
+// vals(tok, dim).
+template <int BITS, typename Get>
+__device__ __forceinline__ uint32_t lane_word(int lane, int w, bool is_value, Get vals) {
+  uint32_t word = 0;
+  int tok, dim;
+  if constexpr (BITS == 8) {
+    int f = w >> 1, half = w & 1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      tile_elem(f, lane, 4 * half + k, is_value, tok, dim);
+      word |= (vals(tok, dim) & 0xFFu) << (8 * k);
+    }
+  } else if constexpr (BITS == 4) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      tile_elem(w, lane, e, is_value, tok, dim);
+      word |= (vals(tok, dim) & 0xFu) << (4 * ((e >> 1) + 4 * (e & 1)));
+    }
+  } else if constexpr (BITS == 2) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        tile_elem(2 * w + u, lane, e, is_value, tok, dim);
+        word |= (vals(tok, dim) & 0x3u) << (2 * (4 * u + (e >> 1) + 8 * (e & 1)));
+      }
+  } else {  // 16-bit (bf16 bit patterns)
+    int f = w >> 2, pair = w & 3;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      tile_elem(f, lane, 2 * pair + k, is_value, tok, dim);
+      word |= (vals(tok, dim) & 0xFFFFu) << (16 * k);
+    }
+  }
+  return word;
+}
+
+// Write one code block (32 tokens x D) as lane-interleaved 16-byte vectors.
+template <int BITS, int D, typename Get>
+__device__ __forceinline__ void store_block(uint8_t* blk, bool is_value, Get vals) {
+  constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
+  for (int v = threadIdx.x; v < kVectors; v += kThreads) {
+    int lane = v & 31, vi = v >> 5;
+    uint4 q;
+    q.x = lane_word<BITS>(lane, 4 * vi + 0, is_value, vals);
+    q.y = lane_word<BITS>(lane, 4 * vi + 1, is_value, vals);
+    q.z = lane_word<BITS>(lane, 4 * vi + 2, is_value, vals);
+    q.w = lane_word<BITS>(lane, 4 * vi + 3, is_value, vals);
+    reinterpret_cast<uint4*>(blk)[v] = q;
+  }
+}
+
+template <bool F32IN>
+__device__ __forceinline__ __nv_bfloat16 load_in(const void* base, int64_t idx) {
+  if constexpr (F32IN) return __float2bfloat16_rn(reinterpret_cast<const float*>(base)[idx]);
+  else return reinterpret_cast<const __nv_bfloat16*>(base)[idx];
+}
+
+// Key scale/zero slot of channel d (inverse of the documented permutation).
+template <int D>
+__device__ __forceinline__ int kmeta_slot(int d) {
+  int dt = d >> 4, r = d & 15;
+  int j = (r & 1) + 2 * (r >> 3);
+  int t = (r & 7) >> 1;
+  return t * (D / 4) + dt * 4 + j;
+}
+
+template <int KB, int VB, int D, bool F32IN>
+__global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
+  constexpr bool kBf16Layer = (KB == 16);
+  const int b = blockIdx.z, h = blockIdx.y, item = blockIdx.x;
+  const int H = a.n_kv_heads;
+  __shared__ int s_T0;
+
+  int T0, n, items;
+  int64_t off;
+  if (a.plan) {
+    T0 = a.plan[4 * b];
+    n = a.plan[4 * b + 1];
+    off = a.plan[4 * b + 2];
+    items = a.plan[4 * b + 3];
+    if (item >= items) return;
+    if (item == 0 && h == 0 && threadIdx.x == 0) a.len[b] = T0 + n;
+  } else {
+    // One token per sequence; every CTA of sequence b reads the old length,
+    // and the last one to have read it publishes the new length.
+    if (threadIdx.x == 0) {
+      int t0 = a.len[b];
+      s_T0 = t0;
+      __threadfence();
+      if (atomicAdd(&a.ctr[b], 1) == H - 1) {
+        a.ctr[b] = 0;
+        __threadfence();
+        a.len[b] = t0 + 1;
+      }
+    }
+    __syncthreads();
+    T0 = s_T0;
+    n = 1;
+    off = b;
+    items = 1;
+  }
+  if (n == 0) return;
+  const int T1 = T0 + n;
+  const int g0 = T0 / kPageTokens;
+  const int ng = T1 / kPageTokens - g0;
+
+  __nv_bfloat16* win = a.window + ((int64_t)(b * H + h) * 2) * kPageTokens * D;
+
+  if (ng > 0) {
+    const int g = g0 + item;
+    uint8_t* page = a.pages + ((int64_t)(b * H + h) * a.max_pages + g) * a.page_bytes;
+    if constexpr (kBf16Layer) {
+      __shared__ uint16_t sv[2][kPageTokens][D];
+      for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
+        int t = idx / D, d = idx % D;
+        int tau = g * kPageTokens + t;
+        __nv_bfloat16 kx, vx;
+        if (tau < T0) {
+          kx = win[(0 * kPageTokens + (tau % kPageTokens)) * D + d];
+          vx = win[(1 * kPageTokens + (tau % kPageTokens)) * D + d];
+        } else {
+          int64_t row = off + (tau - T0);
+          kx = load_in<F32IN>(a.K, (row * H + h) * D + d);
+          vx = load_in<F32IN>(a.V, (row * H + h) * D + d);
+        }
+        sv[0][t][d] = __bfloat16_as_ushort(kx);
+        sv[1][t][d] = __bfloat16_as_ushort(vx);
+      }
+      __syncthreads();
+      store_block<16, D>(page, false, [&](int tok, int dim) { return (uint32_t)sv[0][tok][dim]; });
+      store_block<16, D>(page + code_block_bytes(16, D), true,
+                         [&](int tok, int dim) { return (uint32_t)sv[1][tok][dim]; });
+    } else {
+      __shared__ float xs[2][kPageTokens][D + 1];
+      __shared__ uint8_t cs[2][kPageTokens][D];
+      for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
+        int t = idx / D, d = idx % D;
+        int tau = g * kPageTokens + t;
+        __nv_bfloat16 kx, vx;
+        if (tau < T0) {
+          kx = win[(0 * kPageTokens + (tau % kPageTokens)) * D + d];
+          vx = win[(1 * kPageTokens + (tau % kPageTokens)) * D + d];
+        } else {
+          int64_t row = off + (tau - T0);
+          kx = load_in<F32IN>(a.K, (row * H + h) * D + d);
+          vx = load_in<F32IN>(a.V, (row * H + h) * D + d);
+        }
+        xs[0][t][d] = __bfloat162float(kx);
+        xs[1][t][d] = __bfloat162float(vx);
+      }
+      __syncthreads();
+      uint8_t* vblk = page + code_block_bytes(KB, D);
+      __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
+      __half* kzero = kscale + D;
+      __half* vscale = kzero + D;
+      __half* vzero = vscale + kPageTokens;
+      // keys: one thread per channel, over the group's 32 tokens
+      for (int d = threadIdx.x; d < D; d += kThreads) {
+        constexpr int qmax = (1 << KB) - 1;
+        float mn = xs[0][0][d], mx = mn;
+#pragma unroll 8
+        for (int t = 1; t < kPageTokens; ++t) {
+          float x = xs[0][t][d];
+          mn = fminf(mn, x);
+          mx = fmaxf(mx, x);
+        }
+        QParams q = make_qparams(mn, mx, qmax);
+#pragma unroll 8
+        for (int t = 0; t < kPageTokens; ++t) cs[0][t][d] = (uint8_t)quant_code(xs[0][t][d], q, qmax);
+        int slot = kmeta_slot<D>(d);
+        kscale[slot] = q.s_h;
+        kzero[slot] = q.z_h;
+      }
+      // values: one warp per token, over the head dimension
+      {
+        constexpr int qmax = (1 << VB) - 1;
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        for (int t = warp; t < kPageTokens; t += kThreads / 32) {
+          float mn = xs[1][t][lane], mx = mn;
+#pragma unroll
+          for (int k = 1; k < D / 32; ++k) {
+            float x = xs[1][t][lane + 32 * k];
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          QParams q = make_qparams(mn, mx, qmax);
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k)
+            cs[1][t][lane + 32 * k] = (uint8_t)quant_code(xs[1][t][lane + 32 * k], q, qmax);
+          if (lane == 0) {
+            vscale[t] = q.s_h;
+            vzero[t] = q.z_h;
+          }
+        }
+      }
+      __syncthreads();
+      store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
+      store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
+    }
+  }
+
+  if (item == 0) {
+    __syncthreads();  // the group above may have read old window slots
+    const int wstart = (T1 / kPageTokens) * kPageTokens;
+    const int from = wstart > T0 ? wstart : T0;
+    const int cnt = T1 - from;
+    for (int idx = threadIdx.x; idx < cnt * D; idx += kThreads) {
+      int i = idx / D, d = idx % D;
+      int tau = from + i;
+      int64_t row = off + (tau - T0);
+      int slot = tau % kPageTokens;
+      win[(0 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.K, (row * H + h) * D + d);
+      win[(1 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.V, (row * H + h) * D + d);
+    }
+  }
+}
+
+template <int KB, int VB, int D>
+cudaError_t launch3(kvq_dtype dt, const AppendParams& p, dim3 grid, cudaStream_t s) {
+  if (dt == KVQ_F32) append_kernel<KB, VB, D, true><<<grid, kThreads, 0, s>>>(p);
+  else append_kernel<KB, VB, D, false><<<grid, kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(int kb, int vb, kvq_dtype dt, const AppendParams& p, dim3 grid, cudaStream_t s) {
+#define KVQ_PAIR(K_, V_) \
+  if (kb == K_ && vb == V_) return launch3<K_, V_, D>(dt, p, grid, s);
+  KVQ_PAIR(2, 2) KVQ_PAIR(2, 4) KVQ_PAIR(2, 8)
+  KVQ_PAIR(4, 2) KVQ_PAIR(4, 4) KVQ_PAIR(4, 8)
+  KVQ_PAIR(8, 2) KVQ_PAIR(8, 4) KVQ_PAIR(8, 8)
+  KVQ_PAIR(16, 16)
+#undef KVQ_PAIR
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
+                          cudaStream_t s) {
+  if (D == 64) return launch_d<64>(kb, vb, dtype, p, grid, s);
+  if (D == 128) return launch_d<128>(kb, vb, dtype, p, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kvq

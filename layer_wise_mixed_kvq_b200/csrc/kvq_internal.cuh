@@ -1,0 +1,106 @@
+// kvq_internal.cuh -- internal types of libkvq (not part of the C ABI).
+//
+// Device memory of one layer (all regions 256-byte aligned):
+//   pages : [max_batch][n_kv_heads][max_pages] x page_bytes   (full 32-token pages)
+//   window: [max_batch][n_kv_heads][2][32][head_dim] bf16      (keys, values; slot = token % 32)
+//   len   : [max_batch] int32                                  (tokens held per sequence)
+// Cache-wide scratch:
+//   partials: [slots][G][head_dim + 2] fp32 split-K partial (acc, m, l), slot =
+//             (b * n_kv_heads + h) * splits_stride + split
+//   merge_ctr: [max_batch * n_kv_heads] int32, zero between launches
+//   append_ctr: [max_batch] int32, zero between launches
+//   plan  : [4 * max_batch] int32 (T0, n, row offset, work items) for multi-token appends
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kPageTokens = 32;   // key group size = tokens per page = window capacity
+constexpr int kMaxBatch = 1024;
+constexpr int kMaxGqa = 8;
+
+__host__ __device__ constexpr int64_t code_block_bytes(int bits, int D) { return 4LL * D * bits; }
+
+__host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D) {
+  return code_block_bytes(kb, D) + code_block_bytes(vb, D) + (kb == 16 ? 0 : 4LL * D + 128);
+}
+
+struct LayerState {
+  int kb = 0, vb = 0;
+  int64_t page_bytes = 0;
+  uint8_t* pages = nullptr;
+  __nv_bfloat16* window = nullptr;
+  int32_t* len = nullptr;
+  std::vector<int64_t> host_len;
+};
+
+// Parameters of the append kernel.
+struct AppendParams {
+  uint8_t* pages;
+  __nv_bfloat16* window;
+  int32_t* len;
+  int32_t* ctr;          // append_ctr
+  const void* K;
+  const void* V;
+  const int32_t* plan;   // nullptr: one token per sequence, lengths read from `len`
+  int64_t page_bytes;
+  int max_pages;
+  int n_kv_heads;
+};
+
+// Parameters of the decode attention kernel.
+struct DecodeParams {
+  const uint8_t* pages;
+  const __nv_bfloat16* window;
+  const int32_t* len;
+  const __nv_bfloat16* Q;
+  float* out;
+  float* partials;
+  int32_t* ctr;          // merge_ctr
+  int64_t page_bytes;
+  int max_pages;
+  int n_kv_heads;
+  int gqa;               // query heads per KV head
+  int chunk;             // pages per split
+  int splits_stride;     // partial slots per (b, h)
+  float scale_log2;      // log2(e) / sqrt(head_dim)
+};
+
+// Launchers (defined per kernel file); return the CUDA launch error.
+cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
+                          cudaStream_t s);
+cudaError_t launch_decode_simt(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+// Layer-map dispatcher: the kernel instance for a layer's pair.
+cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+
+}  // namespace kvq
+
+struct kvq_cache {
+  int device = 0;
+  int n_layers = 0, n_q_heads = 0, n_kv_heads = 0, head_dim = 0, max_batch = 0;
+  int64_t max_tokens = 0, max_pages = 0;
+  int sm_count = 148;
+  std::vector<kvq::LayerState> layers;
+  float* partials = nullptr;
+  int64_t partial_slots = 0;
+  int32_t* merge_ctr = nullptr;
+  int32_t* append_ctr = nullptr;
+  int32_t* plan_dev = nullptr;
+  int32_t* plan_host = nullptr;      // pinned
+  cudaEvent_t plan_done = nullptr;
+  bool plan_pending = false;
+  void* pool = nullptr;
+  size_t pool_bytes = 0;
+  bool owns_pool = false;
+  int split_pages = 0;
+  int64_t launches = 0;
+};
