@@ -157,6 +157,36 @@ kvq_status kvq_append(kvq_cache* cache, int layer, const void* K, const void* V,
 kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch, float* out,
                            void* stream);
 
+/* kvq_decode_attn for callers that cannot allocate device memory. The KVTuner
+ * pages have no counterpart of this call; it exists for programs whose device
+ * memory belongs to someone else (a serving engine that reserves all of HBM for
+ * its own arena, a plug-in inside another runtime, a latency-critical loop that
+ * must not call cudaMalloc/cudaFree). Such callers cannot use kvq_cache_create,
+ * which allocates, so they keep one layer in their own buffers, in the storage
+ * format described above:
+ *   pages:   device, [batch][n_kv_heads][max_pages] pages of
+ *            kvq_page_bytes(pair, head_dim) bytes, 16-byte aligned;
+ *   window:  device, bf16 [batch][n_kv_heads][2][32][head_dim] (keys, values);
+ *   seq_len: device int32 [batch]: tokens of each sequence; every entry must be
+ *            in [0, max_seq_len] (entries beyond it read outside `pages`);
+ *   max_seq_len: host bound on seq_len, with max_seq_len/32 <= max_pages;
+ *   Q, out:  as for kvq_decode_attn.
+ * The result is that of kvq_decode_attn on the same state, up to rounding
+ * order. This call allocates nothing: its split-K scratch is a fixed 16 MiB
+ * static device array that every GPU loading the library holds until the
+ * process exits. The first call on a device looks up that array's address
+ * (cudaGetSymbolAddress), so make the first call on each device before any
+ * stream capture. Every call shares the array and clears the part that must
+ * start at zero; calls whose kernels overlap on the GPU race on it, so
+ * serialise them. KVQ_ECAPACITY when batch * n_kv_heads * (n_q_heads /
+ * n_kv_heads) * (head_dim + 2) * 4 bytes of split-K state (plus 4 bytes of
+ * counter per sequence-head) exceed 16 MiB; KVQ_EINVAL for bad arguments.
+ * Nothing is launched on error. */
+kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n_q_heads, int n_kv_heads,
+                                   const void* pages, int64_t max_pages, const void* window,
+                                   const int32_t* seq_len, int64_t max_seq_len, const void* Q,
+                                   int batch, float* out, void* stream);
+
 /* Pages per split-K CTA for kvq_decode_attn: 0 = automatic (default). Changing
  * it changes only the rounding order of the result. */
 kvq_status kvq_set_split_pages(kvq_cache* cache, int pages_per_split);

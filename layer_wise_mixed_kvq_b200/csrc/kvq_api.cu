@@ -112,6 +112,8 @@ int choose_chunk(const kvq_cache* c, int64_t total_pages, int64_t max_p, int bat
 }  // namespace
 
 namespace kvq {
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
 cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s) {
   return launch_decode_simt(kb, vb, D, p, grid, s);
 }

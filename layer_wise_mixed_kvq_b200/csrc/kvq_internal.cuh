@@ -79,6 +79,8 @@ struct DecodeParams {
 cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
                           cudaStream_t s);
 cudaError_t launch_decode_simt(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+// Message returned by kvq_last_error() on this thread.
+void set_last_error(const std::string& msg);
 // Layer-map dispatcher: the kernel instance for a layer's pair.
 cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
 

@@ -20,7 +20,7 @@ KVQ_BF16, KVQ_F32 = 0, 1
 #: every symbol the C header declares
 EXPORTS = (
     "kvq_page_bytes", "kvq_equiv_bits", "kvq_cache_pool_bytes", "kvq_cache_create", "kvq_cache_destroy",
-    "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
+    "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
     "kvq_export_bytes", "kvq_export_layer", "kvq_sync", "kvq_launch_count", "kvq_last_error",
     "kvq_status_string",
 )
@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
         "kvq_cache_reset": (c.c_int, [P, P]),
         "kvq_append": (c.c_int, [P, c.c_int, P, P, c.c_int, P, c.c_int, P]),
         "kvq_decode_attn": (c.c_int, [P, c.c_int, P, c.c_int, P, P]),
+        "kvq_decode_attn_noalloc": (c.c_int, [kvq_pair, c.c_int, c.c_int, c.c_int, P, c.c_int64, P, P, c.c_int64, P,
+                                              c.c_int, P, P]),
         "kvq_set_split_pages": (c.c_int, [P, c.c_int]),
         "kvq_seq_len": (c.c_int64, [P, c.c_int, c.c_int]),
         "kvq_bytes": (c.c_int64, [P, c.c_int, c.c_int, c.c_int]),
@@ -165,6 +167,22 @@ def kvq_decode_attn(cache, layer, Q, out, stream=None) -> None:
         raise ValueError("Q must be bfloat16 and out float32")
     _check(lib.kvq_decode_attn(ctypes.c_void_p(cache), int(layer), _dev_ptr(Q), int(Q.shape[0]), _dev_ptr(out),
                                _stream(stream)))
+
+
+def kvq_decode_attn_noalloc(pair, head_dim, n_q_heads, n_kv_heads, pages, max_pages, window, seq_len,
+                            max_seq_len, Q, out, stream=None) -> None:
+    """Decode attention over caller-owned layer buffers; the library allocates nothing.
+
+    pages: uint8 CUDA [batch, n_kv_heads, max_pages, page_bytes]; window: bf16 CUDA
+    [batch, n_kv_heads, 2, 32, head_dim]; seq_len: int32 CUDA [batch]; Q bf16 / out fp32 CUDA.
+    """
+    import torch
+    if Q.dtype != torch.bfloat16 or out.dtype != torch.float32 or seq_len.dtype != torch.int32:
+        raise ValueError("Q must be bfloat16, out float32 and seq_len int32")
+    _check(lib.kvq_decode_attn_noalloc(kvq_pair(int(pair[0]), int(pair[1])), int(head_dim), int(n_q_heads),
+                                       int(n_kv_heads), _dev_ptr(pages), int(max_pages), _dev_ptr(window),
+                                       _dev_ptr(seq_len), int(max_seq_len), _dev_ptr(Q), int(Q.shape[0]),
+                                       _dev_ptr(out), _stream(stream)))
 
 
 def kvq_set_split_pages(cache, pages_per_split: int) -> None:
