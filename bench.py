@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="llama_k4v4", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profile a truncated stack (first N layers); 0 = the workload's full stack")
     return ap.parse_args()
 
 
@@ -365,6 +367,9 @@ def main():
         print("warmup must be >= 3", file=sys.stderr)
         return 2
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        import dataclasses
+        w = dataclasses.replace(w, layer_map=w.layer_map[:args.layers])
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 
@@ -41,7 +42,7 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Geometry {
   int64_t max_pages = 0;
   std::vector<size_t> page_region, window_region;
-  size_t len_region = 0, partial_region = 0, merge_region = 0, append_region = 0, plan_region = 0;
+  size_t len_region = 0, partial_region = 0, merge_region = 0, append_region = 0, plan_region = 0, err_region = 0;
   int64_t partial_slots = 0;
   size_t total = 0;
 };
@@ -86,7 +87,8 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
   g.merge_region = round_up((size_t)max_batch * n_kv_heads * 4);
   g.append_region = round_up((size_t)max_batch * 4);
   g.plan_region = round_up((size_t)max_batch * 4 * 4);
-  total += g.partial_region + g.merge_region + g.append_region + g.plan_region;
+  g.err_region = round_up(4);
+  total += g.partial_region + g.merge_region + g.append_region + g.plan_region + g.err_region;
   g.total = total;
   return true;
 }
@@ -97,25 +99,27 @@ kvq_status check_cache(const kvq_cache* c, int layer) {
   return KVQ_OK;
 }
 
-// Pages per split-K CTA: enough CTAs to cover the GPU about 4 times over, at
-// least 2 pages per CTA, and no more splits per (b, h) than the partial buffer
-// holds.
-int choose_chunk(const kvq_cache* c, int64_t total_pages, int64_t max_p, int batch) {
-  int64_t target_ctas = (int64_t)c->sm_count * 4;
-  int64_t chunk = std::max<int64_t>(2, (total_pages + target_ctas - 1) / std::max<int64_t>(target_ctas, 1));
-  int64_t stride = c->partial_slots / ((int64_t)batch * c->n_kv_heads);
-  if (stride < 1) stride = 1;
-  chunk = std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
-  return (int)std::max<int64_t>(chunk, 1);
-}
-
 }  // namespace
 
 namespace kvq {
 void set_last_error(const std::string& msg) { g_last_error = msg; }
 
+// The tensor-core kernel serves every pair; KVQ_DECODE_KERNEL=simt selects the
+// CUDA-core kernel instead (a second, independent implementation for checks).
 cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  return launch_decode_simt(kb, vb, D, p, grid, s);
+  static const bool simt = [] {
+    const char* e = std::getenv("KVQ_DECODE_KERNEL");
+    return e && std::string(e) == "simt";
+  }();
+  return simt ? launch_decode_simt(kb, vb, D, p, grid, s) : launch_decode_mma(kb, vb, D, p, grid, s);
+}
+
+int choose_chunk(int sm_count, int64_t total_pages, int64_t max_p, int64_t stride) {
+  const int64_t target_ctas = (int64_t)sm_count * 3;
+  int64_t chunk = std::max<int64_t>(8, (total_pages + target_ctas - 1) / target_ctas);
+  if (stride < 1) stride = 1;
+  chunk = std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
+  return (int)chunk;
 }
 }  // namespace kvq
 
@@ -220,6 +224,8 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
   p += g.append_region;
   c->plan_dev = reinterpret_cast<int32_t*>(p);
   p += g.plan_region;
+  c->err = reinterpret_cast<int32_t*>(p);
+  p += g.err_region;
 
   e = cudaMallocHost(&c->plan_host, (size_t)max_batch * 4 * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->plan_done, cudaEventDisableTiming);
@@ -228,6 +234,7 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     e = cudaMemset(c->layers[l].len, 0, (size_t)max_batch * 4);
   if (e == cudaSuccess) e = cudaMemset(c->merge_ctr, 0, (size_t)max_batch * n_kv_heads * 4);
   if (e == cudaSuccess) e = cudaMemset(c->append_ctr, 0, (size_t)max_batch * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->err, 0, 4);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     kvq_status st = cuda_fail(e, "cache initialisation");
@@ -347,9 +354,9 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
     max_p = std::max(max_p, P);
   }
   total_pages *= c->n_kv_heads;
-  int chunk = c->split_pages > 0 ? c->split_pages : choose_chunk(c, total_pages, max_p, batch);
   int64_t stride = c->partial_slots / ((int64_t)batch * c->n_kv_heads);
   if (stride < 1) return fail(KVQ_EINVAL, "batch too large for the split-K buffer");
+  int chunk = c->split_pages > 0 ? c->split_pages : kvq::choose_chunk(c->sm_count, total_pages, max_p, stride);
   // never more splits than the partial buffer holds
   chunk = (int)std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
   int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
@@ -369,6 +376,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.chunk = chunk;
   p.splits_stride = (int)stride;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
+  p.err = c->err;
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
@@ -445,6 +453,13 @@ kvq_status kvq_sync(kvq_cache* c) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetLastError");
+  int32_t flag = 0;
+  e = cudaMemcpy(&flag, c->err, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(err)");
+  if (flag) {
+    cudaMemset(c->err, 0, 4);
+    return fail(KVQ_ECUDA, "decode attention: a page copy did not complete within its wait limit");
+  }
   return KVQ_OK;
 }
 

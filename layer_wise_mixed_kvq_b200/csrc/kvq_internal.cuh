@@ -73,12 +73,17 @@ struct DecodeParams {
   int chunk;             // pages per split
   int splits_stride;     // partial slots per (b, h)
   float scale_log2;      // log2(e) / sqrt(head_dim)
+  int* err;              // set to nonzero if a bounded wait gave up (may be null)
 };
 
 // Launchers (defined per kernel file); return the CUDA launch error.
 cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
                           cudaStream_t s);
 cudaError_t launch_decode_simt(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+// Pages per split-K CTA for a layer-step: about 3 CTAs per SM, at least 8 pages
+// (2 per warp) per CTA, and no more than `stride` splits per (sequence, head).
+int choose_chunk(int sm_count, int64_t total_pages, int64_t max_pages_per_seq, int64_t stride);
 // Message returned by kvq_last_error() on this thread.
 void set_last_error(const std::string& msg);
 // Layer-map dispatcher: the kernel instance for a layer's pair.
@@ -96,6 +101,7 @@ struct kvq_cache {
   int64_t partial_slots = 0;
   int32_t* merge_ctr = nullptr;
   int32_t* append_ctr = nullptr;
+  int32_t* err = nullptr;            // device flag raised by a decode wait that gave up
   int32_t* plan_dev = nullptr;
   int32_t* plan_host = nullptr;      // pinned
   cudaEvent_t plan_done = nullptr;

@@ -102,9 +102,7 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t max_p = max_seq_len / kvq::kPageTokens;
-  const int64_t target = (int64_t)sms * 4;
-  int64_t chunk = std::max<int64_t>(2, (max_p * pairs + target - 1) / target);
-  chunk = std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
+  const int64_t chunk = kvq::choose_chunk(sms, max_p * pairs, max_p, stride);
   const int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);

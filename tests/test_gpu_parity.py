@@ -262,3 +262,20 @@ def test_full_llama_mixed_decode_run(kvq, oracle, layer):
 def test_full_ragged_long(kvq, oracle, layer):
     w = synth.WORKLOADS["ragged_long"]
     _full_layer(kvq, oracle, w, layer, synth.context_lengths(w), 2, sample_seqs=(0, 3))
+
+
+def test_simt_kernel_matches_oracle(kvq, oracle, tmp_path):
+    """The CUDA-core kernel (KVQ_DECODE_KERNEL=simt) is a second implementation;
+    run a few cases through it in a fresh process."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "import pytest\n"
+        "sys.exit(pytest.main(['-q', '-x', '-m', 'gpu', %r, '-k', "
+        "'test_append_and_decode_small or test_window_boundaries or test_split_count']))\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))), os.path.abspath(__file__))
+    env = dict(os.environ, KVQ_DECODE_KERNEL="simt")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
