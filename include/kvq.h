@@ -178,10 +178,11 @@ kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch
  * (cudaGetSymbolAddress), so make the first call on each device before any
  * stream capture. Every call shares the array and clears the part that must
  * start at zero; calls whose kernels overlap on the GPU race on it, so
- * serialise them. KVQ_ECAPACITY when batch * n_kv_heads * (n_q_heads /
- * n_kv_heads) * (head_dim + 2) * 4 bytes of split-K state (plus 4 bytes of
- * counter per sequence-head) exceed 16 MiB; KVQ_EINVAL for bad arguments.
- * Nothing is launched on error. */
+ * serialise them. The scratch holds one 4-byte merge counter per
+ * (sequence, KV head) and split-K records of (n_q_heads / n_kv_heads) *
+ * (head_dim + 2) * 4 bytes; KVQ_ECAPACITY when the counters leave no room for
+ * two records in 16 MiB; KVQ_EINVAL for bad arguments. Nothing is launched on
+ * error. */
 kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n_q_heads, int n_kv_heads,
                                    const void* pages, int64_t max_pages, const void* window,
                                    const int32_t* seq_len, int64_t max_seq_len, const void* Q,

@@ -111,7 +111,7 @@ cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 gri
     const char* e = std::getenv("KVQ_DECODE_KERNEL");
     return e && std::string(e) == "simt";
   }();
-  return simt ? launch_decode_simt(kb, vb, D, p, grid, s) : launch_decode_mma(kb, vb, D, p, grid, s);
+  return simt ? launch_decode_simt(kb, vb, D, p, grid, s) : launch_decode_mma(kb, vb, D, p, s);
 }
 
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_p, int64_t stride) {
@@ -347,13 +347,16 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   if (!Q || !out) return fail(KVQ_EINVAL, "Q or out is null");
   if (!aligned16(Q) || !aligned16(out)) return fail(KVQ_EINVAL, "Q and out must be 16-byte aligned");
   const kvq::LayerState& L = c->layers[layer];
-  int64_t total_pages = 0, max_p = 0;
+  int64_t total_pages = 0, max_p = 0, n_units = 0;
   for (int b = 0; b < batch; ++b) {
-    int64_t P = L.host_len[b] / kvq::kPageTokens;
+    int64_t T = L.host_len[b], P = T / kvq::kPageTokens;
     total_pages += P;
     max_p = std::max(max_p, P);
+    n_units += std::max<int64_t>(1, P + (T % kvq::kPageTokens ? 1 : 0));
   }
   total_pages *= c->n_kv_heads;
+  n_units *= c->n_kv_heads;
+  if (n_units > INT32_MAX) return fail(KVQ_EINVAL, "too many pages in one call");
   int64_t stride = c->partial_slots / ((int64_t)batch * c->n_kv_heads);
   if (stride < 1) return fail(KVQ_EINVAL, "batch too large for the split-K buffer");
   int chunk = c->split_pages > 0 ? c->split_pages : kvq::choose_chunk(c->sm_count, total_pages, max_p, stride);
@@ -377,6 +380,10 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.splits_stride = (int)stride;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
   p.err = c->err;
+  p.batch = batch;
+  p.n_units = (int)n_units;
+  p.max_ctas = (int)std::min<int64_t>(c->partial_slots / 2, INT32_MAX);
+  p.sm_count = c->sm_count;
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

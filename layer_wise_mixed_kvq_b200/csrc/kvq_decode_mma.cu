@@ -30,6 +30,9 @@
 // scale and the output scale (see the sigma/tau constants below).
 // bf16 layers and the bf16 window use bf16 MMAs on the raw values.
 
+#include <algorithm>
+#include <type_traits>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -141,12 +144,11 @@ struct Cfg {
   static constexpr int KS = D / 16;                       // 16-channel tiles
   static constexpr int PB = (int)page_bytes_of(KB, VB, D);
   // small pages: 3 CTAs per SM with 3-4 stages per warp; larger ones: 2 CTAs per SM
-  static constexpr int MINB = PB <= 5000 ? 3 : 2;
+  static constexpr int MINB = PB <= 5000 ? 3 : 2;      // head-row kernel (64 accumulators per lane)
+  static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;  // token-row kernel (32 accumulators per lane)
   static constexpr int RING_BUDGET = MINB == 3 ? 14336 : 24576;   // bytes of stages per warp
   static constexpr int R = (RING_BUDGET / PB) < 2 ? 2 : ((RING_BUDGET / PB) > 4 ? 4 : (RING_BUDGET / PB));
   static constexpr int STAGE = (PB + 127) / 128 * 128;
-  static constexpr int KW = D * KB / 32;                  // 32-bit words of K codes per lane
-  static constexpr int VW = D * VB / 32;
   // Power-of-two factors of the subnormal unpack (see file comment).
   //   key n-tile parity 1 (tokens 8..15 of each 16) is sigmaK times parity 0;
   //   key channels 2t+8, 2t+9 of each tile carry tauK relative to 2t, 2t+1;
@@ -163,13 +165,16 @@ struct Cfg {
   static constexpr int RING = kWarps * R * STAGE;
   static constexpr int MBAR_OFF = RING;
   static constexpr int MBAR_BYTES = (kWarps * R * 8 + 127) / 128 * 128;
-  static constexpr int WSCR_FLOATS = 4 * KSROW + 64;      // key scales, value scales, value zeros
+  static constexpr int WSCR_FLOATS = 4 * KSROW + 64 + 160;  // key scales, value scales/zeros, p' transpose tile
   static constexpr int WSCR_OFF = MBAR_OFF + MBAR_BYTES;
   static constexpr int WSCR_STRIDE = (WSCR_FLOATS * 4 + 127) / 128 * 128;
   static constexpr int QZ_OFF = WSCR_OFF + kWarps * WSCR_STRIDE;
   static constexpr int QZ_BYTES = KS * 32 * 16;
-  static constexpr int SMEM = QZ_OFF + QZ_BYTES;
-  static_assert(kWarps * kMaxGqa * D * 4 + 2 * kWarps * kMaxGqa * 4 <= RING, "merge area must fit in the ring");
+  static constexpr int MERGE_OFF = QZ_OFF + QZ_BYTES;
+  // then: merge area [kWarps][G][D] + m, l [kWarps][8] floats, unit starts [batch + 1] ints
+  static int smem_bytes(int G, int batch) {
+    return MERGE_OFF + (kWarps * G * D + 2 * kWarps * kMaxGqa) * 4 + (batch + 1) * 4;
+  }
   static_assert(PB % 16 == 0, "bulk copies need 16-byte multiples");
 };
 
@@ -496,227 +501,724 @@ __device__ __forceinline__ void load_qb(const __nv_bfloat16* qrow, bool valid, i
   }
 }
 
-// ------------------------------------------------------------------ kernel --
+// ============================================================================
+// Token-row formulation (G <= 4): MMA rows are tokens (QK) and channels (PV);
+// the 8 columns are (head c/2, part c%2) with part 0 = high f16 half and part 1
+// = low half of q' (QK) or p' (PV). Lane (g, t) keeps head t's scores for
+// tokens g, g+8, g+16, g+24 and head t's output for channels g, g+8 of every
+// 16-channel tile. 16 QK + 16 PV + 8 z-term MMAs per page.
+template <int D>
+struct TokState {
+  float o[D / 16][4];  // [channel tile]: c0/c1 = head t parts at channel g, c2/c3 at channel g+8
+  float m, l, vz;      // head t: reference max, partial sum over this lane's tokens, sum p*z
+};
+
+template <int D>
+__device__ __forceinline__ void tok_rescale_update(TokState<D>& st, float (&sc)[4], float tau) {
+  float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+  if (mx > st.m + tau) {
+    const float alpha = ex2(st.m - mx);
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st.o[j][k] *= alpha;
+    st.l *= alpha;
+    st.vz *= alpha;
+    st.m = mx;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sc[i] = ex2(sc[i] - st.m);
+    st.l += sc[i];
+  }
+}
+
+// A fragment of tile (dt, tt) from this lane's words (rows: tokens for keys,
+// channels for values; columns: channels for keys, tokens for values).
+template <int BITS>
+__device__ __forceinline__ void tile_afrag(const uint32_t (&w)[TileWords<BITS>::N], int tt, uint32_t (&a)[4]) {
+  if constexpr (BITS == 4) {
+    uint32_t x = w[tt], y = x >> 8;
+    a[0] = x & 0x000F000Fu;   // rows g,   cols 2t..     x1
+    a[1] = x & 0x00F000F0u;   // rows g+8, cols 2t..     x16
+    a[2] = y & 0x000F000Fu;   // rows g,   cols 2t+8..   x1
+    a[3] = y & 0x00F000F0u;   // rows g+8, cols 2t+8..   x16
+  } else if constexpr (BITS == 2) {
+    uint32_t x = tt ? (w[0] >> 8) : w[0];
+    a[0] = x & 0x00030003u;   // x1
+    a[1] = x & 0x000C000Cu;   // x4
+    a[2] = x & 0x00300030u;   // x16
+    a[3] = x & 0x00C000C0u;   // x64
+  } else if constexpr (BITS == 8) {
+    uint32_t x = w[2 * tt], y = w[2 * tt + 1];
+    a[0] = __byte_perm(x, 0u, 0x4140);
+    a[1] = __byte_perm(x, 0u, 0x4342);
+    a[2] = __byte_perm(y, 0u, 0x4140);
+    a[3] = __byte_perm(y, 0u, 0x4342);
+  } else {
+    a[0] = w[4 * tt + 0];
+    a[1] = w[4 * tt + 1];
+    a[2] = w[4 * tt + 2];
+    a[3] = w[4 * tt + 3];
+  }
+}
+
+// hi (part 0) or lo (part 1) f16 halves of (x0, x1) as one register.
+__device__ __forceinline__ uint32_t part_f16(float x0, float x1, float partf) {
+  __half2 h = __floats2half2_rn(x0, x1);
+  float2 f = __half22float2(h);
+  return h2_bits(__floats2half2_rn(fmaf(-partf, f.x, x0), fmaf(-partf, f.y, x1)));
+}
+
+__device__ __forceinline__ uint32_t part_bf16(float x0, float x1, float partf) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  float2 f = __bfloat1622float2(h);
+  return b2_bits(__floats2bfloat162_rn(fmaf(-partf, f.x, x0), fmaf(-partf, f.y, x1)));
+}
+
+// Transpose p' (this lane: head t, tokens g + 8i) into the PV B fragments
+// (this lane: column g = (head g/2, part g%2), tokens 2t, 2t+1, 2t+8, 2t+9 of
+// each 16-token k-step). `ptr` is a per-warp [4][40] float tile.
+template <bool BF16>
+__device__ __forceinline__ void tok_pfrags(float* ptr, const float (&pv)[4], int lane, float partf,
+                                           uint32_t (&b)[2][2]) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ptr[t * 40 + g + 8 * i] = pv[i];
+  __syncwarp();
+  const float* row = ptr + (g >> 1) * 40 + 2 * t;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const float2 lo = *reinterpret_cast<const float2*>(row + 16 * ks);
+    const float2 hi = *reinterpret_cast<const float2*>(row + 16 * ks + 8);
+    if constexpr (BF16) {
+      b[ks][0] = part_bf16(lo.x, lo.y, partf);
+      b[ks][1] = part_bf16(hi.x, hi.y, partf);
+    } else {
+      b[ks][0] = part_f16(lo.x, lo.y, partf);
+      b[ks][1] = part_f16(hi.x, hi.y, partf);
+    }
+  }
+  __syncwarp();
+}
+
 template <int KB, int VB, int D>
-__global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D>::MINB) decode_mma_kernel(DecodeParams p) {
+__device__ __forceinline__ void attend_qpage_tok(const uint8_t* page, TokState<D>& st, const float (&qf)[D / 4],
+                                                 const uint32_t (&qzb)[D / 8], float* wscr, float partf,
+                                                 int lane) {
   using C = Cfg<KB, VB, D>;
+  const int g = lane >> 2, t = lane & 3;
+  const uint8_t* vblk = page + code_block_bytes(KB, D);
+  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
+  const __half* kzero = kscale + D;
+  const __half* vscale = kzero + D;
+  const __half* vzero = vscale + kPageTokens;
+  float* ksf = wscr;
+  float* svf = wscr + 4 * C::KSROW;
+  float* zvf = svf + kPageTokens;
+  float* ptr = zvf + kPageTokens;  // [4][40]
+  {
+    constexpr int NE = D / 32;
+    const int i0 = lane * NE;
+    float* dst = ksf + (i0 / (D / 4)) * C::KSROW + (i0 % (D / 4));
+    if constexpr (NE == 4) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(kscale + i0);
+      float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+      float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+      if (C::tauK != 1.f) { c.x *= 1.f / C::tauK; c.y *= 1.f / C::tauK; }
+      *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, c.x, c.y);
+    } else {
+      const uint32_t raw = *reinterpret_cast<const uint32_t*>(kscale + i0);
+      float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw));
+      if (C::tauK != 1.f && (i0 & 2)) { a.x *= 1.f / C::tauK; a.y *= 1.f / C::tauK; }
+      *reinterpret_cast<float2*>(dst) = a;
+    }
+  }
+  const float vs = __half2float(vscale[lane]);
+  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
+  zvf[lane] = __half2float(vzero[lane]);
+  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
+  __syncwarp();
+
+  // --- QK: two token m-tiles, B = q' parts; z-term: A = z rows, B = q parts
+  float s2[2][4], cz[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+  const float* ksl = ksf + t * C::KSROW;
+  const uint32_t* zrow = reinterpret_cast<const uint32_t*>(kzero + t * (D / 4));
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<KB>::N];
+    load_tile_words<KB>(page, lane, dt, w);
+    const float4 sc4 = *reinterpret_cast<const float4*>(ksl + dt * 4);
+    const uint32_t b0 = part_f16(qf[dt * 4 + 0] * sc4.x, qf[dt * 4 + 1] * sc4.y, partf);
+    const uint32_t b1 = part_f16(qf[dt * 4 + 2] * sc4.z, qf[dt * 4 + 3] * sc4.w, partf);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag<KB>(w, mt, a);
+      mma_f16(s2[mt], a[0], a[1], a[2], a[3], b0, b1);
+    }
+    const uint2 z = *reinterpret_cast<const uint2*>(zrow + dt * 2);
+    mma_f16(cz, z.x, z.x, z.y, z.y, qzb[2 * dt], qzb[2 * dt + 1]);
+  }
+  const float czv = cz[0] + cz[1];  // head t: both parts of sum_c q_c z_c
+  float sc[4];
+  sc[0] = fmaf(s2[0][0] + s2[0][1], kTwo24, czv);
+  sc[1] = fmaf(s2[0][2] + s2[0][3], kTwo24 / C::sigmaK, czv);
+  sc[2] = fmaf(s2[1][0] + s2[1][1], kTwo24, czv);
+  sc[3] = fmaf(s2[1][2] + s2[1][3], kTwo24 / C::sigmaK, czv);
+  tok_rescale_update<D>(st, sc, tau);
+
+  // --- p' = p * s_t for tokens g + 8i; value zero term; transpose to B fragments
+  float pv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pv[i] = sc[i] * svf[g + 8 * i];
+    st.vz = fmaf(sc[i], zvf[g + 8 * i], st.vz);
+  }
+  uint32_t pb[2][2];
+  tok_pfrags<false>(ptr, pv, lane, partf, pb);
+
+  // --- PV: A = value codes (rows = channels), B = p' parts
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<VB>::N];
+    load_tile_words<VB>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      tile_afrag<VB>(w, ks, a);
+      mma_f16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void attend_bpage_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qbp)[D / 8],
+                                                 float* wscr, float partf, float scale_log2, int lane) {
+  constexpr int KS = D / 16;
+  float* ptr = wscr + 4 * (D / 4 + 4) + 2 * kPageTokens;
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<16>::N];
+    load_tile_words<16>(page, lane, dt, w);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag<16>(w, mt, a);
+      mma_bf16(s2[mt], a[0], a[1], a[2], a[3], qbp[2 * dt], qbp[2 * dt + 1]);
+    }
+  }
+  float sc[4] = {(s2[0][0] + s2[0][1]) * scale_log2, (s2[0][2] + s2[0][3]) * scale_log2,
+                 (s2[1][0] + s2[1][1]) * scale_log2, (s2[1][2] + s2[1][3]) * scale_log2};
+  tok_rescale_update<D>(st, sc, kTau);
+  uint32_t pb[2][2];
+  tok_pfrags<true>(ptr, sc, lane, partf, pb);
+  const uint8_t* vblk = page + code_block_bytes(16, D);
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<16>::N];
+    load_tile_words<16>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      tile_afrag<16>(w, ks, a);
+      mma_bf16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
+    }
+  }
+}
+
+// bf16 window (natural [32][D] rows in global memory), W < 32 valid tokens.
+template <int D>
+__device__ __forceinline__ void attend_window_tok(const __nv_bfloat16* win, int W, TokState<D>& st,
+                                                  const uint32_t (&qbp)[D / 8], float* wscr, float partf,
+                                                  float scale_log2, int lane) {
+  constexpr int KS = D / 16;
+  const int g = lane >> 2, t = lane & 3;
+  float* ptr = wscr + 4 * (D / 4 + 4) + 2 * kPageTokens;
+  const uint16_t* kw = reinterpret_cast<const uint16_t*>(win);
+  const uint16_t* vw = kw + kPageTokens * D;
+  auto kpair = [&](int tok, int dim) -> uint32_t {
+    return tok < W ? *reinterpret_cast<const uint32_t*>(kw + tok * D + dim) : 0u;
+  };
+  auto vpair = [&](int tok, int dim) -> uint32_t {
+    const uint32_t lo = tok < W ? vw[tok * D + dim] : 0u;
+    const uint32_t hi = tok + 1 < W ? vw[(tok + 1) * D + dim] : 0u;
+    return lo | (hi << 16);
+  };
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    if (16 * mt >= W) continue;  // warp-uniform
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int r0 = 16 * mt + g, c0 = 16 * dt + 2 * t;
+      mma_bf16(s2[mt], kpair(r0, c0), kpair(r0 + 8, c0), kpair(r0, c0 + 8), kpair(r0 + 8, c0 + 8), qbp[2 * dt],
+               qbp[2 * dt + 1]);
+    }
+  }
+  float sc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float v = (i & 1) ? (s2[i >> 1][2] + s2[i >> 1][3]) : (s2[i >> 1][0] + s2[i >> 1][1]);
+    sc[i] = (g + 8 * i) < W ? v * scale_log2 : -INFINITY;
+  }
+  tok_rescale_update<D>(st, sc, kTau);
+  uint32_t pb[2][2];
+  tok_pfrags<true>(ptr, sc, lane, partf, pb);
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    if (16 * ks >= W) continue;  // warp-uniform
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int tk = 16 * ks + 2 * t, ch = 16 * dt + g;
+      mma_bf16(st.o[dt], vpair(tk, ch), vpair(tk, ch + 8), vpair(tk + 8, ch), vpair(tk + 8, ch + 8), pb[ks][0],
+               pb[ks][1]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel --
+// Units: the pages of every (sequence b, KV head h) in order, followed by one
+// window unit when T mod 32 > 0 (or one empty unit when T = 0). Segment
+// (b, h) occupies units [ustart[b] + h * n_b, ... + n_b). The N units are cut
+// into gridDim.x balanced contiguous slices, one per CTA, so every CTA gets the
+// same amount of work whatever the sequence lengths.
+
+// Segment containing unit u.
+struct Seg {
+  int b, h, start, n;
+};
+
+__device__ __forceinline__ Seg seg_of(const int* ustart, int B, int H, int u) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ustart[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  Seg s;
+  s.b = lo;
+  s.n = (ustart[lo + 1] - ustart[lo]) / H;
+  s.h = (u - ustart[lo]) / s.n;
+  s.start = ustart[lo] + s.h * s.n;
+  return s;
+}
+
+// Balanced slices: with N = q * grid + r, CTA c owns
+// [c * q + min(c, r), (c + 1) * q + min(c + 1, r)) -- the first r slices hold one
+// extra unit. All in 32-bit integers (N < 2^31).
+struct Slicer {
+  int q, r;
+  __device__ __forceinline__ int lo(int c) const { return c * q + min(c, r); }
+  __device__ __forceinline__ bool empty(int c) const { return q == 0 && c >= r; }
+  // CTA whose slice contains unit u
+  __device__ __forceinline__ int cta_of(int u) const {
+    const int big = r * (q + 1);
+    return u < big ? u / (q + 1) : r + (u - big) / q;
+  }
+};
+
+// Walks the page units of one warp in the order the warp consumes them:
+// within each segment part [a, e) of the CTA slice, units a + warp + 4j.
+struct PageCursor {
+  int u, e;          // candidate unit, end of the current segment part
+  int seg_start, P;  // current segment's first unit and page count
+  const uint8_t* base;  // pages of the current (b, h)
+};
+
+template <int D>
+__device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p, const int* ustart, int B, int u1,
+                                            int warp) {
+  for (;;) {
+    if (c.u < c.e) {
+      if (c.u - c.seg_start < c.P) return true;
+      c.u += kWarps;  // the window / empty unit is the last of its segment
+      continue;
+    }
+    if (c.e >= u1) return false;
+    const int a = c.e;
+    const Seg sg = seg_of(ustart, B, p.n_kv_heads, a);
+    c.seg_start = sg.start;
+    c.e = min(sg.start + sg.n, u1);
+    c.P = p.len[sg.b] / kPageTokens;
+    c.base = p.pages + ((int64_t)(sg.b * p.n_kv_heads + sg.h) * p.max_pages) * p.page_bytes;
+    c.u = a + warp;
+  }
+}
+
+template <int KB, int VB, int D, bool TOK>
+__global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg<KB, VB, D>::MINB)
+    decode_mma_kernel(DecodeParams p) {
+  using C = Cfg<KB, VB, D>;
+  using State = typename std::conditional<TOK, TokState<D>, WarpState<D>>::type;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_last;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int H = p.n_kv_heads, G = p.gqa;
+  const int H = p.n_kv_heads, G = p.gqa, B = p.batch;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int T = p.len[b];
-  const int P = T / kPageTokens, W = T % kPageTokens;
-  const int nsplit = P > 0 ? (P + p.chunk - 1) / p.chunk : 1;
-  if (s >= nsplit) return;
-  const int p0 = s * p.chunk;
-  const int p1 = min(P, p0 + p.chunk);
+  // this lane's query head: row g (head rows) or column head g/2 (token rows)
+  const int qh = TOK ? (g >> 1) : g;
+  const float partf = (float)(g & 1);
 
   uint8_t* ring = smem + warp * C::R * C::STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + warp * C::R;
   float* wscr = reinterpret_cast<float*>(smem + C::WSCR_OFF + warp * C::WSCR_STRIDE);
   uint32_t* qz = reinterpret_cast<uint32_t*>(smem + C::QZ_OFF);
+  float* mo = reinterpret_cast<float*>(smem + C::MERGE_OFF);        // [kWarps][G][D]
+  float* mm = mo + kWarps * G * D;                                   // [kWarps][8]
+  float* ml = mm + kWarps * kMaxGqa;                                 // [kWarps][8]
+  int* ustart = reinterpret_cast<int*>(ml + kWarps * kMaxGqa);       // [B + 1]
 
-  // ---- pipeline start: this warp's pages are p0 + warp + kWarps * i
-  const int first = p0 + warp;
-  const int n_my = p1 > first ? (p1 - first + kWarps - 1) / kWarps : 0;
-  const uint8_t* seq_pages = p.pages + ((int64_t)(b * H + h) * p.max_pages) * p.page_bytes;
+  // ---- units per sequence: exclusive scan (warp 0), n_b = H * max(1, P + (W > 0))
+  if (warp == 0) {
+    int carry = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int bb = b0 + lane;
+      int n = 0;
+      if (bb < B) {
+        const int T = p.len[bb];
+        n = T / kPageTokens + (T % kPageTokens > 0 ? 1 : 0);
+        n = (n > 0 ? n : 1) * H;
+      }
+      int x = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (bb < B) ustart[bb] = carry + x - n;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) ustart[B] = carry;
+  }
   if (lane == 0) {
     for (int r = 0; r < C::R; ++r) mbar_init(&bars[r], 1);
     mbar_init_fence();
   }
-  __syncwarp();
+  __syncthreads();
+  const int N = ustart[B];
+  const Slicer sl{N / (int)gridDim.x, N % (int)gridDim.x};
+  const int u0 = sl.lo(blockIdx.x), u1 = sl.lo(blockIdx.x + 1);
+  if (u0 >= u1) return;
+
+  // ---- producer: the first R page units of this warp
+  PageCursor cur;
+  cur.u = u0;  // >= e: the first call looks up the segment of u0
+  cur.e = u0;
+  cur.seg_start = 0;
+  cur.P = 0;
+  cur.base = nullptr;
+  int issued = 0;
   if (lane == 0) {
-    for (int i = 0; i < n_my && i < C::R; ++i) {
-      mbar_expect_tx(&bars[i], C::PB);
-      bulk_load(ring + i * C::STAGE, seq_pages + (int64_t)(first + i * kWarps) * p.page_bytes, C::PB, &bars[i]);
+    for (int r = 0; r < C::R; ++r) {
+      if (!cursor_next<D>(cur, p, ustart, B, u1, warp)) break;
+      mbar_expect_tx(&bars[r], C::PB);
+      bulk_load(ring + r * C::STAGE, cur.base + (int64_t)(cur.u - cur.seg_start) * p.page_bytes, C::PB, &bars[r]);
+      cur.u += kWarps;
+      ++issued;
     }
   }
 
-  // ---- query operands (row g = head g; heads >= G are zero)
-  const __nv_bfloat16* qrow = p.Q + ((int64_t)b * H * G + (int64_t)h * G + (g < G ? g : 0)) * D;
-  float qf[D / 4];  // q * log2(e)/sqrt(D) at this lane's channels (quantized pages)
-  if constexpr (!C::kBf16) {
-#pragma unroll
-    for (int dt = 0; dt < C::KS; ++dt) {
-      uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
-      uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
-      if (g >= G) lo = hi = 0u;
-      const float2 l2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&lo));
-      const float2 h2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&hi));
-      qf[dt * 4 + 0] = l2.x * p.scale_log2;
-      qf[dt * 4 + 1] = l2.y * p.scale_log2;
-      qf[dt * 4 + 2] = h2.x * p.scale_log2;
-      qf[dt * 4 + 3] = h2.y * p.scale_log2;
-    }
-    if (warp == 0) {
+  bool ok = true;
+  int consumed = 0;
+  for (int a = u0; a < u1;) {
+    const Seg sg = seg_of(ustart, B, H, a);
+    const int e = min(sg.start + sg.n, u1);
+    const int T = p.len[sg.b];
+    const int P = T / kPageTokens, W = T % kPageTokens;
+    const bool qvalid = qh < G;
+    const __nv_bfloat16* qrow = p.Q + ((int64_t)(sg.b * H + sg.h) * G + (qvalid ? qh : 0)) * D;
+
+    // ---- query operands
+    float qf[D / 4];
+    uint32_t qb[D / 8];   // bf16 pairs (head rows) or bf16 parts (token rows)
+    uint32_t qzb[D / 8];  // token rows: z-term B fragments (q parts)
+    auto load_qbp = [&]() {
 #pragma unroll
       for (int dt = 0; dt < C::KS; ++dt) {
-        uint4 a;
-        split_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], a.x, a.y);
-        split_f16(qf[dt * 4 + 2], qf[dt * 4 + 3], a.z, a.w);
-        *reinterpret_cast<uint4*>(qz + (dt * 32 + lane) * 4) = a;
+        uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
+        uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
+        const bool keep = qvalid && (!TOK || (g & 1) == 0);  // q is exact in bf16: low part is zero
+        qb[2 * dt] = keep ? lo : 0u;
+        qb[2 * dt + 1] = keep ? hi : 0u;
+      }
+    };
+    if constexpr (C::kBf16) {
+      load_qbp();
+    } else {
+#pragma unroll
+      for (int dt = 0; dt < C::KS; ++dt) {
+        uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
+        uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
+        if (!qvalid) lo = hi = 0u;
+        const float2 l2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&lo));
+        const float2 h2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&hi));
+        qf[dt * 4 + 0] = l2.x * p.scale_log2;
+        qf[dt * 4 + 1] = l2.y * p.scale_log2;
+        qf[dt * 4 + 2] = h2.x * p.scale_log2;
+        qf[dt * 4 + 3] = h2.y * p.scale_log2;
+      }
+      if constexpr (TOK) {
+#pragma unroll
+        for (int dt = 0; dt < C::KS; ++dt) {
+          qzb[2 * dt] = part_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], partf);
+          qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2], qf[dt * 4 + 3], partf);
+        }
+      } else {
+        if (warp == 0) {
+#pragma unroll
+          for (int dt = 0; dt < C::KS; ++dt) {
+            uint4 q4;
+            split_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], q4.x, q4.y);
+            split_f16(qf[dt * 4 + 2], qf[dt * 4 + 3], q4.z, q4.w);
+            *reinterpret_cast<uint4*>(qz + (dt * 32 + lane) * 4) = q4;
+          }
+        }
+        __syncthreads();
+      }
+    }
+
+    State st;
+#pragma unroll
+    for (int j = 0; j < (TOK ? D / 16 : D / 8); ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st.o[j][k] = 0.f;
+    st.m = -INFINITY;
+    st.l = 0.f;
+    st.vz = 0.f;
+    bool converted = C::kBf16;
+    // quantized accumulators to true units: acc * 2^24 (/ sigmaV on channels with bit 3 set)
+    auto to_true_units = [&]() {
+      if constexpr (TOK) {
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+          st.o[j][0] *= kTwo24;
+          st.o[j][1] *= kTwo24;
+          st.o[j][2] *= kTwo24 / C::sigmaV;
+          st.o[j][3] *= kTwo24 / C::sigmaV;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+          const float f = (j & 1) ? kTwo24 / C::sigmaV : kTwo24;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) st.o[j][k] *= f;
+        }
+      }
+      converted = true;
+    };
+
+    // ---- this warp's units of the segment part [a, e)
+    for (int u = a + warp; u < e; u += kWarps) {
+      const int k = u - sg.start;
+      if (k < P) {
+        if (ok) {
+          const int stage = consumed % C::R;
+          const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
+          if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
+            ok = false;
+          } else {
+            const uint8_t* page = ring + stage * C::STAGE;
+            if constexpr (TOK) {
+              if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
+              else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
+            } else {
+              if constexpr (C::kBf16) attend_bpage<D>(page, st, qb, p.scale_log2, lane);
+              else attend_qpage<KB, VB, D>(page, st, qf, qz, wscr, lane);
+            }
+            ++consumed;
+            __syncwarp();
+            if (lane == 0 && cursor_next<D>(cur, p, ustart, B, u1, warp)) {
+              fence_proxy_async();
+              mbar_expect_tx(&bars[stage], C::PB);
+              bulk_load(ring + stage * C::STAGE, cur.base + (int64_t)(cur.u - cur.seg_start) * p.page_bytes, C::PB,
+                        &bars[stage]);
+              cur.u += kWarps;
+              ++issued;
+            }
+          }
+        }
+      } else if (W > 0) {
+        if constexpr (!C::kBf16) {
+          to_true_units();
+          load_qbp();
+        }
+        const __nv_bfloat16* win = p.window + ((int64_t)(sg.b * H + sg.h) * 2) * kPageTokens * D;
+        if constexpr (TOK) attend_window_tok<D>(win, W, st, qb, wscr, partf, p.scale_log2, lane);
+        else attend_window<D>(win, W, st, qb, p.scale_log2, lane);
+      }
+    }
+    if (!converted) to_true_units();
+
+    // ---- warps -> shared memory, CTA merge
+    if constexpr (TOK) {
+      float l = st.l, vz = st.vz;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        vz += __shfl_xor_sync(0xffffffffu, vz, o);
+      }
+      if (t < G) {
+        float* dst = mo + (warp * G + t) * D;
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+          dst[16 * j + g] = st.o[j][0] + st.o[j][1] + vz;
+          dst[16 * j + 8 + g] = st.o[j][2] + st.o[j][3] + vz;
+        }
+        if (g == 0) {
+          mm[warp * kMaxGqa + t] = st.m;
+          ml[warp * kMaxGqa + t] = l;
+        }
+      }
+    } else {
+      float l = st.l + __shfl_xor_sync(0xffffffffu, st.l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      float vz = st.vz + __shfl_xor_sync(0xffffffffu, st.vz, 1);
+      vz += __shfl_xor_sync(0xffffffffu, vz, 2);
+      if (g < G) {
+        float* dst = mo + (warp * G + g) * D;
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+          dst[8 * j + 2 * t] = st.o[j][0] + st.o[j][2] + vz;
+          dst[8 * j + 2 * t + 1] = st.o[j][1] + st.o[j][3] + vz;
+        }
+        if (t == 0) {
+          mm[warp * kMaxGqa + g] = st.m;
+          ml[warp * kMaxGqa + g] = l;
+        }
       }
     }
     __syncthreads();
-  }
-
-  WarpState<D> st;
+    const int seg = sg.b * H + sg.h;
+    const bool whole = (a == sg.start) && (e == sg.start + sg.n);
+    float* outp = p.out + (int64_t)seg * G * D;
+    float* part = p.partials + ((int64_t)blockIdx.x * 2 + (a == u0 ? 0 : 1)) * G * (D + 2);
+    for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
+      const int gg = idx / D, d = idx % D;
+      float M = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j)
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * kMaxGqa + gg]);
+      float L = 0.f, O = 0.f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) st.o[j][k] = 0.f;
-  st.m = -INFINITY;
-  st.l = 0.f;
-  st.vz = 0.f;
-
-  // ---- page loop
-  {
-    uint32_t qb[D / 8];
-    if constexpr (C::kBf16) load_qb<D>(qrow, g < G, t, qb);
-    bool ok = true;
-    int consumed = 0;
-    for (int i = 0; i < n_my; ++i) {
-      const int stage = i % C::R;
-      const bool arrived = mbar_wait(&bars[stage], (uint32_t)((i / C::R) & 1));
-      if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
-        ok = false;
-        break;
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = mm[w * kMaxGqa + gg];
+        const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        L = fmaf(f, ml[w * kMaxGqa + gg], L);
+        O = fmaf(f, mo[(w * G + gg) * D + d], O);
       }
-      consumed = i + 1;
-      const uint8_t* page = ring + stage * C::STAGE;
-      if constexpr (C::kBf16) attend_bpage<D>(page, st, qb, p.scale_log2, lane);
-      else attend_qpage<KB, VB, D>(page, st, qf, qz, wscr, lane);
-      __syncwarp();
-      if (lane == 0 && i + C::R < n_my) {
-        fence_proxy_async();
-        mbar_expect_tx(&bars[stage], C::PB);
-        bulk_load(ring + stage * C::STAGE, seq_pages + (int64_t)(first + (i + C::R) * kWarps) * p.page_bytes, C::PB,
-                  &bars[stage]);
+      if (whole) {
+        outp[idx] = L > 0.f ? O / L : 0.f;
+      } else {
+        part[gg * (D + 2) + d] = O;
+        if (d == 0) {
+          part[gg * (D + 2) + D] = M;
+          part[gg * (D + 2) + D + 1] = L;
+        }
       }
     }
-    if (!ok) {
-      // a copy never completed: report it, then let the copies in flight land
-      // (each wait bounded again) before this CTA's shared memory goes away
-      if (lane == 0 && p.err) atomicExch(p.err, 1);
-      const int issued = min(n_my, consumed + C::R);
-      for (int i = consumed; i < issued; ++i) mbar_wait(&bars[i % C::R], (uint32_t)((i / C::R) & 1));
-    }
-  }
-
-  // ---- quantized accumulators to true units: O = acc * 2^24 / sigmaV
-  if constexpr (!C::kBf16) {
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      const float f = (j & 1) ? kTwo24 / C::sigmaV : kTwo24;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) st.o[j][k] *= f;
-    }
-  }
-  if (s == nsplit - 1 && W > 0 && warp == kWarps - 1) {
-    uint32_t qb[D / 8];
-    load_qb<D>(qrow, g < G, t, qb);
-    const __nv_bfloat16* win = p.window + ((int64_t)(b * H + h) * 2) * kPageTokens * D;
-    attend_window<D>(win, W, st, qb, p.scale_log2, lane);
-  }
-
-  // ---- warp results to shared memory (reusing the ring; all copies have landed)
-  float l = st.l + __shfl_xor_sync(0xffffffffu, st.l, 1);
-  l += __shfl_xor_sync(0xffffffffu, l, 2);
-  float vz = st.vz + __shfl_xor_sync(0xffffffffu, st.vz, 1);
-  vz += __shfl_xor_sync(0xffffffffu, vz, 2);
-  __syncthreads();
-  float* mo = reinterpret_cast<float*>(smem);                  // [kWarps][G][D]
-  float* mm = mo + kWarps * kMaxGqa * D;                       // [kWarps][G]
-  float* ml = mm + kWarps * kMaxGqa;
-  if (g < G) {
-    float* dst = mo + (warp * kMaxGqa + g) * D;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      dst[8 * j + 2 * t] = st.o[j][0] + st.o[j][2] + vz;
-      dst[8 * j + 2 * t + 1] = st.o[j][1] + st.o[j][3] + vz;
-    }
-    if (t == 0) {
-      mm[warp * kMaxGqa + g] = st.m;
-      ml[warp * kMaxGqa + g] = l;
-    }
-  }
-  __syncthreads();
-
-  // ---- CTA merge over warps, then output or split-K partial
-  float* outp = p.out + ((int64_t)b * H * G + (int64_t)h * G) * D;
-  const int64_t slot0 = (int64_t)(b * H + h) * p.splits_stride;
-  float* part = p.partials + (slot0 + s) * G * (D + 2);
-  for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
-    const int gg = idx / D, d = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * kMaxGqa + gg]);
-    float L = 0.f, O = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float mw = mm[w * kMaxGqa + gg];
-      const float a = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-      L = fmaf(a, ml[w * kMaxGqa + gg], L);
-      O = fmaf(a, mo[(w * kMaxGqa + gg) * D + d], O);
-    }
-    if (nsplit == 1) {
-      outp[idx] = L > 0.f ? O / L : 0.f;
-    } else {
-      part[gg * (D + 2) + d] = O;
-      if (d == 0) {
-        part[gg * (D + 2) + D] = M;
-        part[gg * (D + 2) + D + 1] = L;
+    if (!whole) {
+      // the last CTA of a split segment merges the slices' partials in slice order
+      // (with more CTAs than units some slices are empty; they hold no part of any segment)
+      const int c_lo = sl.cta_of(sg.start), c_hi = sl.cta_of(sg.start + sg.n - 1);
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int parts = 0;
+        for (int c = c_lo; c <= c_hi; ++c) parts += !sl.empty(c);
+        const int prev = atomicAdd(&p.ctr[seg], 1);
+        s_last = (prev == parts - 1);
+        if (s_last) p.ctr[seg] = 0;
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
+          const int gg = idx / D, d = idx % D;
+          float M = -INFINITY;
+          for (int c = c_lo; c <= c_hi; ++c) {
+            if (sl.empty(c)) continue;
+            const int slot = (sl.lo(c) >= sg.start) ? 0 : 1;
+            const float* r = p.partials + ((int64_t)c * 2 + slot) * G * (D + 2) + gg * (D + 2);
+            M = fmaxf(M, __ldcg(r + D));
+          }
+          float L = 0.f, O = 0.f;
+          for (int c = c_lo; c <= c_hi; ++c) {
+            if (sl.empty(c)) continue;
+            const int slot = (sl.lo(c) >= sg.start) ? 0 : 1;
+            const float* r = p.partials + ((int64_t)c * 2 + slot) * G * (D + 2) + gg * (D + 2);
+            const float mc = __ldcg(r + D);
+            const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+            L = fmaf(f, __ldcg(r + D + 1), L);
+            O = fmaf(f, __ldcg(r + d), O);
+          }
+          outp[idx] = L > 0.f ? O / L : 0.f;
+        }
       }
     }
+    __syncthreads();  // merge area, qz and s_last are reused by the next segment
+    a = e;
   }
-  if (nsplit == 1) return;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(&p.ctr[b * H + h], 1);
-    s_last = (prev == nsplit - 1);
-    if (s_last) p.ctr[b * H + h] = 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* parts = p.partials + slot0 * G * (D + 2);
-  for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
-    const int gg = idx / D, d = idx % D;
-    float M = -INFINITY;
-    for (int j = 0; j < nsplit; ++j) M = fmaxf(M, __ldcg(parts + ((int64_t)j * G + gg) * (D + 2) + D));
-    float L = 0.f, O = 0.f;
-    for (int j = 0; j < nsplit; ++j) {
-      const float* r = parts + ((int64_t)j * G + gg) * (D + 2);
-      const float mj = __ldcg(r + D);
-      const float a = (mj == -INFINITY) ? 0.f : exp2f(mj - M);
-      L = fmaf(a, __ldcg(r + D + 1), L);
-      O = fmaf(a, __ldcg(r + d), O);
-    }
-    outp[idx] = L > 0.f ? O / L : 0.f;
+
+  if (!ok) {
+    // a copy never completed: report it, then let the copies in flight land
+    // (each wait bounded again) before this CTA's shared memory goes away
+    if (lane == 0 && p.err) atomicExch(p.err, 1);
+    for (int i = consumed; i < issued; ++i) mbar_wait(&bars[i % C::R], (uint32_t)((i / C::R) & 1));
   }
 }
 
-template <int KB, int VB, int D>
-cudaError_t launch3(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+template <int KB, int VB, int D, bool TOK>
+cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   using C = Cfg<KB, VB, D>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM);
+  static int configured_smem = 0;
+  static int occ_smem = -1, occ_blocks = 0;
+  const int smem = C::smem_bytes(p.gqa, p.batch);
+  if (smem > configured_smem) {
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured_smem = smem;
   }
-  decode_mma_kernel<KB, VB, D><<<grid, kThreads, C::SMEM, s>>>(p);
+  if (smem != occ_smem) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_blocks, decode_mma_kernel<KB, VB, D, TOK>,
+                                                                  kThreads, smem);
+    if (e != cudaSuccess) return e;
+    occ_smem = smem;
+  }
+  int64_t grid = (int64_t)(occ_blocks > 0 ? occ_blocks : 1) * p.sm_count;
+  grid = std::min<int64_t>(grid, p.n_units);
+  grid = std::min<int64_t>(grid, p.max_ctas);
+  if (grid < 1) grid = 1;
+  decode_mma_kernel<KB, VB, D, TOK><<<(unsigned)grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
+template <int KB, int VB, int D>
+cudaError_t launch3(const DecodeParams& p, cudaStream_t s) {
+  // token rows when the query group fits the 8 (head, part) columns
+  return p.gqa <= 4 ? launch4<KB, VB, D, true>(p, s) : launch4<KB, VB, D, false>(p, s);
+}
+
 template <int D>
-cudaError_t launch_d(int kb, int vb, const DecodeParams& p, dim3 grid, cudaStream_t s) {
+cudaError_t launch_d(int kb, int vb, const DecodeParams& p, cudaStream_t s) {
 #define KVQ_PAIR(K_, V_) \
-  if (kb == K_ && vb == V_) return launch3<K_, V_, D>(p, grid, s);
+  if (kb == K_ && vb == V_) return launch3<K_, V_, D>(p, s);
   KVQ_PAIR(2, 2) KVQ_PAIR(2, 4) KVQ_PAIR(2, 8)
   KVQ_PAIR(4, 2) KVQ_PAIR(4, 4) KVQ_PAIR(4, 8)
   KVQ_PAIR(8, 2) KVQ_PAIR(8, 4) KVQ_PAIR(8, 8)
@@ -727,9 +1229,9 @@ cudaError_t launch_d(int kb, int vb, const DecodeParams& p, dim3 grid, cudaStrea
 
 }  // namespace
 
-cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  if (D == 64) return launch_d<64>(kb, vb, p, grid, s);
-  if (D == 128) return launch_d<128>(kb, vb, p, grid, s);
+cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s) {
+  if (D == 64) return launch_d<64>(kb, vb, p, s);
+  if (D == 128) return launch_d<128>(kb, vb, p, s);
   return cudaErrorInvalidValue;
 }
 

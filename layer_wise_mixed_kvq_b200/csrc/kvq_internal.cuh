@@ -70,8 +70,12 @@ struct DecodeParams {
   int max_pages;
   int n_kv_heads;
   int gqa;               // query heads per KV head
-  int chunk;             // pages per split
-  int splits_stride;     // partial slots per (b, h)
+  int batch;             // sequences b < batch are attended
+  int chunk;             // CUDA-core kernel: pages per split
+  int splits_stride;     // CUDA-core kernel: partial slots per (b, h)
+  int n_units;           // tensor-core kernel: total units (pages + window/empty units), host view
+  int max_ctas;          // tensor-core kernel: CTAs the partial buffer can serve (2 records each)
+  int sm_count;
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
 };
@@ -80,7 +84,8 @@ struct DecodeParams {
 cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
                           cudaStream_t s);
 cudaError_t launch_decode_simt(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
-cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+// Grid chosen inside: resident CTAs x SMs, capped by n_units and max_ctas.
+cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s);
 // Pages per split-K CTA for a layer-step: about 3 CTAs per SM, at least 8 pages
 // (2 per warp) per CTA, and no more than `stride` splits per (sequence, head).
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_pages_per_seq, int64_t stride);

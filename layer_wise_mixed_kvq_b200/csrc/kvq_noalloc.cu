@@ -85,11 +85,11 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   const int G = n_q_heads / n_kv_heads;
   const int64_t pairs = (int64_t)batch * n_kv_heads;
   const size_t ctr_bytes = ((size_t)pairs * 4 + 255) / 256 * 256;
-  const size_t slot_bytes = (size_t)G * (head_dim + 2) * 4;
-  if (ctr_bytes + slot_bytes * (size_t)pairs > kScratchBytes)
-    return fail(KVQ_ECAPACITY, "batch * n_kv_heads * G * (head_dim + 2) * 4 bytes of split-K state exceeds the "
-                               "16 MiB static scratch; use fewer sequences per call");
-  const int64_t stride = (int64_t)((kScratchBytes - ctr_bytes) / (slot_bytes * (size_t)pairs));
+  const size_t rec_bytes = (size_t)G * (head_dim + 2) * 4;  // one split-K record (acc, m, l)
+  if (ctr_bytes + 2 * rec_bytes > kScratchBytes)
+    return fail(KVQ_ECAPACITY, "batch * n_kv_heads merge counters (4 bytes each) leave no room for split records "
+                               "in the 16 MiB static scratch; use fewer sequences per call");
+  const int64_t records = (int64_t)((kScratchBytes - ctr_bytes) / rec_bytes);
 
   void* base = nullptr;
   kvq_status st = scratch_address(&base);
@@ -102,9 +102,10 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t max_p = max_seq_len / kvq::kPageTokens;
-  const int64_t chunk = kvq::choose_chunk(sms, max_p * pairs, max_p, stride);
+  const int64_t stride = records / pairs;  // CUDA-core kernel: records per (sequence, head)
+  const int64_t chunk = stride >= 1 ? kvq::choose_chunk(sms, max_p * pairs, max_p, stride) : max_p + 1;
   const int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
-
+  const int64_t n_units = pairs * (max_p + 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the merge counters must start at zero; the array keeps the last call's contents
   cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)pairs * 4, s);
@@ -123,7 +124,11 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.n_kv_heads = n_kv_heads;
   p.gqa = G;
   p.chunk = (int)chunk;
-  p.splits_stride = (int)stride;
+  p.splits_stride = (int)std::max<int64_t>(stride, 1);
+  p.batch = batch;
+  p.n_units = (int)std::min<int64_t>(n_units, INT32_MAX);
+  p.max_ctas = (int)std::min<int64_t>(records / 2, INT32_MAX);
+  p.sm_count = sms;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   e = kvq::launch_decode(pair.k_bits, pair.v_bits, head_dim, p, dim3(splits, n_kv_heads, batch), s);
   if (e != cudaSuccess) return fail(KVQ_ECUDA, std::string("decode kernel launch: ") + cudaGetErrorString(e));

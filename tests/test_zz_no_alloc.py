@@ -85,13 +85,14 @@ def test_noalloc_matches_decode_attn_twice(kvq, pair, D, G):
 
 
 def test_noalloc_rejects_oversized_scratch(kvq):
+    # 1024 sequences x 8192 KV heads need 32 MiB of merge counters alone
     dev = torch.device("cuda")
     pages = torch.zeros(16, dtype=torch.uint8, device=dev)
     window = torch.zeros(8, dtype=torch.bfloat16, device=dev)
     seq_len = torch.zeros(1024, dtype=torch.int32, device=dev)
-    Q = torch.zeros((1024, 64, 128), dtype=torch.bfloat16, device=dev)
-    out = torch.zeros((1024, 64, 128), dtype=torch.float32, device=dev)
+    Q = torch.zeros((1024, 1, 8), dtype=torch.bfloat16, device=dev)
+    out = torch.zeros((1024, 1, 8), dtype=torch.float32, device=dev)
     with pytest.raises(kvq.KVQError) as e:
-        kvq.kvq_decode_attn_noalloc((4, 4), 128, 64, 8, pages, 0, window, seq_len, 0, Q, out)
+        kvq.kvq_decode_attn_noalloc((4, 4), 128, 8192, 8192, pages, 0, window, seq_len, 0, Q, out)
     assert e.value.status == kvq.KVQ_ECAPACITY
     assert "16 MiB" in str(e.value)
