@@ -382,7 +382,11 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.err = c->err;
   p.batch = batch;
   p.n_units = (int)n_units;
-  p.max_ctas = (int)std::min<int64_t>(c->partial_slots / 2, INT32_MAX);
+  {
+    // partial region holds partial_slots * G * (D + 2) floats; split records are padded
+    const int64_t floats = c->partial_slots * (int64_t)p.gqa * (c->head_dim + 2);
+    p.max_ctas = (int)std::min<int64_t>(floats / kvq::split_record_floats(p.gqa, c->head_dim) / 2, INT32_MAX);
+  }
   p.sm_count = c->sm_count;
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));

@@ -94,6 +94,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// Device-scope fetch-add with acquire-release ordering: releases every write
+// this thread has observed (the CTA's partial records, via the preceding
+// barrier) and acquires the other CTAs' released records.
+__device__ __forceinline__ int atomic_add_acq_rel(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -164,16 +173,19 @@ struct Cfg {
   // shared memory layout
   static constexpr int RING = kWarps * R * STAGE;
   static constexpr int MBAR_OFF = RING;
-  static constexpr int MBAR_BYTES = (kWarps * R * 8 + 127) / 128 * 128;
+  static constexpr int MBAR_BYTES = ((kWarps * R + 2) * 8 + 127) / 128 * 128;  // + 2 query-row barriers
   static constexpr int WSCR_FLOATS = 4 * KSROW + 64 + 160;  // key scales, value scales/zeros, p' transpose tile
   static constexpr int WSCR_OFF = MBAR_OFF + MBAR_BYTES;
   static constexpr int WSCR_STRIDE = (WSCR_FLOATS * 4 + 127) / 128 * 128;
   static constexpr int QZ_OFF = WSCR_OFF + kWarps * WSCR_STRIDE;
-  static constexpr int QZ_BYTES = KS * 32 * 16;
-  static constexpr int MERGE_OFF = QZ_OFF + QZ_BYTES;
+  static constexpr int QZ_BYTES = KS * 32 * 16;            // head rows: z-term q fragments
+  static constexpr int QBUF_BYTES = 2 * kMaxGqa * D * 2;   // 2 x [8][D] bf16 query rows (= QZ_BYTES)
+  // token rows have no z-term fragments in shared memory: their query rows take that place
+  static constexpr int qbuf_off(bool tok) { return tok ? QZ_OFF : QZ_OFF + QZ_BYTES; }
+  static constexpr int merge_off(bool tok) { return qbuf_off(tok) + QBUF_BYTES; }
   // then: merge area [kWarps][G][D] + m, l [kWarps][8] floats, unit starts [batch + 1] ints
-  static int smem_bytes(int G, int batch) {
-    return MERGE_OFF + (kWarps * G * D + 2 * kWarps * kMaxGqa) * 4 + (batch + 1) * 4;
+  static int smem_bytes(bool tok, int G, int batch) {
+    return merge_off(tok) + (kWarps * G * D + 2 * kWarps * kMaxGqa) * 4 + (batch + 1) * 4;
   }
   static_assert(PB % 16 == 0, "bulk copies need 16-byte multiples");
 };
@@ -880,10 +892,12 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + warp * C::R;
   float* wscr = reinterpret_cast<float*>(smem + C::WSCR_OFF + warp * C::WSCR_STRIDE);
   uint32_t* qz = reinterpret_cast<uint32_t*>(smem + C::QZ_OFF);
-  float* mo = reinterpret_cast<float*>(smem + C::MERGE_OFF);        // [kWarps][G][D]
+  float* mo = reinterpret_cast<float*>(smem + C::merge_off(TOK));   // [kWarps][G][D]
   float* mm = mo + kWarps * G * D;                                   // [kWarps][8]
   float* ml = mm + kWarps * kMaxGqa;                                 // [kWarps][8]
   int* ustart = reinterpret_cast<int*>(ml + kWarps * kMaxGqa);       // [B + 1]
+  __nv_bfloat16* qbuf = reinterpret_cast<__nv_bfloat16*>(smem + C::qbuf_off(TOK));  // [2][8][D]
+  uint64_t* qbars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + kWarps * C::R;
 
   // ---- units per sequence: exclusive scan (warp 0), n_b = H * max(1, P + (W > 0))
   if (warp == 0) {
@@ -909,6 +923,10 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   }
   if (lane == 0) {
     for (int r = 0; r < C::R; ++r) mbar_init(&bars[r], 1);
+    if (warp == 0) {
+      mbar_init(&qbars[0], 1);
+      mbar_init(&qbars[1], 1);
+    }
     mbar_init_fence();
   }
   __syncthreads();
@@ -916,6 +934,15 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   const Slicer sl{N / (int)gridDim.x, N % (int)gridDim.x};
   const int u0 = sl.lo(blockIdx.x), u1 = sl.lo(blockIdx.x + 1);
   if (u0 >= u1) return;
+
+  // ---- query rows arrive by bulk copy (the first one ahead of the page stream)
+  const uint32_t qbytes = (uint32_t)(G * D * 2);
+  auto issue_q = [&](int unit, int buf) {
+    const Seg qs = seg_of(ustart, B, H, unit);
+    mbar_expect_tx(&qbars[buf], qbytes);
+    bulk_load(qbuf + buf * kMaxGqa * D, p.Q + (int64_t)(qs.b * H + qs.h) * G * D, qbytes, &qbars[buf]);
+  };
+  if (threadIdx.x == 0) issue_q(u0, 0);
 
   // ---- producer: the first R page units of this warp
   PageCursor cur;
@@ -937,13 +964,19 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
 
   bool ok = true;
   int consumed = 0;
-  for (int a = u0; a < u1;) {
+  int segi = 0;
+  for (int a = u0; a < u1; ++segi) {
     const Seg sg = seg_of(ustart, B, H, a);
     const int e = min(sg.start + sg.n, u1);
     const int T = p.len[sg.b];
     const int P = T / kPageTokens, W = T % kPageTokens;
     const bool qvalid = qh < G;
-    const __nv_bfloat16* qrow = p.Q + ((int64_t)(sg.b * H + sg.h) * G + (qvalid ? qh : 0)) * D;
+    {
+      const bool got = mbar_wait(&qbars[segi & 1], (uint32_t)((segi >> 1) & 1));
+      if (!__all_sync(0xffffffffu, got)) ok = false;
+      if (threadIdx.x == 0 && e < u1) issue_q(e, (segi + 1) & 1);  // prefetch the next segment's query
+    }
+    const __nv_bfloat16* qrow = qbuf + (segi & 1) * kMaxGqa * D + (qvalid ? qh : 0) * D;
 
     // ---- query operands
     float qf[D / 4];
@@ -1108,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
     const int seg = sg.b * H + sg.h;
     const bool whole = (a == sg.start) && (e == sg.start + sg.n);
     float* outp = p.out + (int64_t)seg * G * D;
-    float* part = p.partials + ((int64_t)blockIdx.x * 2 + (a == u0 ? 0 : 1)) * G * (D + 2);
+    float* part = p.partials + ((int64_t)blockIdx.x * 2 + (a == u0 ? 0 : 1)) * split_record_floats(G, D);
     for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
       const int gg = idx / D, d = idx % D;
       float M = -INFINITY;
@@ -1125,49 +1158,52 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
       if (whole) {
         outp[idx] = L > 0.f ? O / L : 0.f;
       } else {
-        part[gg * (D + 2) + d] = O;
+        // record: [G][D] accumulators, then [G] maxima, then [G] sums
+        part[idx] = O;
         if (d == 0) {
-          part[gg * (D + 2) + D] = M;
-          part[gg * (D + 2) + D + 1] = L;
+          part[G * D + gg] = M;
+          part[G * D + G + gg] = L;
         }
       }
     }
     if (!whole) {
-      // the last CTA of a split segment merges the slices' partials in slice order
-      // (with more CTAs than units some slices are empty; they hold no part of any segment)
+      // The last CTA of a split segment merges the slices' partials in slice
+      // order (empty slices, possible when CTAs outnumber units, hold nothing).
       const int c_lo = sl.cta_of(sg.start), c_hi = sl.cta_of(sg.start + sg.n - 1);
-      __threadfence();
-      __syncthreads();
+      __syncthreads();  // this CTA's partial record is complete
       if (threadIdx.x == 0) {
         int parts = 0;
         for (int c = c_lo; c <= c_hi; ++c) parts += !sl.empty(c);
-        const int prev = atomicAdd(&p.ctr[seg], 1);
+        const int prev = atomic_add_acq_rel(&p.ctr[seg], 1);
         s_last = (prev == parts - 1);
         if (s_last) p.ctr[seg] = 0;
       }
       __syncthreads();
       if (s_last) {
-        __threadfence();
-        for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
-          const int gg = idx / D, d = idx % D;
-          float M = -INFINITY;
+        // one pass over the records, online rescaling, four channels per thread
+        for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += kThreads) {
+          const int gg = (4 * i4) / D, d = (4 * i4) % D;
+          float M = -INFINITY, L = 0.f;
+          float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
           for (int c = c_lo; c <= c_hi; ++c) {
             if (sl.empty(c)) continue;
             const int slot = (sl.lo(c) >= sg.start) ? 0 : 1;
-            const float* r = p.partials + ((int64_t)c * 2 + slot) * G * (D + 2) + gg * (D + 2);
-            M = fmaxf(M, __ldcg(r + D));
+            const float* r = p.partials + ((int64_t)c * 2 + slot) * split_record_floats(G, D);
+            const float mc = __ldcg(r + G * D + gg), lc = __ldcg(r + G * D + G + gg);
+            const float4 oc = __ldcg(reinterpret_cast<const float4*>(r + gg * D + d));
+            const float Mn = fmaxf(M, mc);
+            const float fa = (M == -INFINITY) ? 0.f : exp2f(M - Mn);
+            const float fb = (mc == -INFINITY) ? 0.f : exp2f(mc - Mn);
+            L = L * fa + lc * fb;
+            O.x = O.x * fa + oc.x * fb;
+            O.y = O.y * fa + oc.y * fb;
+            O.z = O.z * fa + oc.z * fb;
+            O.w = O.w * fa + oc.w * fb;
+            M = Mn;
           }
-          float L = 0.f, O = 0.f;
-          for (int c = c_lo; c <= c_hi; ++c) {
-            if (sl.empty(c)) continue;
-            const int slot = (sl.lo(c) >= sg.start) ? 0 : 1;
-            const float* r = p.partials + ((int64_t)c * 2 + slot) * G * (D + 2) + gg * (D + 2);
-            const float mc = __ldcg(r + D);
-            const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-            L = fmaf(f, __ldcg(r + D + 1), L);
-            O = fmaf(f, __ldcg(r + d), O);
-          }
-          outp[idx] = L > 0.f ? O / L : 0.f;
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          *reinterpret_cast<float4*>(outp + gg * D + d) = make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
         }
       }
     }
@@ -1188,7 +1224,7 @@ cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   using C = Cfg<KB, VB, D>;
   static int configured_smem = 0;
   static int occ_smem = -1, occ_blocks = 0;
-  const int smem = C::smem_bytes(p.gqa, p.batch);
+  const int smem = C::smem_bytes(TOK, p.gqa, p.batch);
   if (smem > configured_smem) {
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);

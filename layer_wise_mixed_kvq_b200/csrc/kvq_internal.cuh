@@ -34,6 +34,10 @@ __host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D) {
   return code_block_bytes(kb, D) + code_block_bytes(vb, D) + (kb == 16 ? 0 : 4LL * D + 128);
 }
 
+// Tensor-core kernel split record: [G][D] accumulators, [G] maxima, [G] sums,
+// padded to 4 floats so every record starts 16-byte aligned.
+__host__ __device__ constexpr int split_record_floats(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
+
 struct LayerState {
   int kb = 0, vb = 0;
   int64_t page_bytes = 0;
@@ -74,7 +78,7 @@ struct DecodeParams {
   int chunk;             // CUDA-core kernel: pages per split
   int splits_stride;     // CUDA-core kernel: partial slots per (b, h)
   int n_units;           // tensor-core kernel: total units (pages + window/empty units), host view
-  int max_ctas;          // tensor-core kernel: CTAs the partial buffer can serve (2 records each)
+  int max_ctas;          // tensor-core kernel: CTAs the partial buffer can serve (2 split records each)
   int sm_count;
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)

@@ -127,7 +127,8 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.splits_stride = (int)std::max<int64_t>(stride, 1);
   p.batch = batch;
   p.n_units = (int)std::min<int64_t>(n_units, INT32_MAX);
-  p.max_ctas = (int)std::min<int64_t>(records / 2, INT32_MAX);
+  p.max_ctas = (int)std::min<int64_t>(
+      (int64_t)((kScratchBytes - ctr_bytes) / ((size_t)kvq::split_record_floats(G, head_dim) * 4)) / 2, INT32_MAX);
   p.sm_count = sms;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   e = kvq::launch_decode(pair.k_bits, pair.v_bits, head_dim, p, dim3(splits, n_kv_heads, batch), s);

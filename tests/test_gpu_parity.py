@@ -204,6 +204,22 @@ def test_split_count_does_not_change_results(kvq, oracle, split):
         P.close()
 
 
+@pytest.mark.parametrize("G", [1, 3, 5, 8])
+def test_split_segments_odd_gqa(kvq, oracle, G):
+    # more units than resident CTAs: slices hold the tail of one sequence-head and
+    # the head of the next, so both split records of a CTA and the final merge run
+    rng = np.random.default_rng(40 + G)
+    batch, hkv, T = 8, 2, 1790
+    P = Pair(kvq, oracle, (4, 4), batch, hkv * G, hkv, 128, T + 8)
+    try:
+        K, V = _inputs(rng, batch * T, hkv, 128)
+        P.append(K, V, [T] * batch)
+        got, ref = P.attend(_q(rng, batch, hkv * G, 128))
+        _check_attention(got, ref, f"G={G}")
+    finally:
+        P.close()
+
+
 def test_tiny_k8v4_workload(kvq, oracle):
     """The 1-layer K8V4 workload: batch 1, 2 = 2 heads, D 64, 256 tokens + 1."""
     w = synth.WORKLOADS["tiny_k8v4"]
