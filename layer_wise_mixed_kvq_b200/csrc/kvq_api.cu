@@ -114,6 +114,15 @@ cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 gri
   return simt ? launch_decode_simt(kb, vb, D, p, grid, s) : launch_decode_mma(kb, vb, D, p, s);
 }
 
+int seg_overhead_units() {
+  static const int v = [] {
+    const char* e = std::getenv("KVQ_SEG_OVERHEAD_UNITS");
+    int x = e ? std::atoi(e) : 16;
+    return x < 0 ? 0 : (x > 256 ? 256 : x);
+  }();
+  return v;
+}
+
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_p, int64_t stride) {
   const int64_t target_ctas = (int64_t)sm_count * 3;
   int64_t chunk = std::max<int64_t>(8, (total_pages + target_ctas - 1) / target_ctas);
@@ -352,7 +361,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
     int64_t T = L.host_len[b], P = T / kvq::kPageTokens;
     total_pages += P;
     max_p = std::max(max_p, P);
-    n_units += std::max<int64_t>(1, P + (T % kvq::kPageTokens ? 1 : 0));
+    n_units += std::max<int64_t>(1, P + (T % kvq::kPageTokens ? 1 : 0)) + kvq::seg_overhead_units();
   }
   total_pages *= c->n_kv_heads;
   n_units *= c->n_kv_heads;
@@ -388,6 +397,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
     p.max_ctas = (int)std::min<int64_t>(floats / kvq::split_record_floats(p.gqa, c->head_dim) / 2, INT32_MAX);
   }
   p.sm_count = c->sm_count;
+  p.seg_overhead = kvq::seg_overhead_units();
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

@@ -94,6 +94,29 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// L2 policy for data read exactly once (the streamed pages): evict first, so
+// the stream does not push out the small reused data (query rows, windows,
+// split records).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void bulk_load_once(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                               uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+// Bulk prefetch into L2 (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Device-scope fetch-add with acquire-release ordering: releases every write
 // this thread has observed (the CTA's partial records, via the preceding
 // barrier) and acquires the other CTAs' released records.
@@ -806,11 +829,14 @@ __device__ __forceinline__ void attend_window_tok(const __nv_bfloat16* win, int 
 }
 
 // ------------------------------------------------------------------ kernel --
-// Units: the pages of every (sequence b, KV head h) in order, followed by one
-// window unit when T mod 32 > 0 (or one empty unit when T = 0). Segment
-// (b, h) occupies units [ustart[b] + h * n_b, ... + n_b). The N units are cut
-// into gridDim.x balanced contiguous slices, one per CTA, so every CTA gets the
-// same amount of work whatever the sequence lengths.
+// Units: per (sequence b, KV head h) segment, V "overhead" units (no work:
+// they stand for the fixed cost of starting and merging a segment part, so a
+// CTA that spans several segments gets fewer pages), then the pages in order,
+// then one window unit when T mod 32 > 0 (or one empty unit when T = 0).
+// Segment (b, h) occupies units [ustart[b] + h * n_b, ... + n_b). The N units
+// are cut into gridDim.x balanced contiguous slices, one per CTA. A slice that
+// ends inside a segment's overhead units takes no part in that segment: the
+// segment's parts are held by the CTAs from the one owning unit start + V on.
 
 // Segment containing unit u.
 struct Seg {
@@ -850,7 +876,7 @@ struct Slicer {
 // within each segment part [a, e) of the CTA slice, units a + warp + 4j.
 struct PageCursor {
   int u, e;          // candidate unit, end of the current segment part
-  int seg_start, P;  // current segment's first unit and page count
+  int first, P;      // current segment's first page unit and page count
   const uint8_t* base;  // pages of the current (b, h)
 };
 
@@ -859,14 +885,15 @@ __device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p
                                             int warp) {
   for (;;) {
     if (c.u < c.e) {
-      if (c.u - c.seg_start < c.P) return true;
-      c.u += kWarps;  // the window / empty unit is the last of its segment
+      const int k = c.u - c.first;
+      if (k >= 0 && k < c.P) return true;
+      c.u += kWarps;  // overhead units lead a segment, the window / empty unit ends it
       continue;
     }
     if (c.e >= u1) return false;
     const int a = c.e;
     const Seg sg = seg_of(ustart, B, p.n_kv_heads, a);
-    c.seg_start = sg.start;
+    c.first = sg.start + p.seg_overhead;
     c.e = min(sg.start + sg.n, u1);
     c.P = p.len[sg.b] / kPageTokens;
     c.base = p.pages + ((int64_t)(sg.b * p.n_kv_heads + sg.h) * p.max_pages) * p.page_bytes;
@@ -908,7 +935,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
       if (bb < B) {
         const int T = p.len[bb];
         n = T / kPageTokens + (T % kPageTokens > 0 ? 1 : 0);
-        n = (n > 0 ? n : 1) * H;
+        n = ((n > 0 ? n : 1) + p.seg_overhead) * H;
       }
       int x = n;
 #pragma unroll
@@ -934,6 +961,11 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   const Slicer sl{N / (int)gridDim.x, N % (int)gridDim.x};
   const int u0 = sl.lo(blockIdx.x), u1 = sl.lo(blockIdx.x + 1);
   if (u0 >= u1) return;
+  {
+    // nothing to do when the whole slice lies in one segment's overhead units
+    const Seg s0 = seg_of(ustart, B, H, u0);
+    if (u1 <= s0.start + p.seg_overhead) return;
+  }
 
   // ---- query rows arrive by bulk copy (the first one ahead of the page stream)
   const uint32_t qbytes = (uint32_t)(G * D * 2);
@@ -948,15 +980,17 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   PageCursor cur;
   cur.u = u0;  // >= e: the first call looks up the segment of u0
   cur.e = u0;
-  cur.seg_start = 0;
+  cur.first = 0;
   cur.P = 0;
   cur.base = nullptr;
   int issued = 0;
+  const uint64_t pol = l2_evict_first_policy();
   if (lane == 0) {
     for (int r = 0; r < C::R; ++r) {
       if (!cursor_next<D>(cur, p, ustart, B, u1, warp)) break;
       mbar_expect_tx(&bars[r], C::PB);
-      bulk_load(ring + r * C::STAGE, cur.base + (int64_t)(cur.u - cur.seg_start) * p.page_bytes, C::PB, &bars[r]);
+      bulk_load_once(ring + r * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes, C::PB, &bars[r],
+                     pol);
       cur.u += kWarps;
       ++issued;
     }
@@ -968,13 +1002,21 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   for (int a = u0; a < u1; ++segi) {
     const Seg sg = seg_of(ustart, B, H, a);
     const int e = min(sg.start + sg.n, u1);
+    if (e <= sg.start + p.seg_overhead) break;  // overhead units only (the slice's last part)
     const int T = p.len[sg.b];
     const int P = T / kPageTokens, W = T % kPageTokens;
+    if (threadIdx.x == 0 && W > 0 && e == sg.start + sg.n) {
+      // this part ends with the bf16 window: bring its W key and W value rows into L2
+      const __nv_bfloat16* w0 = p.window + ((int64_t)(sg.b * H + sg.h) * 2) * kPageTokens * D;
+      prefetch_l2(w0, (uint32_t)(W * D * 2));
+      prefetch_l2(w0 + kPageTokens * D, (uint32_t)(W * D * 2));
+    }
     const bool qvalid = qh < G;
     {
       const bool got = mbar_wait(&qbars[segi & 1], (uint32_t)((segi >> 1) & 1));
       if (!__all_sync(0xffffffffu, got)) ok = false;
-      if (threadIdx.x == 0 && e < u1) issue_q(e, (segi + 1) & 1);  // prefetch the next segment's query
+      // prefetch the next segment's query row (unless that part is overhead units only)
+      if (threadIdx.x == 0 && e < u1 && u1 > e + p.seg_overhead) issue_q(e, (segi + 1) & 1);
     }
     const __nv_bfloat16* qrow = qbuf + (segi & 1) * kMaxGqa * D + (qvalid ? qh : 0) * D;
 
@@ -1059,7 +1101,8 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
 
     // ---- this warp's units of the segment part [a, e)
     for (int u = a + warp; u < e; u += kWarps) {
-      const int k = u - sg.start;
+      const int k = u - sg.start - p.seg_overhead;
+      if (k < 0) continue;  // overhead unit: no work
       if (k < P) {
         if (ok) {
           const int stage = consumed % C::R;
@@ -1080,8 +1123,8 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
             if (lane == 0 && cursor_next<D>(cur, p, ustart, B, u1, warp)) {
               fence_proxy_async();
               mbar_expect_tx(&bars[stage], C::PB);
-              bulk_load(ring + stage * C::STAGE, cur.base + (int64_t)(cur.u - cur.seg_start) * p.page_bytes, C::PB,
-                        &bars[stage]);
+              bulk_load_once(ring + stage * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes,
+                             C::PB, &bars[stage], pol);
               cur.u += kWarps;
               ++issued;
             }
@@ -1139,7 +1182,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
     }
     __syncthreads();
     const int seg = sg.b * H + sg.h;
-    const bool whole = (a == sg.start) && (e == sg.start + sg.n);
+    const bool whole = (a <= sg.start + p.seg_overhead) && (e == sg.start + sg.n);
     float* outp = p.out + (int64_t)seg * G * D;
     float* part = p.partials + ((int64_t)blockIdx.x * 2 + (a == u0 ? 0 : 1)) * split_record_floats(G, D);
     for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
@@ -1169,7 +1212,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
     if (!whole) {
       // The last CTA of a split segment merges the slices' partials in slice
       // order (empty slices, possible when CTAs outnumber units, hold nothing).
-      const int c_lo = sl.cta_of(sg.start), c_hi = sl.cta_of(sg.start + sg.n - 1);
+      const int c_lo = sl.cta_of(sg.start + p.seg_overhead), c_hi = sl.cta_of(sg.start + sg.n - 1);
       __syncthreads();  // this CTA's partial record is complete
       if (threadIdx.x == 0) {
         int parts = 0;

@@ -80,6 +80,7 @@ struct DecodeParams {
   int n_units;           // tensor-core kernel: total units (pages + window/empty units), host view
   int max_ctas;          // tensor-core kernel: CTAs the partial buffer can serve (2 split records each)
   int sm_count;
+  int seg_overhead;      // tensor-core kernel: overhead units leading each segment (>= 0)
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
 };
@@ -93,6 +94,9 @@ cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, cuda
 // Pages per split-K CTA for a layer-step: about 3 CTAs per SM, at least 8 pages
 // (2 per warp) per CTA, and no more than `stride` splits per (sequence, head).
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_pages_per_seq, int64_t stride);
+// Overhead units per segment for the tensor-core kernel's balanced slices
+// (KVQ_SEG_OVERHEAD_UNITS overrides the default).
+int seg_overhead_units();
 // Message returned by kvq_last_error() on this thread.
 void set_last_error(const std::string& msg);
 // Layer-map dispatcher: the kernel instance for a layer's pair.

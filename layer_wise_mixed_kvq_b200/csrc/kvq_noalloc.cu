@@ -105,7 +105,7 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   const int64_t stride = records / pairs;  // CUDA-core kernel: records per (sequence, head)
   const int64_t chunk = stride >= 1 ? kvq::choose_chunk(sms, max_p * pairs, max_p, stride) : max_p + 1;
   const int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
-  const int64_t n_units = pairs * (max_p + 1);
+  const int64_t n_units = pairs * (max_p + 1 + kvq::seg_overhead_units());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the merge counters must start at zero; the array keeps the last call's contents
   cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)pairs * 4, s);
@@ -130,6 +130,7 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.max_ctas = (int)std::min<int64_t>(
       (int64_t)((kScratchBytes - ctr_bytes) / ((size_t)kvq::split_record_floats(G, head_dim) * 4)) / 2, INT32_MAX);
   p.sm_count = sms;
+  p.seg_overhead = kvq::seg_overhead_units();
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   e = kvq::launch_decode(pair.k_bits, pair.v_bits, head_dim, p, dim3(splits, n_kv_heads, batch), s);
   if (e != cudaSuccess) return fail(KVQ_ECUDA, std::string("decode kernel launch: ") + cudaGetErrorString(e));
