@@ -49,14 +49,14 @@ def lib() -> ctypes.CDLL:
             "oracle_f32_to_f16_ru": (c.c_uint16, [c.c_float]),
             "oracle_f16_value": (c.c_double, [c.c_uint16]),
             "oracle_equiv_bits": (c.c_double, [P, P, c.c_int]),
-            "oracle_layer_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int64, c.c_int, c.c_int, c.c_int]),
+            "oracle_layer_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int, c.c_int, c.c_int]),
             "oracle_quantize": (None, [P, c.c_int, c.c_int, P, P, P]),
-            "oracle_page_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int]),
+            "oracle_page_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int, c.c_int]),
             "oracle_pack_block": (None, [P, P, c.c_int, c.c_int, c.c_int]),
             "oracle_unpack_block": (None, [P, P, c.c_int, c.c_int, c.c_int]),
-            "oracle_build_page": (None, [P, P, P, c.c_int, c.c_int, c.c_int]),
-            "oracle_dequant_page": (None, [P, c.c_int, c.c_int, c.c_int, P, P]),
-            "oracle_layer_new": (P, [c.c_int, c.c_int, c.c_int, c.c_int, c.c_int]),
+            "oracle_build_page": (None, [P, P, P, c.c_int, c.c_int, c.c_int, c.c_int]),
+            "oracle_dequant_page": (None, [P, c.c_int, c.c_int, c.c_int, c.c_int, P, P]),
+            "oracle_layer_new": (P, [c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int]),
             "oracle_layer_free": (None, [P]),
             "oracle_layer_len": (c.c_int64, [P, c.c_int]),
             "oracle_layer_append": (None, [P, P, P, P, c.c_int]),
@@ -111,13 +111,17 @@ def equiv_bits(pairs) -> float:
     return float(lib().oracle_equiv_bits(_ptr(k), _ptr(v), len(pairs)))
 
 
+#: key modes: per-channel keys over the 32-token group, or per-token keys
+KEY_PER_CHANNEL, KEY_PER_TOKEN = 0, 1
+
+
 def layer_bytes(k_bits: int, v_bits: int, tokens: int, n_kv_heads: int, head_dim: int,
-                with_meta: bool = False) -> int:
-    return int(lib().oracle_layer_bytes(k_bits, v_bits, tokens, n_kv_heads, head_dim, int(with_meta)))
+                with_meta: bool = False, key_mode: int = KEY_PER_CHANNEL) -> int:
+    return int(lib().oracle_layer_bytes(k_bits, v_bits, key_mode, tokens, n_kv_heads, head_dim, int(with_meta)))
 
 
-def page_bytes(k_bits: int, v_bits: int, head_dim: int) -> int:
-    return int(lib().oracle_page_bytes(k_bits, v_bits, head_dim))
+def page_bytes(k_bits: int, v_bits: int, head_dim: int, key_mode: int = KEY_PER_CHANNEL) -> int:
+    return int(lib().oracle_page_bytes(k_bits, v_bits, head_dim, key_mode))
 
 
 # -------------------------------------------------------------- quantizer --
@@ -146,19 +150,19 @@ def unpack_block(blk: np.ndarray, head_dim: int, bits: int, is_value: bool) -> n
 
 
 def build_page(k_bf16_bits: np.ndarray, v_bf16_bits: np.ndarray, head_dim: int, k_bits: int,
-               v_bits: int) -> np.ndarray:
+               v_bits: int, key_mode: int = KEY_PER_CHANNEL) -> np.ndarray:
     kb = np.ascontiguousarray(k_bf16_bits, dtype=np.uint16).reshape(32, head_dim)
     vb = np.ascontiguousarray(v_bf16_bits, dtype=np.uint16).reshape(32, head_dim)
-    page = np.zeros(page_bytes(k_bits, v_bits, head_dim), dtype=np.uint8)
-    lib().oracle_build_page(_ptr(page), _ptr(kb), _ptr(vb), head_dim, k_bits, v_bits)
+    page = np.zeros(page_bytes(k_bits, v_bits, head_dim, key_mode), dtype=np.uint8)
+    lib().oracle_build_page(_ptr(page), _ptr(kb), _ptr(vb), head_dim, k_bits, v_bits, key_mode)
     return page
 
 
-def dequant_page(page: np.ndarray, head_dim: int, k_bits: int, v_bits: int):
+def dequant_page(page: np.ndarray, head_dim: int, k_bits: int, v_bits: int, key_mode: int = KEY_PER_CHANNEL):
     page = np.ascontiguousarray(page, dtype=np.uint8)
     K = np.zeros((32, head_dim), dtype=np.float64)
     V = np.zeros((32, head_dim), dtype=np.float64)
-    lib().oracle_dequant_page(_ptr(page), head_dim, k_bits, v_bits, _ptr(K), _ptr(V))
+    lib().oracle_dequant_page(_ptr(page), head_dim, k_bits, v_bits, key_mode, _ptr(K), _ptr(V))
     return K, V
 
 
@@ -166,10 +170,11 @@ def dequant_page(page: np.ndarray, head_dim: int, k_bits: int, v_bits: int):
 class OracleLayer:
     """One layer's KV cache for `batch` sequences, mirroring the library's semantics."""
 
-    def __init__(self, k_bits: int, v_bits: int, batch: int, n_kv_heads: int, head_dim: int):
-        self.k_bits, self.v_bits = k_bits, v_bits
+    def __init__(self, k_bits: int, v_bits: int, batch: int, n_kv_heads: int, head_dim: int,
+                 key_mode: int = KEY_PER_CHANNEL):
+        self.k_bits, self.v_bits, self.key_mode = k_bits, v_bits, key_mode
         self.batch, self.n_kv_heads, self.head_dim = batch, n_kv_heads, head_dim
-        self._h = lib().oracle_layer_new(k_bits, v_bits, batch, n_kv_heads, head_dim)
+        self._h = lib().oracle_layer_new(k_bits, v_bits, key_mode, batch, n_kv_heads, head_dim)
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -17,6 +17,10 @@
 //    MiB, FP8 layer half of it, scales and metadata ignored).
 //  * key quantizer -- per-channel asymmetric over a token group (facts page;
 //    OpenReview rebuttal on KIVI's per-channel per-group keys); group = 32.
+//    Second key mode: per-token asymmetric, one (scale, zero) per key token over
+//    the head dimension, exactly like values (OpenReview rebuttal, section 4
+//    "Per-channel vs. per-token quantization"; facts page: the two modes give
+//    different Pareto-optimal pairs). The mode is a per-layer setting.
 //  * value quantizer -- per-token asymmetric (OpenReview rebuttal, "value
 //    per-token-asym").
 //  * only new tokens are quantized, with the layer's fixed pair (OpenReview
@@ -35,6 +39,8 @@
 //  * fp32 inputs are rounded to bf16 (round-to-nearest-even) at entry.
 //  * q head h reads KV head h / (Hq/Hkv); softmax scale 1/sqrt(D); no mask.
 //  * empty sequence: output 0.
+//  * per-token key mode keeps the same 32-token pages and bf16 residual window:
+//    a key token is quantized when its page fills, like a value token.
 //
 // The packed page layout implemented here is the library's documented storage
 // format (written out independently below from its definition).
@@ -160,6 +166,8 @@ void quantize_set(const float* x, int n, int bits, uint8_t* codes,
 // One page = 32 consecutive tokens of one (sequence, KV head):
 //   [K code block][V code block][K scales (D fp16)][K zeros (D fp16)]
 //   [V scales (32 fp16)][V zeros (32 fp16)]          (quantized pair)
+//   per-token key mode: [K scales (32 fp16)][K zeros (32 fp16)] in token order
+//   take the place of the D key scales and zeros
 //   [K block (bf16)][V block (bf16)]                 (bf16 layer)
 // A code block is split into 16x16 tiles f = 2*dt + tt (dt: 16-dim tile,
 // tt: 16-token tile). In tile f, lane l = 4g + t owns 8 elements e = 2p + j:
@@ -194,9 +202,10 @@ int64_t word_byte(int lane, int64_t w) { return ((w / 4) * 32 + lane) * 16 + (w 
 
 int64_t code_block_bytes(int bits, int D) { return (int64_t)32 * D * bits / 8; }
 
-int64_t page_bytes(int kb, int vb, int D) {
+// key_mode: 0 = per-channel keys (D scale/zero pairs), 1 = per-token keys (32).
+int64_t page_bytes(int kb, int vb, int D, int key_mode) {
   int64_t b = code_block_bytes(kb, D) + code_block_bytes(vb, D);
-  if (kb != 16) b += (int64_t)4 * D + 128;
+  if (kb != 16) b += (key_mode ? 128 : (int64_t)4 * D) + 128;
   return b;
 }
 
@@ -260,8 +269,8 @@ void unpack_block(const uint8_t* blk, uint16_t* vals, int D, int bits, bool is_v
 }
 
 // Build one page from 32 tokens of bf16 keys/values ([32][D] bit patterns).
-void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb) {
-  std::memset(page, 0, (size_t)page_bytes(kb, vb, D));
+void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb, int key_mode) {
+  std::memset(page, 0, (size_t)page_bytes(kb, vb, D, key_mode));
   uint8_t* kblk = page;
   uint8_t* vblk = page + code_block_bytes(kb, D);
   if (kb == 16) {
@@ -269,19 +278,32 @@ void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, 
     pack_block(vblk, vbf, D, 16, true);
     return;
   }
+  const int nk = key_mode ? 32 : D;  // key scale/zero pairs in the page
   uint8_t* kscale = vblk + code_block_bytes(vb, D);
-  uint8_t* kzero = kscale + 2 * D;
-  uint8_t* vscale = kzero + 2 * D;
+  uint8_t* kzero = kscale + 2 * nk;
+  uint8_t* vscale = kzero + 2 * nk;
   uint8_t* vzero = vscale + 64;
   std::vector<uint16_t> kc(32 * D), vc(32 * D);
   std::vector<float> col(32), row(D);
   std::vector<uint8_t> codes(std::max(32, D));
   std::vector<uint16_t> ks(D), kz(D);
-  // keys: one set per channel over the page's 32 tokens
-  for (int d = 0; d < D; ++d) {
-    for (int t = 0; t < 32; ++t) col[t] = bf16_to_f32(kbf[t * D + d]);
-    quantize_set(col.data(), 32, kb, codes.data(), &ks[d], &kz[d]);
-    for (int t = 0; t < 32; ++t) kc[t * D + d] = codes[t];
+  if (key_mode) {
+    // keys: one set per token over the head dimension
+    for (int t = 0; t < 32; ++t) {
+      for (int d = 0; d < D; ++d) row[d] = bf16_to_f32(kbf[t * D + d]);
+      uint16_t sb, zb;
+      quantize_set(row.data(), D, kb, codes.data(), &sb, &zb);
+      for (int d = 0; d < D; ++d) kc[t * D + d] = codes[d];
+      std::memcpy(kscale + 2 * t, &sb, 2);
+      std::memcpy(kzero + 2 * t, &zb, 2);
+    }
+  } else {
+    // keys: one set per channel over the page's 32 tokens
+    for (int d = 0; d < D; ++d) {
+      for (int t = 0; t < 32; ++t) col[t] = bf16_to_f32(kbf[t * D + d]);
+      quantize_set(col.data(), 32, kb, codes.data(), &ks[d], &kz[d]);
+      for (int t = 0; t < 32; ++t) kc[t * D + d] = codes[t];
+    }
   }
   // values: one set per token over the head dimension
   for (int t = 0; t < 32; ++t) {
@@ -294,15 +316,17 @@ void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, 
   }
   pack_block(kblk, kc.data(), D, kb, false);
   pack_block(vblk, vc.data(), D, vb, true);
-  for (int i = 0; i < D; ++i) {
-    int d = kmeta_channel(i, D);
-    std::memcpy(kscale + 2 * i, &ks[d], 2);
-    std::memcpy(kzero + 2 * i, &kz[d], 2);
+  if (!key_mode) {
+    for (int i = 0; i < D; ++i) {
+      int d = kmeta_channel(i, D);
+      std::memcpy(kscale + 2 * i, &ks[d], 2);
+      std::memcpy(kzero + 2 * i, &kz[d], 2);
+    }
   }
 }
 
 // Dequantize one page into [32][D] doubles (x = code * s + z, exact in fp64).
-void dequant_page(const uint8_t* page, int D, int kb, int vb, double* Kh, double* Vh) {
+void dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, double* Kh, double* Vh) {
   std::vector<uint16_t> kc(32 * D), vc(32 * D);
   const uint8_t* kblk = page;
   const uint8_t* vblk = page + code_block_bytes(kb, D);
@@ -312,21 +336,32 @@ void dequant_page(const uint8_t* page, int D, int kb, int vb, double* Kh, double
     for (int i = 0; i < 32 * D; ++i) { Kh[i] = bf16_to_f32(kc[i]); Vh[i] = bf16_to_f32(vc[i]); }
     return;
   }
+  const int nk = key_mode ? 32 : D;
   const uint8_t* kscale = vblk + code_block_bytes(vb, D);
-  const uint8_t* kzero = kscale + 2 * D;
-  const uint8_t* vscale = kzero + 2 * D;
+  const uint8_t* kzero = kscale + 2 * nk;
+  const uint8_t* vscale = kzero + 2 * nk;
   const uint8_t* vzero = vscale + 64;
-  std::vector<double> s(D), z(D);
-  for (int i = 0; i < D; ++i) {
-    uint16_t sb, zb;
-    std::memcpy(&sb, kscale + 2 * i, 2);
-    std::memcpy(&zb, kzero + 2 * i, 2);
-    int d = kmeta_channel(i, D);
-    s[d] = f16_value(sb);
-    z[d] = f16_value(zb);
+  if (key_mode) {
+    for (int t = 0; t < 32; ++t) {
+      uint16_t sb, zb;
+      std::memcpy(&sb, kscale + 2 * t, 2);
+      std::memcpy(&zb, kzero + 2 * t, 2);
+      double ks = f16_value(sb), kz = f16_value(zb);
+      for (int d = 0; d < D; ++d) Kh[t * D + d] = (double)kc[t * D + d] * ks + kz;
+    }
+  } else {
+    std::vector<double> s(D), z(D);
+    for (int i = 0; i < D; ++i) {
+      uint16_t sb, zb;
+      std::memcpy(&sb, kscale + 2 * i, 2);
+      std::memcpy(&zb, kzero + 2 * i, 2);
+      int d = kmeta_channel(i, D);
+      s[d] = f16_value(sb);
+      z[d] = f16_value(zb);
+    }
+    for (int t = 0; t < 32; ++t)
+      for (int d = 0; d < D; ++d) Kh[t * D + d] = (double)kc[t * D + d] * s[d] + z[d];
   }
-  for (int t = 0; t < 32; ++t)
-    for (int d = 0; d < D; ++d) Kh[t * D + d] = (double)kc[t * D + d] * s[d] + z[d];
   for (int t = 0; t < 32; ++t) {
     uint16_t sb, zb;
     std::memcpy(&sb, vscale + 2 * t, 2);
@@ -345,7 +380,7 @@ struct Seq {
 };
 
 struct Layer {
-  int kb, vb, batch, hkv, D;
+  int kb, vb, key_mode, batch, hkv, D;
   std::vector<Seq> seqs;
 };
 
@@ -369,12 +404,14 @@ double oracle_equiv_bits(const uint8_t* kbits, const uint8_t* vbits, int n_layer
 
 // Bytes of one layer's K and V for `tokens` tokens per KV head: codes only
 // (with_meta = 0, the idealised count of the worked example), or codes plus
-// fp16 scale/zero (2 bytes each: D/32 key pairs and one value pair per token).
-int64_t oracle_layer_bytes(int kbits, int vbits, int64_t tokens, int n_kv_heads, int head_dim,
+// fp16 scale/zero (2 bytes each: D/32 key pairs -- one key pair in per-token key
+// mode -- and one value pair per token).
+int64_t oracle_layer_bytes(int kbits, int vbits, int key_mode, int64_t tokens, int n_kv_heads, int head_dim,
                            int with_meta) {
   int64_t bits = tokens * n_kv_heads * (int64_t)head_dim * (kbits + vbits);
   int64_t bytes = bits / 8;
-  if (with_meta && kbits != 16) bytes += tokens * n_kv_heads * ((int64_t)head_dim * 4 / 32 + 4);
+  if (with_meta && kbits != 16)
+    bytes += tokens * n_kv_heads * ((key_mode ? 4 : (int64_t)head_dim * 4 / 32) + 4);
   return bytes;
 }
 
@@ -383,7 +420,7 @@ void oracle_quantize(const float* x, int n, int bits, uint8_t* codes, uint16_t* 
   quantize_set(x, n, bits, codes, scale_bits, zero_bits);
 }
 
-int64_t oracle_page_bytes(int kb, int vb, int D) { return page_bytes(kb, vb, D); }
+int64_t oracle_page_bytes(int kb, int vb, int D, int key_mode) { return page_bytes(kb, vb, D, key_mode); }
 
 // Pack/unpack one code block (vals [32][D]); is_value selects the V tiling.
 void oracle_pack_block(uint8_t* blk, const uint16_t* vals, int D, int bits, int is_value) {
@@ -394,16 +431,17 @@ void oracle_unpack_block(const uint8_t* blk, uint16_t* vals, int D, int bits, in
   unpack_block(blk, vals, D, bits, is_value != 0);
 }
 
-void oracle_build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb) {
-  build_page(page, kbf, vbf, D, kb, vb);
+void oracle_build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb,
+                       int key_mode) {
+  build_page(page, kbf, vbf, D, kb, vb, key_mode);
 }
-void oracle_dequant_page(const uint8_t* page, int D, int kb, int vb, double* Kh, double* Vh) {
-  dequant_page(page, D, kb, vb, Kh, Vh);
+void oracle_dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, double* Kh, double* Vh) {
+  dequant_page(page, D, kb, vb, key_mode, Kh, Vh);
 }
 
 // ---- one-layer cache simulator -------------------------------------------
-void* oracle_layer_new(int kb, int vb, int batch, int n_kv_heads, int head_dim) {
-  Layer* L = new Layer{kb, vb, batch, n_kv_heads, head_dim, {}};
+void* oracle_layer_new(int kb, int vb, int key_mode, int batch, int n_kv_heads, int head_dim) {
+  Layer* L = new Layer{kb, vb, kb == 16 ? 0 : key_mode, batch, n_kv_heads, head_dim, {}};
   L->seqs.resize(batch);
   for (auto& s : L->seqs) {
     s.pages.resize(n_kv_heads);
@@ -424,7 +462,7 @@ int64_t oracle_layer_len(void* p, int b) { return static_cast<Layer*>(p)->seqs[b
 void oracle_layer_append(void* p, const float* K, const float* V, const int32_t* n_new, int batch) {
   Layer* L = static_cast<Layer*>(p);
   const int D = L->D, H = L->hkv;
-  const int64_t pb = page_bytes(L->kb, L->vb, D);
+  const int64_t pb = page_bytes(L->kb, L->vb, D, L->key_mode);
   int64_t row = 0;
   for (int b = 0; b < batch; ++b) {
     Seq& s = L->seqs[b];
@@ -439,7 +477,7 @@ void oracle_layer_append(void* p, const float* K, const float* V, const int32_t*
         if ((int64_t)s.wk[h].size() == 32LL * D) {
           size_t off = s.pages[h].size();
           s.pages[h].resize(off + pb);
-          build_page(s.pages[h].data() + off, s.wk[h].data(), s.wv[h].data(), D, L->kb, L->vb);
+          build_page(s.pages[h].data() + off, s.wk[h].data(), s.wv[h].data(), D, L->kb, L->vb, L->key_mode);
           s.wk[h].clear();
           s.wv[h].clear();
         }
@@ -479,10 +517,10 @@ void oracle_layer_dequant(void* p, int b, int h, double* Kh, double* Vh) {
   Layer* L = static_cast<Layer*>(p);
   const int D = L->D;
   const Seq& s = L->seqs[b];
-  const int64_t pb = page_bytes(L->kb, L->vb, D);
+  const int64_t pb = page_bytes(L->kb, L->vb, D, L->key_mode);
   int64_t npages = (int64_t)s.pages[h].size() / pb;
   for (int64_t pg = 0; pg < npages; ++pg)
-    dequant_page(s.pages[h].data() + pg * pb, D, L->kb, L->vb, Kh + pg * 32 * D, Vh + pg * 32 * D);
+    dequant_page(s.pages[h].data() + pg * pb, D, L->kb, L->vb, L->key_mode, Kh + pg * 32 * D, Vh + pg * 32 * D);
   int64_t base = npages * 32 * D;
   for (size_t i = 0; i < s.wk[h].size(); ++i) {
     Kh[base + i] = bf16_to_f32(s.wk[h][i]);
