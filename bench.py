@@ -146,7 +146,8 @@ def cpu_baseline(w, seconds):
     ctx = int(synth.context_lengths(w, 1)[0])
     while t_attn < seconds and samples < 64:
         pair = w.layer_map[layer % w.n_layers]
-        L = oracle.OracleLayer(pair[0], pair[1], 1, w.n_kv_heads, w.head_dim)
+        key_mode = pair[2] if len(pair) > 2 else 0
+        L = oracle.OracleLayer(pair[0], pair[1], 1, w.n_kv_heads, w.head_dim, key_mode=key_mode)
         K, V = synth.kv_tokens(w, layer, ctx + 1)
         L.append(K, V, [ctx + 1])
         Q = synth.queries(w, layer, batch=1)
@@ -155,7 +156,7 @@ def cpu_baseline(w, seconds):
         t_attn += time.perf_counter() - t0
         T = ctx + 1
         P, W = T // 32, T % 32
-        page = oracle.page_bytes(pair[0], pair[1], w.head_dim)
+        page = oracle.page_bytes(pair[0], pair[1], w.head_dim, key_mode)
         done_bytes += w.n_kv_heads * (P * page + W * w.head_dim * 4)
         samples += 1
         layer += 1

@@ -49,12 +49,25 @@ extern "C" {
 
 typedef struct kvq_cache kvq_cache;
 
+/* Key quantization mode of a layer ([rebut] section 4 "Per-channel vs.
+ * per-token quantization"; [facts]: per-channel asymmetric keys beat per-token
+ * asymmetric keys on channel-outlier keys, and the Pareto-optimal pairs differ
+ * between the two modes). */
+typedef enum {
+  KVQ_KEY_PER_CHANNEL = 0, /* one scale/zero per key channel over each 32-token group (KIVI-like) */
+  KVQ_KEY_PER_TOKEN = 1    /* one scale/zero per key token over head_dim (per-token-asym) */
+} kvq_key_mode;
+
 /* One layer's precision pair: k_bits, v_bits in {2, 4, 8}, or {16, 16} for a
  * layer kept in bf16 ([qa] section 2: sensitive layers stay BF16; [facts]:
- * vLLM-style skip layers). Mixed bf16/int pairs are rejected. */
+ * vLLM-style skip layers). Mixed bf16/int pairs are rejected. key_mode is a
+ * kvq_key_mode (must be KVQ_KEY_PER_CHANNEL, i.e. 0, for a bf16 layer);
+ * reserved must be 0. A zero-initialised pair field means per-channel keys. */
 typedef struct {
   uint8_t k_bits;
   uint8_t v_bits;
+  uint8_t key_mode;
+  uint8_t reserved;
 } kvq_pair;
 
 typedef enum {
@@ -77,6 +90,8 @@ typedef enum {
  * row = slot = token mod 32). A page is 16-byte aligned and holds
  *   quantized pair: [K codes 4*D*k_bits B][V codes 4*D*v_bits B]
  *                   [K scale D x fp16][K zero D x fp16][V scale 32 x fp16][V zero 32 x fp16]
+ *   per-token keys: [K codes][V codes][K scale 32 x fp16][K zero 32 x fp16][V scale][V zero]
+ *                   (key scales and zeros in token order, like the values')
  *   bf16 layer:     [K 64*D B][V 64*D B]
  * Code blocks are stored as 16x16 tiles f = 2*dt + tt (dt: 16-channel tile,
  * tt: 16-token tile) laid out so that lane l = 4g + t of a warp reads its eight
@@ -86,8 +101,8 @@ typedef enum {
  * ((w/4)*32 + l)*16 + (w%4)*4; 8-bit tiles take two words (element e in byte e),
  * 4-bit tiles one word (nibble (e>>1) + 4*(e&1)), two 2-bit tiles share a word
  * (slot 4u + (e>>1) + 8*(e&1) for tile 2w+u), bf16 tiles four words (half e).
- * Key scale/zero entry i holds channel 16*dt + 2t + (j&1) + 8*(j>>1) with
- * t = i/(D/4), dt = (i%(D/4))/4, j = i%4.
+ * Key scale/zero entry i (per-channel keys) holds channel 16*dt + 2t + (j&1) +
+ * 8*(j>>1) with t = i/(D/4), dt = (i%(D/4))/4, j = i%4.
  */
 
 /* Bytes of one 32-token page of `pair` at head_dim D (0 if invalid). */
@@ -132,8 +147,9 @@ kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
  *   n_new: host array [batch], each >= 0.
  * Tokens enter the bf16 window; every time a sequence's window reaches 32
  * tokens they are quantized as one group -- keys per channel over the 32
- * tokens, values per token over head_dim ([facts]: per-channel asymmetric keys,
- * per-token asymmetric values) -- bit-packed into the next page, and the window
+ * tokens (per token over head_dim in a KVQ_KEY_PER_TOKEN layer), values per
+ * token over head_dim ([facts]: per-channel asymmetric keys, per-token
+ * asymmetric values) -- bit-packed into the next page, and the window
  * is emptied. The stored result does not depend on how tokens are split across
  * calls. Quantizer: z = fp16 round-down(min), s = fp16 round-up((max - z)/qmax),
  * code = clamp(rint((x - z) * (1/s)), 0, 2^bits - 1); all fp32 steps are single

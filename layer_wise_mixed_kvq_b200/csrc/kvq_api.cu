@@ -31,7 +31,9 @@ kvq_status cuda_fail(cudaError_t e, const char* what) {
 
 bool valid_pair(kvq_pair p) {
   auto ok = [](int b) { return b == 2 || b == 4 || b == 8; };
-  return (p.k_bits == 16 && p.v_bits == 16) || (ok(p.k_bits) && ok(p.v_bits));
+  if (p.reserved != 0 || p.key_mode > KVQ_KEY_PER_TOKEN) return false;
+  if (p.k_bits == 16 && p.v_bits == 16) return p.key_mode == KVQ_KEY_PER_CHANNEL;
+  return ok(p.k_bits) && ok(p.v_bits);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -58,8 +60,9 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
   if (!map || n_layers <= 0) { why = "layer_map is null or n_layers <= 0"; return false; }
   for (int l = 0; l < n_layers; ++l)
     if (!valid_pair(map[l])) {
-      why = "layer " + std::to_string(l) + " has an unsupported pair (k_bits, v_bits) = (" +
-            std::to_string(map[l].k_bits) + ", " + std::to_string(map[l].v_bits) + ")";
+      why = "layer " + std::to_string(l) + " has an unsupported pair (k_bits, v_bits, key_mode, reserved) = (" +
+            std::to_string(map[l].k_bits) + ", " + std::to_string(map[l].v_bits) + ", " +
+            std::to_string(map[l].key_mode) + ", " + std::to_string(map[l].reserved) + ")";
       return false;
     }
   if (head_dim != 64 && head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
@@ -73,7 +76,7 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
   g.max_pages = max_tokens / kvq::kPageTokens;
   size_t total = 0;
   for (int l = 0; l < n_layers; ++l) {
-    size_t pb = (size_t)kvq::page_bytes_of(map[l].k_bits, map[l].v_bits, head_dim);
+    size_t pb = (size_t)kvq::page_bytes_of(map[l].k_bits, map[l].v_bits, head_dim, map[l].key_mode);
     size_t pr = round_up((size_t)max_batch * n_kv_heads * std::max<int64_t>(g.max_pages, 1) * pb);
     size_t wr = round_up((size_t)max_batch * n_kv_heads * 2 * kvq::kPageTokens * head_dim * 2);
     g.page_region.push_back(pr);
@@ -149,7 +152,7 @@ const char* kvq_status_string(kvq_status s) {
 
 int64_t kvq_page_bytes(kvq_pair pair, int head_dim) {
   if (!valid_pair(pair) || (head_dim != 64 && head_dim != 128)) return 0;
-  return kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim);
+  return kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim, pair.key_mode);
 }
 
 double kvq_equiv_bits(const kvq_pair* map, int n_layers) {
@@ -216,7 +219,8 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     kvq::LayerState& L = c->layers[l];
     L.kb = map[l].k_bits;
     L.vb = map[l].v_bits;
-    L.page_bytes = kvq::page_bytes_of(L.kb, L.vb, head_dim);
+    L.km = map[l].key_mode;
+    L.page_bytes = kvq::page_bytes_of(L.kb, L.vb, head_dim, L.km);
     L.pages = p;
     p += g.page_region[l];
     L.window = reinterpret_cast<__nv_bfloat16*>(p);
@@ -318,6 +322,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
   p.page_bytes = L.page_bytes;
   p.max_pages = (int)c->max_pages;
   p.n_kv_heads = c->n_kv_heads;
+  p.key_mode = L.km;
   p.plan = nullptr;
   if (!all_one) {
     // multi-token append: per-sequence plan (start, count, row offset, items)
@@ -398,6 +403,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   }
   p.sm_count = c->sm_count;
   p.seg_overhead = kvq::seg_overhead_units();
+  p.key_mode = L.km;
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

@@ -5,7 +5,9 @@
 // keys and values are quantized online, with the layer's calibrated precision
 // pair. Keys are quantized per channel and values per token, both asymmetric
 // (llms-explorer facts page; rebuttal "key per-channel-asym and value
-// per-token-asym"). The group size (32 tokens) and the fp16 scale/zero format
+// per-token-asym"); a layer in per-token key mode quantizes its keys per token
+// like its values (rebuttal section 4, "Per-channel vs. per-token
+// quantization"). The group size (32 tokens) and the fp16 scale/zero format
 // are this library's choices.
 //
 // Grid (items, n_kv_heads, batch), 128 threads. Work item i of (b, h) quantizes
@@ -223,13 +225,42 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         xs[1][t][d] = __bfloat162float(vx);
       }
       __syncthreads();
+      const bool per_token_keys = a.key_mode != 0;
+      const int nk = per_token_keys ? kPageTokens : D;  // key scale/zero pairs
       uint8_t* vblk = page + code_block_bytes(KB, D);
       __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
-      __half* kzero = kscale + D;
-      __half* vscale = kzero + D;
+      __half* kzero = kscale + nk;
+      __half* vscale = kzero + nk;
       __half* vzero = vscale + kPageTokens;
-      // keys: one thread per channel, over the group's 32 tokens
-      for (int d = threadIdx.x; d < D; d += kThreads) {
+      // one warp per token over the head dimension: row r of xs (0 keys, 1 values)
+      auto quantize_tokens = [&](int r, int qmax, __half* sdst, __half* zdst) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        for (int t = warp; t < kPageTokens; t += kThreads / 32) {
+          float mn = xs[r][t][lane], mx = mn;
+#pragma unroll
+          for (int k = 1; k < D / 32; ++k) {
+            float x = xs[r][t][lane + 32 * k];
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          QParams q = make_qparams(mn, mx, qmax);
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k)
+            cs[r][t][lane + 32 * k] = (uint8_t)quant_code(xs[r][t][lane + 32 * k], q, qmax);
+          if (lane == 0) {
+            sdst[t] = q.s_h;
+            zdst[t] = q.z_h;
+          }
+        }
+      };
+      if (per_token_keys) quantize_tokens(0, (1 << KB) - 1, kscale, kzero);
+      // keys (per-channel mode): one thread per channel, over the group's 32 tokens
+      for (int d = threadIdx.x; d < (per_token_keys ? 0 : D); d += kThreads) {
         constexpr int qmax = (1 << KB) - 1;
         float mn = xs[0][0][d], mx = mn;
 #pragma unroll 8
@@ -246,32 +277,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         kzero[slot] = q.z_h;
       }
       // values: one warp per token, over the head dimension
-      {
-        constexpr int qmax = (1 << VB) - 1;
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        for (int t = warp; t < kPageTokens; t += kThreads / 32) {
-          float mn = xs[1][t][lane], mx = mn;
-#pragma unroll
-          for (int k = 1; k < D / 32; ++k) {
-            float x = xs[1][t][lane + 32 * k];
-            mn = fminf(mn, x);
-            mx = fmaxf(mx, x);
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          }
-          QParams q = make_qparams(mn, mx, qmax);
-#pragma unroll
-          for (int k = 0; k < D / 32; ++k)
-            cs[1][t][lane + 32 * k] = (uint8_t)quant_code(xs[1][t][lane + 32 * k], q, qmax);
-          if (lane == 0) {
-            vscale[t] = q.s_h;
-            vzero[t] = q.z_h;
-          }
-        }
-      }
+      quantize_tokens(1, (1 << VB) - 1, vscale, vzero);
       __syncthreads();
       store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
       store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });

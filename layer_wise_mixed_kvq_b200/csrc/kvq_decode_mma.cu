@@ -170,11 +170,12 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ------------------------------------------------------------ configuration --
-template <int KB, int VB, int D>
+// PT: per-token key mode (32 key scales/zeros per page instead of D).
+template <int KB, int VB, int D, bool PT = false>
 struct Cfg {
   static constexpr bool kBf16 = (KB == 16);
   static constexpr int KS = D / 16;                       // 16-channel tiles
-  static constexpr int PB = (int)page_bytes_of(KB, VB, D);
+  static constexpr int PB = (int)page_bytes_of(KB, VB, D, PT ? 1 : 0);
   // small pages: 3 CTAs per SM with 3-4 stages per warp; larger ones: 2 CTAs per SM
   static constexpr int MINB = PB <= 5000 ? 3 : 2;      // head-row kernel (64 accumulators per lane)
   static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;  // token-row kernel (32 accumulators per lane)
@@ -391,6 +392,86 @@ __device__ __forceinline__ void attend_qpage(const uint8_t* page, WarpState<D>& 
   softmax_update<D>(st, sc, tau);
 
   // --- PV: A = p' (hi/lo) per 16-token k-step, B = value codes
+  uint32_t pa[2][4];
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const int t0 = 16 * ks + 2 * t, t1 = t0 + 8;
+    const float2 s0 = *reinterpret_cast<const float2*>(svf + t0);
+    const float2 s1 = *reinterpret_cast<const float2*>(svf + t1);
+    const float2 z0 = *reinterpret_cast<const float2*>(zvf + t0);
+    const float2 z1 = *reinterpret_cast<const float2*>(zvf + t1);
+    const float p0 = sc[4 * ks + 0], p1 = sc[4 * ks + 1], p2 = sc[4 * ks + 2], p3 = sc[4 * ks + 3];
+    split_f16(p0 * s0.x, p1 * s0.y, pa[ks][0], pa[ks][1]);
+    split_f16(p2 * s1.x, p3 * s1.y, pa[ks][2], pa[ks][3]);
+    st.vz = fmaf(p0, z0.x, fmaf(p1, z0.y, fmaf(p2, z1.x, fmaf(p3, z1.y, st.vz))));
+  }
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<VB>::N];
+    load_tile_words<VB>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t b[4];
+      tile_frags<VB>(w, ks, b);
+      mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
+      mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
+    }
+  }
+}
+
+// Per-token keys, head rows: score of head g, token t = s_t * sum_c q'_c code_tc
+// + z_t * sum_c q'_c. The A operand is the segment's q' hi/lo fragments in
+// shared memory (2-bit tauK already folded in); no key-scale table, no z-term MMA.
+template <int KB, int VB, int D>
+__device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D>& st, const uint32_t* qz,
+                                                float qsum, float* wscr, int lane) {
+  using C = Cfg<KB, VB, D, true>;
+  const int t = lane & 3;
+  const uint8_t* vblk = page + code_block_bytes(KB, D);
+  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
+  const __half* kzero = kscale + kPageTokens;
+  const __half* vscale = kzero + kPageTokens;
+  const __half* vzero = vscale + kPageTokens;
+  float* kst = wscr;                   // [32] key scales x 2^24 (/ sigmaK on tokens with bit 3 set)
+  float* kzt = wscr + kPageTokens;     // [32] key zeros
+  float* svf = wscr + 4 * C::KSROW;    // [32] value scales, tauV folded
+  float* zvf = svf + kPageTokens;      // [32] value zeros
+  kst[lane] = __half2float(kscale[lane]) * ((lane & 8) ? kTwo24 / C::sigmaK : kTwo24);
+  kzt[lane] = __half2float(kzero[lane]);
+  const float vs = __half2float(vscale[lane]);
+  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
+  zvf[lane] = __half2float(vzero[lane]);
+  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
+  __syncwarp();
+
+  float s4[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s4[j][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<KB>::N];
+    load_tile_words<KB>(page, lane, dt, w);
+    const uint4 a = *reinterpret_cast<const uint4*>(qz + (dt * 32 + lane) * 4);
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      uint32_t b[4];
+      tile_frags<KB>(w, tt, b);
+      mma_f16(s4[2 * tt], a.x, a.y, a.z, a.w, b[0], b[1]);
+      mma_f16(s4[2 * tt + 1], a.x, a.y, a.z, a.w, b[2], b[3]);
+    }
+  }
+  float sc[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int tok = 8 * j + 2 * t + jj;
+      sc[2 * j + jj] = fmaf(s4[j][jj] + s4[j][jj + 2], kst[tok], kzt[tok] * qsum);
+    }
+  softmax_update<D>(st, sc, tau);
+
   uint32_t pa[2][4];
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
@@ -734,6 +815,78 @@ __device__ __forceinline__ void attend_qpage_tok(const uint8_t* page, TokState<D
   }
 }
 
+// Per-token keys, token rows: B = the segment's q' parts (tauK folded, fixed per
+// segment); score of token g + 8i for head t = s * acc + z * sum_c q'_c.
+template <int KB, int VB, int D>
+__device__ __forceinline__ void attend_qpage_tok_pt(const uint8_t* page, TokState<D>& st,
+                                                    const uint32_t (&qkb)[D / 8], float qsum, float* wscr,
+                                                    float partf, int lane) {
+  using C = Cfg<KB, VB, D, true>;
+  const int g = lane >> 2;
+  const uint8_t* vblk = page + code_block_bytes(KB, D);
+  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
+  const __half* kzero = kscale + kPageTokens;
+  const __half* vscale = kzero + kPageTokens;
+  const __half* vzero = vscale + kPageTokens;
+  float* kst = wscr;
+  float* kzt = wscr + kPageTokens;
+  float* svf = wscr + 4 * C::KSROW;
+  float* zvf = svf + kPageTokens;
+  float* ptr = zvf + kPageTokens;  // [4][40]
+  kst[lane] = __half2float(kscale[lane]) * ((lane & 8) ? kTwo24 / C::sigmaK : kTwo24);
+  kzt[lane] = __half2float(kzero[lane]);
+  const float vs = __half2float(vscale[lane]);
+  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
+  zvf[lane] = __half2float(vzero[lane]);
+  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
+  __syncwarp();
+
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<KB>::N];
+    load_tile_words<KB>(page, lane, dt, w);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag<KB>(w, mt, a);
+      mma_f16(s2[mt], a[0], a[1], a[2], a[3], qkb[2 * dt], qkb[2 * dt + 1]);
+    }
+  }
+  float sc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int tok = g + 8 * i;
+    const float acc = s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1];
+    sc[i] = fmaf(acc, kst[tok], kzt[tok] * qsum);
+  }
+  tok_rescale_update<D>(st, sc, tau);
+
+  float pv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pv[i] = sc[i] * svf[g + 8 * i];
+    st.vz = fmaf(sc[i], zvf[g + 8 * i], st.vz);
+  }
+  uint32_t pb[2][2];
+  tok_pfrags<false>(ptr, pv, lane, partf, pb);
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<VB>::N];
+    load_tile_words<VB>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      tile_afrag<VB>(w, ks, a);
+      mma_f16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
+    }
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void attend_bpage_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qbp)[D / 8],
                                                  float* wscr, float partf, float scale_log2, int lane) {
@@ -901,10 +1054,10 @@ __device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p
   }
 }
 
-template <int KB, int VB, int D, bool TOK>
-__global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg<KB, VB, D>::MINB)
+template <int KB, int VB, int D, bool TOK, bool PT>
+__global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK : Cfg<KB, VB, D, PT>::MINB)
     decode_mma_kernel(DecodeParams p) {
-  using C = Cfg<KB, VB, D>;
+  using C = Cfg<KB, VB, D, PT>;
   using State = typename std::conditional<TOK, TokState<D>, WarpState<D>>::type;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_last;
@@ -1023,7 +1176,8 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
     // ---- query operands
     float qf[D / 4];
     uint32_t qb[D / 8];   // bf16 pairs (head rows) or bf16 parts (token rows)
-    uint32_t qzb[D / 8];  // token rows: z-term B fragments (q parts)
+    uint32_t qzb[D / 8];  // token rows: z-term B fragments (q parts); QK B fragments with per-token keys
+    float qsum = 0.f;     // per-token keys: sum_c q'_c of the head this lane scores
     auto load_qbp = [&]() {
 #pragma unroll
       for (int dt = 0; dt < C::KS; ++dt) {
@@ -1049,11 +1203,14 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
         qf[dt * 4 + 2] = h2.x * p.scale_log2;
         qf[dt * 4 + 3] = h2.y * p.scale_log2;
       }
+      // q parts: the z-term B/A operands (per-channel keys) or the QK operands
+      // themselves (per-token keys: the 2-bit tauK channel factor is folded here)
+      constexpr float qhi = PT ? 1.f / C::tauK : 1.f;  // channels 2t+8, 2t+9 of each tile
       if constexpr (TOK) {
 #pragma unroll
         for (int dt = 0; dt < C::KS; ++dt) {
           qzb[2 * dt] = part_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], partf);
-          qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2], qf[dt * 4 + 3], partf);
+          qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, partf);
         }
       } else {
         if (warp == 0) {
@@ -1061,11 +1218,21 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
           for (int dt = 0; dt < C::KS; ++dt) {
             uint4 q4;
             split_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], q4.x, q4.y);
-            split_f16(qf[dt * 4 + 2], qf[dt * 4 + 3], q4.z, q4.w);
+            split_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, q4.z, q4.w);
             *reinterpret_cast<uint4*>(qz + (dt * 32 + lane) * 4) = q4;
           }
         }
         __syncthreads();
+      }
+      if constexpr (PT) {
+        // sum_c q'_c of this lane's query head (its D/4 channels, then the quad)
+        float qs = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 4; ++i) qs += qf[i];
+        qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+        qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+        // token rows score head t (held by lanes with g = 2t); head rows score head g
+        qsum = TOK ? __shfl_sync(0xffffffffu, qs, 8 * t) : qs;
       }
     }
 
@@ -1113,9 +1280,11 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
             const uint8_t* page = ring + stage * C::STAGE;
             if constexpr (TOK) {
               if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
+              else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
               else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
             } else {
               if constexpr (C::kBf16) attend_bpage<D>(page, st, qb, p.scale_log2, lane);
+              else if constexpr (PT) attend_qpage_pt<KB, VB, D>(page, st, qz, qsum, wscr, lane);
               else attend_qpage<KB, VB, D>(page, st, qf, qz, wscr, lane);
             }
             ++consumed;
@@ -1262,20 +1431,20 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D>::MINB_TOK : Cfg
   }
 }
 
-template <int KB, int VB, int D, bool TOK>
+template <int KB, int VB, int D, bool TOK, bool PT>
 cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
-  using C = Cfg<KB, VB, D>;
+  using C = Cfg<KB, VB, D, PT>;
   static int configured_smem = 0;
   static int occ_smem = -1, occ_blocks = 0;
   const int smem = C::smem_bytes(TOK, p.gqa, p.batch);
   if (smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK, PT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);
     if (e != cudaSuccess) return e;
     configured_smem = smem;
   }
   if (smem != occ_smem) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_blocks, decode_mma_kernel<KB, VB, D, TOK>,
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_blocks, decode_mma_kernel<KB, VB, D, TOK, PT>,
                                                                   kThreads, smem);
     if (e != cudaSuccess) return e;
     occ_smem = smem;
@@ -1284,14 +1453,18 @@ cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   grid = std::min<int64_t>(grid, p.n_units);
   grid = std::min<int64_t>(grid, p.max_ctas);
   if (grid < 1) grid = 1;
-  decode_mma_kernel<KB, VB, D, TOK><<<(unsigned)grid, kThreads, smem, s>>>(p);
+  decode_mma_kernel<KB, VB, D, TOK, PT><<<(unsigned)grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <int KB, int VB, int D>
 cudaError_t launch3(const DecodeParams& p, cudaStream_t s) {
   // token rows when the query group fits the 8 (head, part) columns
-  return p.gqa <= 4 ? launch4<KB, VB, D, true>(p, s) : launch4<KB, VB, D, false>(p, s);
+  if constexpr (KB != 16) {
+    if (p.key_mode != 0)
+      return p.gqa <= 4 ? launch4<KB, VB, D, true, true>(p, s) : launch4<KB, VB, D, false, true>(p, s);
+  }
+  return p.gqa <= 4 ? launch4<KB, VB, D, true, false>(p, s) : launch4<KB, VB, D, false, false>(p, s);
 }
 
 template <int D>

@@ -71,9 +71,10 @@ struct Smem {
   int last;
 };
 
-// Dequantize one full page into kd/vd (fp32).
+// Dequantize one full page into kd/vd (fp32). per_token_keys: the page holds 32
+// key scales/zeros in token order instead of D in channel-slot order.
 template <int KB, int VB, int D>
-__device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page) {
+__device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page, bool per_token_keys) {
   constexpr int F = 2 * (D / 16);
   const uint8_t* kblk = page;
   const uint8_t* vblk = page + code_block_bytes(KB, D);
@@ -90,12 +91,13 @@ __device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page) {
       }
     }
   } else {
+    const int nk = per_token_keys ? kPageTokens : D;
     const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
-    const __half* kzero = kscale + D;
-    const __half* vscale = kzero + D;
+    const __half* kzero = kscale + nk;
+    const __half* vscale = kzero + nk;
     const __half* vzero = vscale + kPageTokens;
-    for (int i = threadIdx.x; i < D; i += kThreads) {
-      int d = kmeta_channel<D>(i);
+    for (int i = threadIdx.x; i < nk; i += kThreads) {
+      int d = per_token_keys ? i : kmeta_channel<D>(i);  // ks/kz indexed by token or by channel
       sm.ks[d] = __half2float(kscale[i]);
       sm.kz[d] = __half2float(kzero[i]);
     }
@@ -110,7 +112,8 @@ __device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page) {
       for (int e = 0; e < 8; ++e) {
         int tok, dim;
         tile_elem(f, lane, e, false, tok, dim);
-        sm.kd[tok][dim] = fmaf((float)elem_code<KB>(kblk, f, lane, e), sm.ks[dim], sm.kz[dim]);
+        const int ki = per_token_keys ? tok : dim;
+        sm.kd[tok][dim] = fmaf((float)elem_code<KB>(kblk, f, lane, e), sm.ks[ki], sm.kz[ki]);
         tile_elem(f, lane, e, true, tok, dim);
         sm.vd[tok][dim] = fmaf((float)elem_code<VB>(vblk, f, lane, e), sm.vs[tok], sm.vz[tok]);
       }
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeParams p) {
 
   const uint8_t* base = p.pages + ((int64_t)(b * H + h) * p.max_pages) * p.page_bytes;
   for (int pg = p0; pg < p1; ++pg) {
-    load_page<KB, VB, D>(sm, base + (int64_t)pg * p.page_bytes);
+    load_page<KB, VB, D>(sm, base + (int64_t)pg * p.page_bytes, p.key_mode != 0);
     attend_tokens<KB, VB, D, NACC>(sm, G, kPageTokens, p.scale_log2, acc);
   }
   if (s == nsplit - 1 && W > 0) {

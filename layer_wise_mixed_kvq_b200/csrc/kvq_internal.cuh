@@ -30,8 +30,9 @@ constexpr int kMaxGqa = 8;
 
 __host__ __device__ constexpr int64_t code_block_bytes(int bits, int D) { return 4LL * D * bits; }
 
-__host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D) {
-  return code_block_bytes(kb, D) + code_block_bytes(vb, D) + (kb == 16 ? 0 : 4LL * D + 128);
+// km: key mode (0 = per-channel keys, D scale/zero pairs; 1 = per-token keys, 32).
+__host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D, int km) {
+  return code_block_bytes(kb, D) + code_block_bytes(vb, D) + (kb == 16 ? 0 : (km ? 128LL : 4LL * D) + 128);
 }
 
 // Tensor-core kernel split record: [G][D] accumulators, [G] maxima, [G] sums,
@@ -39,7 +40,7 @@ __host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D) {
 __host__ __device__ constexpr int split_record_floats(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
 
 struct LayerState {
-  int kb = 0, vb = 0;
+  int kb = 0, vb = 0, km = 0;
   int64_t page_bytes = 0;
   uint8_t* pages = nullptr;
   __nv_bfloat16* window = nullptr;
@@ -59,6 +60,7 @@ struct AppendParams {
   int64_t page_bytes;
   int max_pages;
   int n_kv_heads;
+  int key_mode;          // 0 = per-channel keys, 1 = per-token keys
 };
 
 // Parameters of the decode attention kernel.
@@ -81,11 +83,13 @@ struct DecodeParams {
   int max_ctas;          // tensor-core kernel: CTAs the partial buffer can serve (2 split records each)
   int sm_count;
   int seg_overhead;      // tensor-core kernel: overhead units leading each segment (>= 0)
+  int key_mode;          // 0 = per-channel keys, 1 = per-token keys
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
 };
 
 // Launchers (defined per kernel file); return the CUDA launch error.
+// The key mode travels in the parameter blocks (AppendParams/DecodeParams::key_mode).
 cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
                           cudaStream_t s);
 cudaError_t launch_decode_simt(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);

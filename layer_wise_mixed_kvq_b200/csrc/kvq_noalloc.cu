@@ -69,7 +69,9 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
                                               const void* pages, int64_t max_pages, const void* window,
                                               const int32_t* seq_len, int64_t max_seq_len, const void* Q,
                                               int batch, float* out, void* stream) {
-  if (!((pair.k_bits == 16 && pair.v_bits == 16) || (ok_bits(pair.k_bits) && ok_bits(pair.v_bits))))
+  if (!((pair.k_bits == 16 && pair.v_bits == 16) || (ok_bits(pair.k_bits) && ok_bits(pair.v_bits))) ||
+      pair.reserved != 0 || pair.key_mode > KVQ_KEY_PER_TOKEN ||
+      (pair.k_bits == 16 && pair.key_mode != KVQ_KEY_PER_CHANNEL))
     return fail(KVQ_EINVAL, "unsupported pair");
   if (head_dim != 64 && head_dim != 128) return fail(KVQ_EINVAL, "head_dim must be 64 or 128");
   if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads != 0 || n_q_heads / n_kv_heads > kvq::kMaxGqa)
@@ -119,7 +121,8 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.out = out;
   p.partials = partials;
   p.ctr = ctr;
-  p.page_bytes = kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim);
+  p.page_bytes = kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim, pair.key_mode);
+  p.key_mode = pair.key_mode;
   p.max_pages = (int)max_pages;
   p.n_kv_heads = n_kv_heads;
   p.gqa = G;

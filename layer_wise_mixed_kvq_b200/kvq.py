@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 KVQ_OK, KVQ_EINVAL, KVQ_ECAPACITY, KVQ_ENOMEM, KVQ_ECUDA = 0, 1, 2, 3, 4
 KVQ_BF16, KVQ_F32 = 0, 1
+KVQ_KEY_PER_CHANNEL, KVQ_KEY_PER_TOKEN = 0, 1
 
 #: every symbol the C header declares
 EXPORTS = (
@@ -27,7 +28,13 @@ EXPORTS = (
 
 
 class kvq_pair(ctypes.Structure):
-    _fields_ = [("k_bits", ctypes.c_uint8), ("v_bits", ctypes.c_uint8)]
+    _fields_ = [("k_bits", ctypes.c_uint8), ("v_bits", ctypes.c_uint8), ("key_mode", ctypes.c_uint8),
+                ("reserved", ctypes.c_uint8)]
+
+
+def _pair(p) -> kvq_pair:
+    """(k_bits, v_bits) or (k_bits, v_bits, key_mode) -> kvq_pair."""
+    return kvq_pair(int(p[0]), int(p[1]), int(p[2]) if len(p) > 2 else KVQ_KEY_PER_CHANNEL, 0)
 
 
 class KVQError(RuntimeError):
@@ -86,8 +93,8 @@ def _check(st: int) -> None:
 
 def _pairs(layer_map):
     arr = (kvq_pair * len(layer_map))()
-    for i, (k, v) in enumerate(layer_map):
-        arr[i].k_bits, arr[i].v_bits = int(k), int(v)
+    for i, p in enumerate(layer_map):
+        arr[i] = _pair(p)
     return arr
 
 
@@ -112,8 +119,7 @@ def _dev_ptr(t):
 
 # ----------------------------------------------------------------- host-only --
 def kvq_page_bytes(pair, head_dim: int) -> int:
-    p = kvq_pair(int(pair[0]), int(pair[1]))
-    return int(lib.kvq_page_bytes(p, int(head_dim)))
+    return int(lib.kvq_page_bytes(_pair(pair), int(head_dim)))
 
 
 def kvq_equiv_bits(layer_map) -> float:
@@ -179,7 +185,7 @@ def kvq_decode_attn_noalloc(pair, head_dim, n_q_heads, n_kv_heads, pages, max_pa
     import torch
     if Q.dtype != torch.bfloat16 or out.dtype != torch.float32 or seq_len.dtype != torch.int32:
         raise ValueError("Q must be bfloat16, out float32 and seq_len int32")
-    _check(lib.kvq_decode_attn_noalloc(kvq_pair(int(pair[0]), int(pair[1])), int(head_dim), int(n_q_heads),
+    _check(lib.kvq_decode_attn_noalloc(_pair(pair), int(head_dim), int(n_q_heads),
                                        int(n_kv_heads), _dev_ptr(pages), int(max_pages), _dev_ptr(window),
                                        _dev_ptr(seq_len), int(max_seq_len), _dev_ptr(Q), int(Q.shape[0]),
                                        _dev_ptr(out), _stream(stream)))

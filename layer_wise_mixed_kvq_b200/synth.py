@@ -13,6 +13,8 @@ and the 3.25 / 4.0-bit results):
 * ``tiny_k8v4``      -- 1 layer K8V4, batch 1, 2 query = 2 KV heads, D 64,
   256 cached tokens + 1 decode token, fp32 N(0,1) with 2 key channels x10.
 * ``llama_k4v4``     -- 32 layers K4V4, batch 16, context 4096 + 1.
+* ``llama_k4v4_pt``  -- the same shapes, draws and seed with per-token keys
+  (third pair field 1: the per-token-asym key mode).
 * ``llama_mixed325`` -- layers 0,1,2,31 K4V8; 3-26 K4V2; 27-30 K2V2; batch 64,
   prefill 128 then 512 decode steps.
 * ``qwen_mixed40``   -- 28 layers: 0-3 K8V4, 4-19 K4V4, 20-27 K4V2; batch 32,
@@ -35,7 +37,7 @@ BF16 = (16, 16)
 @dataclass(frozen=True)
 class Workload:
     name: str
-    layer_map: tuple            # ((k_bits, v_bits), ...) one per layer
+    layer_map: tuple            # ((k_bits, v_bits[, key_mode]), ...) one per layer
     batch: int
     n_q_heads: int
     n_kv_heads: int
@@ -91,6 +93,8 @@ WORKLOADS = {
     "tiny_k8v4": Workload("tiny_k8v4", ((8, 4),), 1, 2, 2, 64, 256, 1, "normal", 2, 10.0, "f32", 0),
     "llama_k4v4": Workload("llama_k4v4", tuple([(4, 4)] * 32), 16, 32, 8, 128, 4096, 1, "normal", 4,
                            8.0, "bf16", 1),
+    "llama_k4v4_pt": Workload("llama_k4v4_pt", tuple([(4, 4, 1)] * 32), 16, 32, 8, 128, 4096, 1, "normal", 4,
+                              8.0, "bf16", 1),
     "llama_mixed325": Workload("llama_mixed325", _llama_mixed_map(), 64, 32, 8, 128, 128, 512, "normal",
                                4, 8.0, "bf16", 2),
     "qwen_mixed40": Workload("qwen_mixed40", _qwen_map(), 32, 28, 4, 128, 8192, 1, "student_t3", 8, 16.0,

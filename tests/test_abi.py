@@ -57,6 +57,22 @@ def test_page_bytes(kvq):
     assert kvq.kvq_page_bytes((1, 4), 128) == 0
 
 
+def test_page_bytes_per_token_keys(kvq):
+    # per-token keys: 32 key scale/zero pairs per page instead of D
+    for D in (64, 128):
+        for k in (2, 4, 8):
+            for v in (2, 4, 8):
+                assert kvq.kvq_page_bytes((k, v, kvq.KVQ_KEY_PER_TOKEN), D) == 4 * D * (k + v) + 256
+    assert kvq.kvq_page_bytes((16, 16, kvq.KVQ_KEY_PER_TOKEN), 128) == 0   # bf16 layers have no key mode
+    assert kvq.kvq_page_bytes((4, 4, 2), 128) == 0                         # unknown mode
+    bad = kvq.kvq_pair(4, 4, 0, 1)                                          # reserved byte set
+    assert kvq.lib.kvq_page_bytes(bad, 128) == 0
+    assert kvq.kvq_equiv_bits([(4, 4, 1), (4, 2, 0)]) == 3.5               # the mode does not change bits
+    pc = kvq.kvq_cache_pool_bytes([(4, 4)] * 2, 32, 8, 128, 16, 4097)
+    pt = kvq.kvq_cache_pool_bytes([(4, 4, 1)] * 2, 32, 8, 128, 16, 4097)
+    assert 0 < pt < pc
+
+
 def test_pool_bytes_validation(kvq):
     good = kvq.kvq_cache_pool_bytes([(4, 4)] * 2, 32, 8, 128, 16, 4097)
     assert good > 2 * 16 * 8 * 128 * kvq.kvq_page_bytes((4, 4), 128)

@@ -44,7 +44,7 @@ class Pair:
         self.kvq, self.pair, self.batch, self.hq, self.hkv, self.D = kvq, pair, batch, hq, hkv, D
         self.dtype = dtype
         self.cache = kvq.kvq_cache_create([pair], hq, hkv, D, batch, max_tokens)
-        self.ref = oracle.OracleLayer(pair[0], pair[1], batch, hkv, D)
+        self.ref = oracle.OracleLayer(pair[0], pair[1], batch, hkv, D, key_mode=pair[2] if len(pair) > 2 else 0)
 
     def close(self):
         self.kvq.kvq_cache_destroy(self.cache)

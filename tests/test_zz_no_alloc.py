@@ -56,7 +56,8 @@ def _close(got, want):
     assert np.linalg.norm(got - want) / np.linalg.norm(want) <= REL_L2
 
 
-@pytest.mark.parametrize("pair,D,G", [((4, 4), 128, 4), ((8, 2), 64, 7), ((16, 16), 128, 1)])
+@pytest.mark.parametrize("pair,D,G", [((4, 4), 128, 4), ((8, 2), 64, 7), ((16, 16), 128, 1), ((2, 4, 1), 128, 4),
+                                      ((4, 8, 1), 64, 7)])
 def test_noalloc_matches_decode_attn_twice(kvq, pair, D, G):
     rng = np.random.default_rng(77)
     batch, hkv, max_tokens = 3, 2, 1100
