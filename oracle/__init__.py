@@ -49,14 +49,20 @@ def lib() -> ctypes.CDLL:
             "oracle_f32_to_f16_ru": (c.c_uint16, [c.c_float]),
             "oracle_f16_value": (c.c_double, [c.c_uint16]),
             "oracle_equiv_bits": (c.c_double, [P, P, c.c_int]),
-            "oracle_layer_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int, c.c_int, c.c_int]),
+            "oracle_layer_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int, c.c_int,
+                                               c.c_int]),
             "oracle_quantize": (None, [P, c.c_int, c.c_int, P, P, P]),
-            "oracle_page_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int, c.c_int]),
+            "oracle_page_bytes": (c.c_int64, [c.c_int, c.c_int, c.c_int, c.c_int, c.c_int]),
+            "oracle_e4m3_encode": (c.c_uint8, [c.c_float]),
+            "oracle_e4m3_value": (c.c_double, [c.c_uint8]),
             "oracle_pack_block": (None, [P, P, c.c_int, c.c_int, c.c_int]),
             "oracle_unpack_block": (None, [P, P, c.c_int, c.c_int, c.c_int]),
-            "oracle_build_page": (None, [P, P, P, c.c_int, c.c_int, c.c_int, c.c_int]),
-            "oracle_dequant_page": (None, [P, c.c_int, c.c_int, c.c_int, c.c_int, P, P]),
-            "oracle_layer_new": (P, [c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int]),
+            "oracle_build_page": (None, [P, P, P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_float,
+                                         c.c_float]),
+            "oracle_dequant_page": (None, [P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_float, c.c_float,
+                                           P, P]),
+            "oracle_layer_new": (P, [c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int]),
+            "oracle_layer_set_fp8_scales": (None, [P, P, P]),
             "oracle_layer_free": (None, [P]),
             "oracle_layer_len": (c.c_int64, [P, c.c_int]),
             "oracle_layer_append": (None, [P, P, P, P, c.c_int]),
@@ -113,15 +119,27 @@ def equiv_bits(pairs) -> float:
 
 #: key modes: per-channel keys over the 32-token group, or per-token keys
 KEY_PER_CHANNEL, KEY_PER_TOKEN = 0, 1
+#: layer formats: integer codes with fp16 scale/zero, or fp8 e4m3 with per-head scales
+FMT_INT, FMT_FP8 = 0, 1
 
 
 def layer_bytes(k_bits: int, v_bits: int, tokens: int, n_kv_heads: int, head_dim: int,
-                with_meta: bool = False, key_mode: int = KEY_PER_CHANNEL) -> int:
-    return int(lib().oracle_layer_bytes(k_bits, v_bits, key_mode, tokens, n_kv_heads, head_dim, int(with_meta)))
+                with_meta: bool = False, key_mode: int = KEY_PER_CHANNEL, fmt: int = FMT_INT) -> int:
+    return int(lib().oracle_layer_bytes(k_bits, v_bits, key_mode, fmt, tokens, n_kv_heads, head_dim,
+                                        int(with_meta)))
 
 
-def page_bytes(k_bits: int, v_bits: int, head_dim: int, key_mode: int = KEY_PER_CHANNEL) -> int:
-    return int(lib().oracle_page_bytes(k_bits, v_bits, head_dim, key_mode))
+def page_bytes(k_bits: int, v_bits: int, head_dim: int, key_mode: int = KEY_PER_CHANNEL, fmt: int = FMT_INT) -> int:
+    return int(lib().oracle_page_bytes(k_bits, v_bits, head_dim, key_mode, fmt))
+
+
+def e4m3_encode(x: float) -> int:
+    """fp32 -> e4m3 bits (round to nearest even, saturating at 448)."""
+    return int(lib().oracle_e4m3_encode(float(x)))
+
+
+def e4m3_value(bits: int) -> float:
+    return float(lib().oracle_e4m3_value(int(bits) & 0xFF))
 
 
 # -------------------------------------------------------------- quantizer --
@@ -150,19 +168,23 @@ def unpack_block(blk: np.ndarray, head_dim: int, bits: int, is_value: bool) -> n
 
 
 def build_page(k_bf16_bits: np.ndarray, v_bf16_bits: np.ndarray, head_dim: int, k_bits: int,
-               v_bits: int, key_mode: int = KEY_PER_CHANNEL) -> np.ndarray:
+               v_bits: int, key_mode: int = KEY_PER_CHANNEL, fmt: int = FMT_INT, k_scale: float = 1.0,
+               v_scale: float = 1.0) -> np.ndarray:
     kb = np.ascontiguousarray(k_bf16_bits, dtype=np.uint16).reshape(32, head_dim)
     vb = np.ascontiguousarray(v_bf16_bits, dtype=np.uint16).reshape(32, head_dim)
-    page = np.zeros(page_bytes(k_bits, v_bits, head_dim, key_mode), dtype=np.uint8)
-    lib().oracle_build_page(_ptr(page), _ptr(kb), _ptr(vb), head_dim, k_bits, v_bits, key_mode)
+    page = np.zeros(page_bytes(k_bits, v_bits, head_dim, key_mode, fmt), dtype=np.uint8)
+    lib().oracle_build_page(_ptr(page), _ptr(kb), _ptr(vb), head_dim, k_bits, v_bits, key_mode, fmt,
+                            float(k_scale), float(v_scale))
     return page
 
 
-def dequant_page(page: np.ndarray, head_dim: int, k_bits: int, v_bits: int, key_mode: int = KEY_PER_CHANNEL):
+def dequant_page(page: np.ndarray, head_dim: int, k_bits: int, v_bits: int, key_mode: int = KEY_PER_CHANNEL,
+                 fmt: int = FMT_INT, k_scale: float = 1.0, v_scale: float = 1.0):
     page = np.ascontiguousarray(page, dtype=np.uint8)
     K = np.zeros((32, head_dim), dtype=np.float64)
     V = np.zeros((32, head_dim), dtype=np.float64)
-    lib().oracle_dequant_page(_ptr(page), head_dim, k_bits, v_bits, key_mode, _ptr(K), _ptr(V))
+    lib().oracle_dequant_page(_ptr(page), head_dim, k_bits, v_bits, key_mode, fmt, float(k_scale), float(v_scale),
+                              _ptr(K), _ptr(V))
     return K, V
 
 
@@ -171,10 +193,15 @@ class OracleLayer:
     """One layer's KV cache for `batch` sequences, mirroring the library's semantics."""
 
     def __init__(self, k_bits: int, v_bits: int, batch: int, n_kv_heads: int, head_dim: int,
-                 key_mode: int = KEY_PER_CHANNEL):
-        self.k_bits, self.v_bits, self.key_mode = k_bits, v_bits, key_mode
+                 key_mode: int = KEY_PER_CHANNEL, fmt: int = FMT_INT, k_scales=None, v_scales=None):
+        self.k_bits, self.v_bits, self.key_mode, self.fmt = k_bits, v_bits, key_mode, fmt
         self.batch, self.n_kv_heads, self.head_dim = batch, n_kv_heads, head_dim
-        self._h = lib().oracle_layer_new(k_bits, v_bits, key_mode, batch, n_kv_heads, head_dim)
+        self._h = lib().oracle_layer_new(k_bits, v_bits, key_mode, fmt, batch, n_kv_heads, head_dim)
+        if k_scales is not None or v_scales is not None:
+            ks = np.ascontiguousarray(np.ones(n_kv_heads) if k_scales is None else k_scales, dtype=np.float32)
+            vs = np.ascontiguousarray(np.ones(n_kv_heads) if v_scales is None else v_scales, dtype=np.float32)
+            assert ks.size == n_kv_heads and vs.size == n_kv_heads
+            lib().oracle_layer_set_fp8_scales(self._h, _ptr(ks), _ptr(vs))
 
     def __del__(self):
         h = getattr(self, "_h", None)

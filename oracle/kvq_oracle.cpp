@@ -41,6 +41,15 @@
 //  * empty sequence: output 0.
 //  * per-token key mode keeps the same 32-token pages and bf16 residual window:
 //    a key token is quantized when its page fills, like a value token.
+//  * FP8 layer format (llms-explorer facts page: vLLM-style FP8 KV cache with
+//    per-attention-head scales and BF16 skip layers; machinoai Q&A section 2
+//    worked example of BF16 and FP8 layers): each key/value element of KV head
+//    h is stored as e4m3(x / s_h) with a per-layer, per-head fp32 scale s_h
+//    (k and v scales separate, calibrated offline, an input here, default 1).
+//    e4m3 = 1 sign, 4 exponent (bias 7), 3 mantissa bits, no infinities,
+//    largest finite 448; rounding to nearest, ties to even, and magnitudes
+//    above 448 saturate to 448. Dequantized value: e4m3 value * s_h. Same
+//    32-token pages (no per-page metadata) and bf16 residual window.
 //
 // The packed page layout implemented here is the library's documented storage
 // format (written out independently below from its definition).
@@ -123,6 +132,49 @@ uint16_t f32_to_f16_directed(float xf, bool up) {
   return f16_encode_exact(v, v == 0 && x < 0);
 }
 
+// ------------------------------------------------------------------ e4m3 --
+
+// Value of an e4m3 bit pattern (NaN for S.1111.111).
+double e4m3_value(uint8_t c) {
+  int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = (e == 0) ? std::ldexp((double)m, -9) : std::ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+// fp32 -> e4m3: round to nearest, ties to even, saturating at 448 (inf too).
+// Written from the definition: the spacing of the e4m3 grid around |x| is
+// 2^-9 below 2^-6 (subnormals) and 2^(floor(log2|x|) - 3) above; all exact
+// in double.
+uint8_t e4m3_encode(float xf) {
+  double x = xf;
+  uint8_t sign = std::signbit(xf) ? 0x80 : 0x00;
+  double a = std::fabs(x);
+  if (!(a < 448.0)) return sign | 0x7E;  // 448 (this also saturates inf)
+  double spacing;
+  if (a < std::ldexp(1.0, -6)) {
+    spacing = std::ldexp(1.0, -9);
+  } else {
+    int ex;
+    std::frexp(a, &ex);  // a = f * 2^ex, f in [0.5, 1)
+    spacing = std::ldexp(1.0, ex - 1 - 3);
+  }
+  double q = a / spacing;               // exact (power-of-two spacing)
+  double r = std::floor(q);
+  double frac = q - r;
+  if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) r += 1.0;
+  double v = r * spacing;               // rounded magnitude, <= 448
+  if (v > 448.0) v = 448.0;
+  if (v == 0.0) return sign;
+  // encode v: subnormal if below 2^-6
+  if (v < std::ldexp(1.0, -6)) return sign | (uint8_t)(v / std::ldexp(1.0, -9));
+  int ex;
+  double f = std::frexp(v, &ex);        // v = f * 2^ex, f in [0.5, 1)
+  int e = ex - 1 + 7;                   // biased exponent of 1.m form
+  int m = (int)((f * 2.0 - 1.0) * 8.0);  // exact: v has 3 fraction bits
+  return sign | (uint8_t)(e << 3) | (uint8_t)m;
+}
+
 // ------------------------------------------------------------- quantizer --
 
 // Quantize n values (already bf16-exact fp32) to `bits`-bit unsigned codes with
@@ -203,9 +255,10 @@ int64_t word_byte(int lane, int64_t w) { return ((w / 4) * 32 + lane) * 16 + (w 
 int64_t code_block_bytes(int bits, int D) { return (int64_t)32 * D * bits / 8; }
 
 // key_mode: 0 = per-channel keys (D scale/zero pairs), 1 = per-token keys (32).
-int64_t page_bytes(int kb, int vb, int D, int key_mode) {
+// fmt: 0 = integer codes with fp16 scale/zero, 1 = fp8 e4m3 (8/8 bits, no page metadata).
+int64_t page_bytes(int kb, int vb, int D, int key_mode, int fmt) {
   int64_t b = code_block_bytes(kb, D) + code_block_bytes(vb, D);
-  if (kb != 16) b += (key_mode ? 128 : (int64_t)4 * D) + 128;
+  if (kb != 16 && !fmt) b += (key_mode ? 128 : (int64_t)4 * D) + 128;
   return b;
 }
 
@@ -269,13 +322,25 @@ void unpack_block(const uint8_t* blk, uint16_t* vals, int D, int bits, bool is_v
 }
 
 // Build one page from 32 tokens of bf16 keys/values ([32][D] bit patterns).
-void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb, int key_mode) {
-  std::memset(page, 0, (size_t)page_bytes(kb, vb, D, key_mode));
+// fp8 pages: ksc/vsc are the KV head's fp32 key and value scales.
+void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb, int key_mode,
+                int fmt, float ksc, float vsc) {
+  std::memset(page, 0, (size_t)page_bytes(kb, vb, D, key_mode, fmt));
   uint8_t* kblk = page;
   uint8_t* vblk = page + code_block_bytes(kb, D);
   if (kb == 16) {
     pack_block(kblk, kbf, D, 16, false);
     pack_block(vblk, vbf, D, 16, true);
+    return;
+  }
+  if (fmt) {
+    std::vector<uint16_t> kc(32 * D), vc(32 * D);
+    for (int i = 0; i < 32 * D; ++i) {
+      kc[i] = e4m3_encode(bf16_to_f32(kbf[i]) / ksc);  // one IEEE fp32 division
+      vc[i] = e4m3_encode(bf16_to_f32(vbf[i]) / vsc);
+    }
+    pack_block(kblk, kc.data(), D, 8, false);
+    pack_block(vblk, vc.data(), D, 8, true);
     return;
   }
   const int nk = key_mode ? 32 : D;  // key scale/zero pairs in the page
@@ -326,7 +391,8 @@ void build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, 
 }
 
 // Dequantize one page into [32][D] doubles (x = code * s + z, exact in fp64).
-void dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, double* Kh, double* Vh) {
+void dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, int fmt, float ksc, float vsc,
+                  double* Kh, double* Vh) {
   std::vector<uint16_t> kc(32 * D), vc(32 * D);
   const uint8_t* kblk = page;
   const uint8_t* vblk = page + code_block_bytes(kb, D);
@@ -334,6 +400,13 @@ void dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, doub
   unpack_block(vblk, vc.data(), D, vb, true);
   if (kb == 16) {
     for (int i = 0; i < 32 * D; ++i) { Kh[i] = bf16_to_f32(kc[i]); Vh[i] = bf16_to_f32(vc[i]); }
+    return;
+  }
+  if (fmt) {
+    for (int i = 0; i < 32 * D; ++i) {
+      Kh[i] = e4m3_value((uint8_t)kc[i]) * (double)ksc;
+      Vh[i] = e4m3_value((uint8_t)vc[i]) * (double)vsc;
+    }
     return;
   }
   const int nk = key_mode ? 32 : D;
@@ -380,8 +453,9 @@ struct Seq {
 };
 
 struct Layer {
-  int kb, vb, key_mode, batch, hkv, D;
+  int kb, vb, key_mode, fmt, batch, hkv, D;
   std::vector<Seq> seqs;
+  std::vector<float> kscale, vscale;  // fp8 format: per KV head
 };
 
 }  // namespace
@@ -406,11 +480,11 @@ double oracle_equiv_bits(const uint8_t* kbits, const uint8_t* vbits, int n_layer
 // (with_meta = 0, the idealised count of the worked example), or codes plus
 // fp16 scale/zero (2 bytes each: D/32 key pairs -- one key pair in per-token key
 // mode -- and one value pair per token).
-int64_t oracle_layer_bytes(int kbits, int vbits, int key_mode, int64_t tokens, int n_kv_heads, int head_dim,
-                           int with_meta) {
+int64_t oracle_layer_bytes(int kbits, int vbits, int key_mode, int fmt, int64_t tokens, int n_kv_heads,
+                           int head_dim, int with_meta) {
   int64_t bits = tokens * n_kv_heads * (int64_t)head_dim * (kbits + vbits);
   int64_t bytes = bits / 8;
-  if (with_meta && kbits != 16)
+  if (with_meta && kbits != 16 && !fmt)
     bytes += tokens * n_kv_heads * ((key_mode ? 4 : (int64_t)head_dim * 4 / 32) + 4);
   return bytes;
 }
@@ -420,7 +494,10 @@ void oracle_quantize(const float* x, int n, int bits, uint8_t* codes, uint16_t* 
   quantize_set(x, n, bits, codes, scale_bits, zero_bits);
 }
 
-int64_t oracle_page_bytes(int kb, int vb, int D, int key_mode) { return page_bytes(kb, vb, D, key_mode); }
+int64_t oracle_page_bytes(int kb, int vb, int D, int key_mode, int fmt) { return page_bytes(kb, vb, D, key_mode, fmt); }
+
+uint8_t oracle_e4m3_encode(float x) { return e4m3_encode(x); }
+double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
 
 // Pack/unpack one code block (vals [32][D]); is_value selects the V tiling.
 void oracle_pack_block(uint8_t* blk, const uint16_t* vals, int D, int bits, int is_value) {
@@ -432,16 +509,19 @@ void oracle_unpack_block(const uint8_t* blk, uint16_t* vals, int D, int bits, in
 }
 
 void oracle_build_page(uint8_t* page, const uint16_t* kbf, const uint16_t* vbf, int D, int kb, int vb,
-                       int key_mode) {
-  build_page(page, kbf, vbf, D, kb, vb, key_mode);
+                       int key_mode, int fmt, float ksc, float vsc) {
+  build_page(page, kbf, vbf, D, kb, vb, key_mode, fmt, ksc, vsc);
 }
-void oracle_dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, double* Kh, double* Vh) {
-  dequant_page(page, D, kb, vb, key_mode, Kh, Vh);
+void oracle_dequant_page(const uint8_t* page, int D, int kb, int vb, int key_mode, int fmt, float ksc, float vsc,
+                         double* Kh, double* Vh) {
+  dequant_page(page, D, kb, vb, key_mode, fmt, ksc, vsc, Kh, Vh);
 }
 
 // ---- one-layer cache simulator -------------------------------------------
-void* oracle_layer_new(int kb, int vb, int key_mode, int batch, int n_kv_heads, int head_dim) {
-  Layer* L = new Layer{kb, vb, kb == 16 ? 0 : key_mode, batch, n_kv_heads, head_dim, {}};
+void* oracle_layer_new(int kb, int vb, int key_mode, int fmt, int batch, int n_kv_heads, int head_dim) {
+  Layer* L = new Layer{kb, vb, kb == 16 ? 0 : key_mode, kb == 16 ? 0 : fmt, batch, n_kv_heads, head_dim, {}, {}, {}};
+  L->kscale.assign(n_kv_heads, 1.0f);
+  L->vscale.assign(n_kv_heads, 1.0f);
   L->seqs.resize(batch);
   for (auto& s : L->seqs) {
     s.pages.resize(n_kv_heads);
@@ -453,6 +533,15 @@ void* oracle_layer_new(int kb, int vb, int key_mode, int batch, int n_kv_heads, 
 
 void oracle_layer_free(void* p) { delete static_cast<Layer*>(p); }
 
+// fp8 format: per-KV-head key and value scales (before the first append).
+void oracle_layer_set_fp8_scales(void* p, const float* kscale, const float* vscale) {
+  Layer* L = static_cast<Layer*>(p);
+  for (int h = 0; h < L->hkv; ++h) {
+    L->kscale[h] = kscale[h];
+    L->vscale[h] = vscale[h];
+  }
+}
+
 int64_t oracle_layer_len(void* p, int b) { return static_cast<Layer*>(p)->seqs[b].len; }
 
 // Append n_new[b] tokens to every sequence b < batch. K and V are packed
@@ -462,7 +551,7 @@ int64_t oracle_layer_len(void* p, int b) { return static_cast<Layer*>(p)->seqs[b
 void oracle_layer_append(void* p, const float* K, const float* V, const int32_t* n_new, int batch) {
   Layer* L = static_cast<Layer*>(p);
   const int D = L->D, H = L->hkv;
-  const int64_t pb = page_bytes(L->kb, L->vb, D, L->key_mode);
+  const int64_t pb = page_bytes(L->kb, L->vb, D, L->key_mode, L->fmt);
   int64_t row = 0;
   for (int b = 0; b < batch; ++b) {
     Seq& s = L->seqs[b];
@@ -477,7 +566,8 @@ void oracle_layer_append(void* p, const float* K, const float* V, const int32_t*
         if ((int64_t)s.wk[h].size() == 32LL * D) {
           size_t off = s.pages[h].size();
           s.pages[h].resize(off + pb);
-          build_page(s.pages[h].data() + off, s.wk[h].data(), s.wv[h].data(), D, L->kb, L->vb, L->key_mode);
+          build_page(s.pages[h].data() + off, s.wk[h].data(), s.wv[h].data(), D, L->kb, L->vb, L->key_mode, L->fmt,
+                     L->kscale[h], L->vscale[h]);
           s.wk[h].clear();
           s.wv[h].clear();
         }
@@ -517,10 +607,11 @@ void oracle_layer_dequant(void* p, int b, int h, double* Kh, double* Vh) {
   Layer* L = static_cast<Layer*>(p);
   const int D = L->D;
   const Seq& s = L->seqs[b];
-  const int64_t pb = page_bytes(L->kb, L->vb, D, L->key_mode);
+  const int64_t pb = page_bytes(L->kb, L->vb, D, L->key_mode, L->fmt);
   int64_t npages = (int64_t)s.pages[h].size() / pb;
   for (int64_t pg = 0; pg < npages; ++pg)
-    dequant_page(s.pages[h].data() + pg * pb, D, L->kb, L->vb, L->key_mode, Kh + pg * 32 * D, Vh + pg * 32 * D);
+    dequant_page(s.pages[h].data() + pg * pb, D, L->kb, L->vb, L->key_mode, L->fmt, L->kscale[h], L->vscale[h],
+                 Kh + pg * 32 * D, Vh + pg * 32 * D);
   int64_t base = npages * 32 * D;
   for (size_t i = 0; i < s.wk[h].size(); ++i) {
     Kh[base + i] = bf16_to_f32(s.wk[h][i]);
