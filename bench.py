@@ -147,7 +147,10 @@ def cpu_baseline(w, seconds):
     while t_attn < seconds and samples < 64:
         pair = w.layer_map[layer % w.n_layers]
         key_mode = pair[2] if len(pair) > 2 else 0
-        L = oracle.OracleLayer(pair[0], pair[1], 1, w.n_kv_heads, w.head_dim, key_mode=key_mode)
+        fmt = pair[3] if len(pair) > 3 else 0
+        scales = w.fp8_scales if fmt else (None, None)
+        L = oracle.OracleLayer(pair[0], pair[1], 1, w.n_kv_heads, w.head_dim, key_mode=key_mode, fmt=fmt,
+                               k_scales=scales[0], v_scales=scales[1])
         K, V = synth.kv_tokens(w, layer, ctx + 1)
         L.append(K, V, [ctx + 1])
         Q = synth.queries(w, layer, batch=1)
@@ -156,7 +159,7 @@ def cpu_baseline(w, seconds):
         t_attn += time.perf_counter() - t0
         T = ctx + 1
         P, W = T // 32, T % 32
-        page = oracle.page_bytes(pair[0], pair[1], w.head_dim, key_mode)
+        page = oracle.page_bytes(pair[0], pair[1], w.head_dim, key_mode, fmt)
         done_bytes += w.n_kv_heads * (P * page + W * w.head_dim * 4)
         samples += 1
         layer += 1
@@ -208,6 +211,9 @@ def run_gpu(args, w):
     total_steps = args.warmup + args.steps
     max_tokens = int(lens.max()) + total_steps + 32  # + the end-to-end steps
     cache = kvq.kvq_cache_create(list(w.layer_map), Hq, Hkv, D, B, max_tokens)
+    for layer, pair in enumerate(w.layer_map):
+        if len(pair) > 3 and pair[3]:
+            kvq.kvq_set_fp8_scales(cache, layer, w.fp8_scales[0], w.fp8_scales[1])
     gen = torch.Generator(device=dev)
     gen.manual_seed(w.seed * 1000 + rank)
 

@@ -58,16 +58,26 @@ typedef enum {
   KVQ_KEY_PER_TOKEN = 1    /* one scale/zero per key token over head_dim (per-token-asym) */
 } kvq_key_mode;
 
+/* Element format of a layer's pages. */
+typedef enum {
+  KVQ_FMT_INT = 0, /* asymmetric integer codes with fp16 scale/zero in every page */
+  KVQ_FMT_FP8 = 1  /* fp8 e4m3 elements, x / s_h rounded to nearest even and saturated
+                      at 448, with per-KV-head fp32 key and value scales s_h
+                      ([facts]: vLLM FP8 KV cache with per-attention-head scales;
+                      [qa] section 2: BF16 and FP8 layers); k_bits = v_bits = 8 */
+} kvq_format;
+
 /* One layer's precision pair: k_bits, v_bits in {2, 4, 8}, or {16, 16} for a
  * layer kept in bf16 ([qa] section 2: sensitive layers stay BF16; [facts]:
  * vLLM-style skip layers). Mixed bf16/int pairs are rejected. key_mode is a
- * kvq_key_mode (must be KVQ_KEY_PER_CHANNEL, i.e. 0, for a bf16 layer);
- * reserved must be 0. A zero-initialised pair field means per-channel keys. */
+ * kvq_key_mode and format a kvq_format; both must be 0 for a bf16 layer, and
+ * an fp8 layer is (8, 8, KVQ_KEY_PER_CHANNEL, KVQ_FMT_FP8). A zero-initialised
+ * pair field means per-channel integer keys. */
 typedef struct {
   uint8_t k_bits;
   uint8_t v_bits;
   uint8_t key_mode;
-  uint8_t reserved;
+  uint8_t format;
 } kvq_pair;
 
 typedef enum {
@@ -92,6 +102,8 @@ typedef enum {
  *                   [K scale D x fp16][K zero D x fp16][V scale 32 x fp16][V zero 32 x fp16]
  *   per-token keys: [K codes][V codes][K scale 32 x fp16][K zero 32 x fp16][V scale][V zero]
  *                   (key scales and zeros in token order, like the values')
+ *   fp8 layer:      [K e4m3 32*D B][V e4m3 32*D B] (8-bit tile layout, scales per KV head
+ *                   held by the cache, see kvq_set_fp8_scales)
  *   bf16 layer:     [K 64*D B][V 64*D B]
  * Code blocks are stored as 16x16 tiles f = 2*dt + tt (dt: 16-channel tile,
  * tt: 16-token tile) laid out so that lane l = 4g + t of a warp reads its eight
@@ -203,6 +215,14 @@ kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n_q_heads, i
                                    const void* pages, int64_t max_pages, const void* window,
                                    const int32_t* seq_len, int64_t max_seq_len, const void* Q,
                                    int batch, float* out, void* stream);
+
+/* Set the per-KV-head fp32 scales of an fp8 layer (host arrays of n_kv_heads
+ * values, each finite and > 0; every head defaults to 1.0). Stored elements are
+ * e4m3(x / scale) and read back as e4m3 * scale. The layer must be empty (no
+ * token appended to any sequence since creation or the last reset), so every
+ * stored element uses the same scales. Synchronous. Errors: KVQ_EINVAL (not an
+ * fp8 layer, non-empty layer, bad scale), KVQ_ECUDA. */
+kvq_status kvq_set_fp8_scales(kvq_cache* cache, int layer, const float* k_scale, const float* v_scale);
 
 /* Pages per split-K CTA for kvq_decode_attn: 0 = automatic (default). Changing
  * it changes only the rounding order of the result. */

@@ -31,8 +31,9 @@ kvq_status cuda_fail(cudaError_t e, const char* what) {
 
 bool valid_pair(kvq_pair p) {
   auto ok = [](int b) { return b == 2 || b == 4 || b == 8; };
-  if (p.reserved != 0 || p.key_mode > KVQ_KEY_PER_TOKEN) return false;
-  if (p.k_bits == 16 && p.v_bits == 16) return p.key_mode == KVQ_KEY_PER_CHANNEL;
+  if (p.format > KVQ_FMT_FP8 || p.key_mode > KVQ_KEY_PER_TOKEN) return false;
+  if (p.k_bits == 16 && p.v_bits == 16) return p.key_mode == KVQ_KEY_PER_CHANNEL && p.format == KVQ_FMT_INT;
+  if (p.format == KVQ_FMT_FP8) return p.k_bits == 8 && p.v_bits == 8 && p.key_mode == KVQ_KEY_PER_CHANNEL;
   return ok(p.k_bits) && ok(p.v_bits);
 }
 
@@ -60,9 +61,9 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
   if (!map || n_layers <= 0) { why = "layer_map is null or n_layers <= 0"; return false; }
   for (int l = 0; l < n_layers; ++l)
     if (!valid_pair(map[l])) {
-      why = "layer " + std::to_string(l) + " has an unsupported pair (k_bits, v_bits, key_mode, reserved) = (" +
+      why = "layer " + std::to_string(l) + " has an unsupported pair (k_bits, v_bits, key_mode, format) = (" +
             std::to_string(map[l].k_bits) + ", " + std::to_string(map[l].v_bits) + ", " +
-            std::to_string(map[l].key_mode) + ", " + std::to_string(map[l].reserved) + ")";
+            std::to_string(map[l].key_mode) + ", " + std::to_string(map[l].format) + ")";
       return false;
     }
   if (head_dim != 64 && head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
@@ -76,12 +77,13 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
   g.max_pages = max_tokens / kvq::kPageTokens;
   size_t total = 0;
   for (int l = 0; l < n_layers; ++l) {
-    size_t pb = (size_t)kvq::page_bytes_of(map[l].k_bits, map[l].v_bits, head_dim, map[l].key_mode);
+    size_t pb = (size_t)kvq::page_bytes_of(map[l].k_bits, map[l].v_bits, head_dim, map[l].key_mode,
+                                           map[l].format);
     size_t pr = round_up((size_t)max_batch * n_kv_heads * std::max<int64_t>(g.max_pages, 1) * pb);
     size_t wr = round_up((size_t)max_batch * n_kv_heads * 2 * kvq::kPageTokens * head_dim * 2);
     g.page_region.push_back(pr);
     g.window_region.push_back(wr);
-    total += pr + wr + round_up((size_t)max_batch * 4);
+    total += pr + wr + round_up((size_t)max_batch * 4) + round_up((size_t)n_kv_heads * 2 * 4);
   }
   g.len_region = round_up((size_t)max_batch * 4);
   g.partial_slots = partial_slots_for(max_batch, n_kv_heads);
@@ -152,7 +154,7 @@ const char* kvq_status_string(kvq_status s) {
 
 int64_t kvq_page_bytes(kvq_pair pair, int head_dim) {
   if (!valid_pair(pair) || (head_dim != 64 && head_dim != 128)) return 0;
-  return kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim, pair.key_mode);
+  return kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim, pair.key_mode, pair.format);
 }
 
 double kvq_equiv_bits(const kvq_pair* map, int n_layers) {
@@ -220,13 +222,16 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     L.kb = map[l].k_bits;
     L.vb = map[l].v_bits;
     L.km = map[l].key_mode;
-    L.page_bytes = kvq::page_bytes_of(L.kb, L.vb, head_dim, L.km);
+    L.fmt = map[l].format;
+    L.page_bytes = kvq::page_bytes_of(L.kb, L.vb, head_dim, L.km, L.fmt);
     L.pages = p;
     p += g.page_region[l];
     L.window = reinterpret_cast<__nv_bfloat16*>(p);
     p += g.window_region[l];
     L.len = reinterpret_cast<int32_t*>(p);
     p += g.len_region;
+    L.fp8_scales = reinterpret_cast<float*>(p);
+    p += round_up((size_t)n_kv_heads * 2 * 4);
     L.host_len.assign(max_batch, 0);
   }
   c->partials = reinterpret_cast<float*>(p);
@@ -243,8 +248,12 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
   e = cudaMallocHost(&c->plan_host, (size_t)max_batch * 4 * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->plan_done, cudaEventDisableTiming);
   // lengths and counters start at zero; pages and windows need no initialisation
-  for (int l = 0; l < n_layers && e == cudaSuccess; ++l)
+  const std::vector<float> ones((size_t)n_kv_heads * 2, 1.0f);
+  for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
     e = cudaMemset(c->layers[l].len, 0, (size_t)max_batch * 4);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(c->layers[l].fp8_scales, ones.data(), ones.size() * 4, cudaMemcpyHostToDevice);
+  }
   if (e == cudaSuccess) e = cudaMemset(c->merge_ctr, 0, (size_t)max_batch * n_kv_heads * 4);
   if (e == cudaSuccess) e = cudaMemset(c->append_ctr, 0, (size_t)max_batch * 4);
   if (e == cudaSuccess) e = cudaMemset(c->err, 0, 4);
@@ -275,6 +284,26 @@ kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     std::fill(L.host_len.begin(), L.host_len.end(), 0);
   }
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_fp8_scales(kvq_cache* c, int layer, const float* k_scale, const float* v_scale) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  kvq::LayerState& L = c->layers[layer];
+  if (L.fmt != KVQ_FMT_FP8) return fail(KVQ_EINVAL, "layer is not an fp8 layer");
+  if (!k_scale || !v_scale) return fail(KVQ_EINVAL, "scale arrays are null");
+  for (int64_t T : L.host_len)
+    if (T != 0) return fail(KVQ_EINVAL, "fp8 scales must be set while the layer is empty");
+  std::vector<float> s((size_t)c->n_kv_heads * 2);
+  for (int h = 0; h < c->n_kv_heads; ++h) {
+    if (!(std::isfinite(k_scale[h]) && k_scale[h] > 0.f && std::isfinite(v_scale[h]) && v_scale[h] > 0.f))
+      return fail(KVQ_EINVAL, "fp8 scales must be finite and > 0");
+    s[h] = k_scale[h];
+    s[c->n_kv_heads + h] = v_scale[h];
+  }
+  cudaError_t e = cudaMemcpy(L.fp8_scales, s.data(), s.size() * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(fp8 scales)");
   return KVQ_OK;
 }
 
@@ -323,6 +352,8 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
   p.max_pages = (int)c->max_pages;
   p.n_kv_heads = c->n_kv_heads;
   p.key_mode = L.km;
+  p.fmt = L.fmt;
+  p.fp8_scales = L.fp8_scales;
   p.plan = nullptr;
   if (!all_one) {
     // multi-token append: per-sequence plan (start, count, row offset, items)
@@ -404,6 +435,8 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.sm_count = c->sm_count;
   p.seg_overhead = kvq::seg_overhead_units();
   p.key_mode = L.km;
+  p.fmt = L.fmt;
+  p.fp8_scales = L.fp8_scales;
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

@@ -21,6 +21,11 @@
 //   z = fp16_round_down(mn) clamped to >= -65504
 //   s = fp16_round_up((mx - z) / qmax) clamped to <= 65504
 //   code = s == 0 ? 0 : clamp(rint((x - z) * (1/s)), 0, qmax)
+// FP8 layers (e4m3 elements, per-KV-head scale s_h; llms-explorer facts page on
+// vLLM FP8 KV caches): code = e4m3(x / s_h), one IEEE division, then round to
+// nearest even with saturation at 448.
+
+#include <cuda_fp8.h>
 
 #include "kvq_internal.cuh"
 
@@ -225,6 +230,19 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         xs[1][t][d] = __bfloat162float(vx);
       }
       __syncthreads();
+      if (a.fmt != 0) {
+        if constexpr (KB == 8 && VB == 8) {
+          const float ksc = a.fp8_scales[h], vsc = a.fp8_scales[H + h];
+          for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
+            const int t = idx / D, d = idx % D;
+            cs[0][t][d] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(xs[0][t][d], ksc), __NV_SATFINITE, __NV_E4M3);
+            cs[1][t][d] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(xs[1][t][d], vsc), __NV_SATFINITE, __NV_E4M3);
+          }
+          __syncthreads();
+          store_block<8, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
+          store_block<8, D>(page + code_block_bytes(8, D), true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
+        }
+      } else {
       const bool per_token_keys = a.key_mode != 0;
       const int nk = per_token_keys ? kPageTokens : D;  // key scale/zero pairs
       uint8_t* vblk = page + code_block_bytes(KB, D);
@@ -281,6 +299,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
       __syncthreads();
       store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
       store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
+      }
     }
   }
 

@@ -33,6 +33,8 @@
 #include <algorithm>
 #include <type_traits>
 
+#include <cuda_fp8.h>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -171,11 +173,12 @@ __device__ __forceinline__ float ex2(float x) {
 
 // ------------------------------------------------------------ configuration --
 // PT: per-token key mode (32 key scales/zeros per page instead of D).
-template <int KB, int VB, int D, bool PT = false>
+// F8: fp8 e4m3 elements (8/8 bits, no page metadata, per-KV-head scales).
+template <int KB, int VB, int D, bool PT = false, bool F8 = false>
 struct Cfg {
   static constexpr bool kBf16 = (KB == 16);
   static constexpr int KS = D / 16;                       // 16-channel tiles
-  static constexpr int PB = (int)page_bytes_of(KB, VB, D, PT ? 1 : 0);
+  static constexpr int PB = (int)page_bytes_of(KB, VB, D, PT ? 1 : 0, F8 ? 1 : 0);
   // small pages: 3 CTAs per SM with 3-4 stages per warp; larger ones: 2 CTAs per SM
   static constexpr int MINB = PB <= 5000 ? 3 : 2;      // head-row kernel (64 accumulators per lane)
   static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;  // token-row kernel (32 accumulators per lane)
@@ -282,6 +285,30 @@ __device__ __forceinline__ void tile_frags(const uint32_t (&w)[TileWords<BITS>::
     b[2] = w[4 * tt + 1];
     b[3] = w[4 * tt + 3];
   }
+}
+
+// Two e4m3 values (low, high byte of v) -> f16x2, exact (e4m3 is a subset of f16).
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t v) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// fp8 counterparts of the 8-bit A and B fragments: the same bytes, converted
+// to their f16 values instead of being spread as integer codes.
+__device__ __forceinline__ void tile_afrag_f8(const uint32_t (&w)[TileWords<8>::N], int tt, uint32_t (&a)[4]) {
+  const uint32_t x = w[2 * tt], y = w[2 * tt + 1];
+  a[0] = e4m3x2_f16x2(x);
+  a[1] = e4m3x2_f16x2(x >> 16);
+  a[2] = e4m3x2_f16x2(y);
+  a[3] = e4m3x2_f16x2(y >> 16);
+}
+
+__device__ __forceinline__ void tile_frags_f8(const uint32_t (&w)[TileWords<8>::N], int tt, uint32_t (&b)[4]) {
+  const uint32_t x = w[2 * tt], y = w[2 * tt + 1];
+  b[0] = e4m3x2_f16x2(x);
+  b[1] = e4m3x2_f16x2(y);
+  b[2] = e4m3x2_f16x2(x >> 16);
+  b[3] = e4m3x2_f16x2(y >> 16);
 }
 
 // Online-softmax update with this page's scores sc[8] (log2 domain; tokens
@@ -493,6 +520,58 @@ __device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D
     for (int ks = 0; ks < 2; ++ks) {
       uint32_t b[4];
       tile_frags<VB>(w, ks, b);
+      mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
+      mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
+    }
+  }
+}
+
+// fp8 page, head rows: A = the segment's q' hi/lo fragments with the KV head's
+// key scale folded in, B = e4m3 keys as f16; p hi/lo against e4m3 values (the
+// value scale is applied once, to the accumulators).
+template <int D>
+__device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>& st, const uint32_t* qz, int lane) {
+  constexpr int KS = D / 16;
+  float s4[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s4[j][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<8>::N];
+    load_tile_words<8>(page, lane, dt, w);
+    const uint4 a = *reinterpret_cast<const uint4*>(qz + (dt * 32 + lane) * 4);
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      uint32_t b[4];
+      tile_frags_f8(w, tt, b);
+      mma_f16(s4[2 * tt], a.x, a.y, a.z, a.w, b[0], b[1]);
+      mma_f16(s4[2 * tt + 1], a.x, a.y, a.z, a.w, b[2], b[3]);
+    }
+  }
+  float sc[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    sc[2 * j] = s4[j][0] + s4[j][2];
+    sc[2 * j + 1] = s4[j][1] + s4[j][3];
+  }
+  softmax_update<D>(st, sc, kTau);
+  uint32_t pa[2][4];
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    split_f16(sc[4 * ks + 0], sc[4 * ks + 1], pa[ks][0], pa[ks][1]);
+    split_f16(sc[4 * ks + 2], sc[4 * ks + 3], pa[ks][2], pa[ks][3]);
+  }
+  const uint8_t* vblk = page + code_block_bytes(8, D);
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<8>::N];
+    load_tile_words<8>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t b[4];
+      tile_frags_f8(w, ks, b);
       mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
       mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
     }
@@ -887,6 +966,49 @@ __device__ __forceinline__ void attend_qpage_tok_pt(const uint8_t* page, TokStat
   }
 }
 
+// fp8 page, token rows: A = e4m3 keys/values as f16, B = the segment's q' parts
+// (key scale folded in) or p parts.
+template <int D>
+__device__ __forceinline__ void attend_f8page_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qkb)[D / 8],
+                                                  float* wscr, float partf, int lane) {
+  constexpr int KS = D / 16;
+  float* ptr = wscr + 4 * (D / 4 + 4) + 2 * kPageTokens;
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<8>::N];
+    load_tile_words<8>(page, lane, dt, w);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag_f8(w, mt, a);
+      mma_f16(s2[mt], a[0], a[1], a[2], a[3], qkb[2 * dt], qkb[2 * dt + 1]);
+    }
+  }
+  float sc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sc[i] = s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1];
+  tok_rescale_update<D>(st, sc, kTau);
+  uint32_t pb[2][2];
+  tok_pfrags<false>(ptr, sc, lane, partf, pb);
+  const uint8_t* vblk = page + code_block_bytes(8, D);
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<8>::N];
+    load_tile_words<8>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      tile_afrag_f8(w, ks, a);
+      mma_f16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
+    }
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void attend_bpage_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qbp)[D / 8],
                                                  float* wscr, float partf, float scale_log2, int lane) {
@@ -1054,10 +1176,10 @@ __device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p
   }
 }
 
-template <int KB, int VB, int D, bool TOK, bool PT>
-__global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK : Cfg<KB, VB, D, PT>::MINB)
+template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
+__global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_TOK : Cfg<KB, VB, D, PT, F8>::MINB)
     decode_mma_kernel(DecodeParams p) {
-  using C = Cfg<KB, VB, D, PT>;
+  using C = Cfg<KB, VB, D, PT, F8>;
   using State = typename std::conditional<TOK, TokState<D>, WarpState<D>>::type;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_last;
@@ -1204,12 +1326,14 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK :
         qf[dt * 4 + 3] = h2.y * p.scale_log2;
       }
       // q parts: the z-term B/A operands (per-channel keys) or the QK operands
-      // themselves (per-token keys: the 2-bit tauK channel factor is folded here)
-      constexpr float qhi = PT ? 1.f / C::tauK : 1.f;  // channels 2t+8, 2t+9 of each tile
+      // themselves (per-token keys: the 2-bit tauK channel factor is folded
+      // here; fp8: the KV head's key scale is)
+      const float qlo = F8 ? p.fp8_scales[sg.h] : 1.f;
+      const float qhi = PT ? 1.f / C::tauK : qlo;  // channels 2t+8, 2t+9 of each tile
       if constexpr (TOK) {
 #pragma unroll
         for (int dt = 0; dt < C::KS; ++dt) {
-          qzb[2 * dt] = part_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], partf);
+          qzb[2 * dt] = part_f16(qf[dt * 4 + 0] * qlo, qf[dt * 4 + 1] * qlo, partf);
           qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, partf);
         }
       } else {
@@ -1217,7 +1341,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK :
 #pragma unroll
           for (int dt = 0; dt < C::KS; ++dt) {
             uint4 q4;
-            split_f16(qf[dt * 4 + 0], qf[dt * 4 + 1], q4.x, q4.y);
+            split_f16(qf[dt * 4 + 0] * qlo, qf[dt * 4 + 1] * qlo, q4.x, q4.y);
             split_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, q4.z, q4.w);
             *reinterpret_cast<uint4*>(qz + (dt * 32 + lane) * 4) = q4;
           }
@@ -1245,9 +1369,16 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK :
     st.l = 0.f;
     st.vz = 0.f;
     bool converted = C::kBf16;
-    // quantized accumulators to true units: acc * 2^24 (/ sigmaV on channels with bit 3 set)
+    // quantized accumulators to true units: acc * 2^24 (/ sigmaV on channels with
+    // bit 3 set); fp8: acc * the KV head's value scale
     auto to_true_units = [&]() {
-      if constexpr (TOK) {
+      if constexpr (F8) {
+        const float vsc = p.fp8_scales[H + sg.h];
+#pragma unroll
+        for (int j = 0; j < (TOK ? D / 16 : D / 8); ++j)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) st.o[j][k] *= vsc;
+      } else if constexpr (TOK) {
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
           st.o[j][0] *= kTwo24;
@@ -1280,10 +1411,12 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK :
             const uint8_t* page = ring + stage * C::STAGE;
             if constexpr (TOK) {
               if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
+              else if constexpr (F8) attend_f8page_tok<D>(page, st, qzb, wscr, partf, lane);
               else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
               else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
             } else {
               if constexpr (C::kBf16) attend_bpage<D>(page, st, qb, p.scale_log2, lane);
+              else if constexpr (F8) attend_f8page<D>(page, st, qz, lane);
               else if constexpr (PT) attend_qpage_pt<KB, VB, D>(page, st, qz, qsum, wscr, lane);
               else attend_qpage<KB, VB, D>(page, st, qf, qz, wscr, lane);
             }
@@ -1431,20 +1564,20 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT>::MINB_TOK :
   }
 }
 
-template <int KB, int VB, int D, bool TOK, bool PT>
+template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
 cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
-  using C = Cfg<KB, VB, D, PT>;
+  using C = Cfg<KB, VB, D, PT, F8>;
   static int configured_smem = 0;
   static int occ_smem = -1, occ_blocks = 0;
   const int smem = C::smem_bytes(TOK, p.gqa, p.batch);
   if (smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK, PT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK, PT, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);
     if (e != cudaSuccess) return e;
     configured_smem = smem;
   }
   if (smem != occ_smem) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_blocks, decode_mma_kernel<KB, VB, D, TOK, PT>,
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_blocks, decode_mma_kernel<KB, VB, D, TOK, PT, F8>,
                                                                   kThreads, smem);
     if (e != cudaSuccess) return e;
     occ_smem = smem;
@@ -1453,18 +1586,22 @@ cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   grid = std::min<int64_t>(grid, p.n_units);
   grid = std::min<int64_t>(grid, p.max_ctas);
   if (grid < 1) grid = 1;
-  decode_mma_kernel<KB, VB, D, TOK, PT><<<(unsigned)grid, kThreads, smem, s>>>(p);
+  decode_mma_kernel<KB, VB, D, TOK, PT, F8><<<(unsigned)grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <int KB, int VB, int D>
 cudaError_t launch3(const DecodeParams& p, cudaStream_t s) {
   // token rows when the query group fits the 8 (head, part) columns
+  if constexpr (KB == 8 && VB == 8) {
+    if (p.fmt != 0)
+      return p.gqa <= 4 ? launch4<KB, VB, D, true, false, true>(p, s) : launch4<KB, VB, D, false, false, true>(p, s);
+  }
   if constexpr (KB != 16) {
     if (p.key_mode != 0)
-      return p.gqa <= 4 ? launch4<KB, VB, D, true, true>(p, s) : launch4<KB, VB, D, false, true>(p, s);
+      return p.gqa <= 4 ? launch4<KB, VB, D, true, true, false>(p, s) : launch4<KB, VB, D, false, true, false>(p, s);
   }
-  return p.gqa <= 4 ? launch4<KB, VB, D, true, false>(p, s) : launch4<KB, VB, D, false, false>(p, s);
+  return p.gqa <= 4 ? launch4<KB, VB, D, true, false, false>(p, s) : launch4<KB, VB, D, false, false, false>(p, s);
 }
 
 template <int D>

@@ -15,6 +15,8 @@
 // to finish merges: out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
 // Scores are kept in the log2 domain (scale includes log2(e)).
 
+#include <cuda_fp8.h>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -71,10 +73,16 @@ struct Smem {
   int last;
 };
 
+__device__ __forceinline__ float e4m3_to_float(uint32_t code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3)));
+}
+
 // Dequantize one full page into kd/vd (fp32). per_token_keys: the page holds 32
-// key scales/zeros in token order instead of D in channel-slot order.
+// key scales/zeros in token order instead of D in channel-slot order. fp8: the
+// elements are e4m3 values times the KV head's scales ksc/vsc.
 template <int KB, int VB, int D>
-__device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page, bool per_token_keys) {
+__device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page, bool per_token_keys, bool fp8, float ksc,
+                          float vsc) {
   constexpr int F = 2 * (D / 16);
   const uint8_t* kblk = page;
   const uint8_t* vblk = page + code_block_bytes(KB, D);
@@ -88,6 +96,18 @@ __device__ void load_page(Smem<KB, VB, D>& sm, const uint8_t* page, bool per_tok
         sm.kd[tok][dim] = __bfloat162float(__ushort_as_bfloat16((unsigned short)elem_code<16>(kblk, f, lane, e)));
         tile_elem(f, lane, e, true, tok, dim);
         sm.vd[tok][dim] = __bfloat162float(__ushort_as_bfloat16((unsigned short)elem_code<16>(vblk, f, lane, e)));
+      }
+    }
+  } else if (KB == 8 && VB == 8 && fp8) {
+    for (int idx = threadIdx.x; idx < F * 32; idx += kThreads) {
+      int f = idx >> 5, lane = idx & 31;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        int tok, dim;
+        tile_elem(f, lane, e, false, tok, dim);
+        sm.kd[tok][dim] = e4m3_to_float(elem_code<KB>(kblk, f, lane, e)) * ksc;
+        tile_elem(f, lane, e, true, tok, dim);
+        sm.vd[tok][dim] = e4m3_to_float(elem_code<VB>(vblk, f, lane, e)) * vsc;
       }
     }
   } else {
@@ -194,7 +214,8 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeParams p) {
 
   const uint8_t* base = p.pages + ((int64_t)(b * H + h) * p.max_pages) * p.page_bytes;
   for (int pg = p0; pg < p1; ++pg) {
-    load_page<KB, VB, D>(sm, base + (int64_t)pg * p.page_bytes, p.key_mode != 0);
+    load_page<KB, VB, D>(sm, base + (int64_t)pg * p.page_bytes, p.key_mode != 0, p.fmt != 0,
+                         p.fmt ? p.fp8_scales[h] : 1.f, p.fmt ? p.fp8_scales[p.n_kv_heads + h] : 1.f);
     attend_tokens<KB, VB, D, NACC>(sm, G, kPageTokens, p.scale_log2, acc);
   }
   if (s == nsplit - 1 && W > 0) {

@@ -31,8 +31,10 @@ constexpr int kMaxGqa = 8;
 __host__ __device__ constexpr int64_t code_block_bytes(int bits, int D) { return 4LL * D * bits; }
 
 // km: key mode (0 = per-channel keys, D scale/zero pairs; 1 = per-token keys, 32).
-__host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D, int km) {
-  return code_block_bytes(kb, D) + code_block_bytes(vb, D) + (kb == 16 ? 0 : (km ? 128LL : 4LL * D) + 128);
+// fmt: 0 = integer codes with page metadata, 1 = fp8 e4m3 (no page metadata).
+__host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D, int km, int fmt) {
+  return code_block_bytes(kb, D) + code_block_bytes(vb, D) +
+         ((kb == 16 || fmt) ? 0 : (km ? 128LL : 4LL * D) + 128);
 }
 
 // Tensor-core kernel split record: [G][D] accumulators, [G] maxima, [G] sums,
@@ -40,7 +42,8 @@ __host__ __device__ constexpr int64_t page_bytes_of(int kb, int vb, int D, int k
 __host__ __device__ constexpr int split_record_floats(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
 
 struct LayerState {
-  int kb = 0, vb = 0, km = 0;
+  int kb = 0, vb = 0, km = 0, fmt = 0;
+  float* fp8_scales = nullptr;   // fp8 layers: [2][n_kv_heads] key then value scales (device)
   int64_t page_bytes = 0;
   uint8_t* pages = nullptr;
   __nv_bfloat16* window = nullptr;
@@ -61,6 +64,8 @@ struct AppendParams {
   int max_pages;
   int n_kv_heads;
   int key_mode;          // 0 = per-channel keys, 1 = per-token keys
+  int fmt;               // 0 = integer codes, 1 = fp8 e4m3
+  const float* fp8_scales;  // fmt 1: [2][n_kv_heads] key then value scales
 };
 
 // Parameters of the decode attention kernel.
@@ -84,6 +89,8 @@ struct DecodeParams {
   int sm_count;
   int seg_overhead;      // tensor-core kernel: overhead units leading each segment (>= 0)
   int key_mode;          // 0 = per-channel keys, 1 = per-token keys
+  int fmt;               // 0 = integer codes, 1 = fp8 e4m3
+  const float* fp8_scales;  // fmt 1: [2][n_kv_heads] key then value scales
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
 };

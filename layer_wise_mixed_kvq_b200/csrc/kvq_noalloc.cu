@@ -70,9 +70,10 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
                                               const int32_t* seq_len, int64_t max_seq_len, const void* Q,
                                               int batch, float* out, void* stream) {
   if (!((pair.k_bits == 16 && pair.v_bits == 16) || (ok_bits(pair.k_bits) && ok_bits(pair.v_bits))) ||
-      pair.reserved != 0 || pair.key_mode > KVQ_KEY_PER_TOKEN ||
-      (pair.k_bits == 16 && pair.key_mode != KVQ_KEY_PER_CHANNEL))
+      pair.key_mode > KVQ_KEY_PER_TOKEN || (pair.k_bits == 16 && pair.key_mode != KVQ_KEY_PER_CHANNEL))
     return fail(KVQ_EINVAL, "unsupported pair");
+  if (pair.format != KVQ_FMT_INT)
+    return fail(KVQ_EINVAL, "fp8 layers need their per-head scales: use kvq_decode_attn on a cache");
   if (head_dim != 64 && head_dim != 128) return fail(KVQ_EINVAL, "head_dim must be 64 or 128");
   if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads != 0 || n_q_heads / n_kv_heads > kvq::kMaxGqa)
     return fail(KVQ_EINVAL, "n_q_heads must be a multiple of n_kv_heads with at most 8 per KV head");
@@ -121,7 +122,7 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.out = out;
   p.partials = partials;
   p.ctr = ctr;
-  p.page_bytes = kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim, pair.key_mode);
+  p.page_bytes = kvq::page_bytes_of(pair.k_bits, pair.v_bits, head_dim, pair.key_mode, KVQ_FMT_INT);
   p.key_mode = pair.key_mode;
   p.max_pages = (int)max_pages;
   p.n_kv_heads = n_kv_heads;

@@ -17,24 +17,26 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 KVQ_OK, KVQ_EINVAL, KVQ_ECAPACITY, KVQ_ENOMEM, KVQ_ECUDA = 0, 1, 2, 3, 4
 KVQ_BF16, KVQ_F32 = 0, 1
 KVQ_KEY_PER_CHANNEL, KVQ_KEY_PER_TOKEN = 0, 1
+KVQ_FMT_INT, KVQ_FMT_FP8 = 0, 1
 
 #: every symbol the C header declares
 EXPORTS = (
     "kvq_page_bytes", "kvq_equiv_bits", "kvq_cache_pool_bytes", "kvq_cache_create", "kvq_cache_destroy",
     "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
     "kvq_export_bytes", "kvq_export_layer", "kvq_sync", "kvq_launch_count", "kvq_last_error",
-    "kvq_status_string",
+    "kvq_status_string", "kvq_set_fp8_scales",
 )
 
 
 class kvq_pair(ctypes.Structure):
     _fields_ = [("k_bits", ctypes.c_uint8), ("v_bits", ctypes.c_uint8), ("key_mode", ctypes.c_uint8),
-                ("reserved", ctypes.c_uint8)]
+                ("format", ctypes.c_uint8)]
 
 
 def _pair(p) -> kvq_pair:
-    """(k_bits, v_bits) or (k_bits, v_bits, key_mode) -> kvq_pair."""
-    return kvq_pair(int(p[0]), int(p[1]), int(p[2]) if len(p) > 2 else KVQ_KEY_PER_CHANNEL, 0)
+    """(k_bits, v_bits[, key_mode[, format]]) -> kvq_pair."""
+    return kvq_pair(int(p[0]), int(p[1]), int(p[2]) if len(p) > 2 else KVQ_KEY_PER_CHANNEL,
+                    int(p[3]) if len(p) > 3 else KVQ_FMT_INT)
 
 
 class KVQError(RuntimeError):
@@ -71,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "kvq_launch_count": (c.c_int64, [P]),
         "kvq_last_error": (c.c_char_p, []),
         "kvq_status_string": (c.c_char_p, [c.c_int]),
+        "kvq_set_fp8_scales": (c.c_int, [P, c.c_int, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -189,6 +192,14 @@ def kvq_decode_attn_noalloc(pair, head_dim, n_q_heads, n_kv_heads, pages, max_pa
                                        int(n_kv_heads), _dev_ptr(pages), int(max_pages), _dev_ptr(window),
                                        _dev_ptr(seq_len), int(max_seq_len), _dev_ptr(Q), int(Q.shape[0]),
                                        _dev_ptr(out), _stream(stream)))
+
+
+def kvq_set_fp8_scales(cache, layer, k_scale, v_scale) -> None:
+    """Per-KV-head scales of an fp8 layer (sequences of n_kv_heads floats; host)."""
+    ks = (ctypes.c_float * len(k_scale))(*[float(x) for x in k_scale])
+    vs = (ctypes.c_float * len(v_scale))(*[float(x) for x in v_scale])
+    _check(lib.kvq_set_fp8_scales(ctypes.c_void_p(cache), int(layer), ctypes.cast(ks, ctypes.c_void_p),
+                                  ctypes.cast(vs, ctypes.c_void_p)))
 
 
 def kvq_set_split_pages(cache, pages_per_split: int) -> None:

@@ -15,6 +15,10 @@ and the 3.25 / 4.0-bit results):
 * ``llama_k4v4``     -- 32 layers K4V4, batch 16, context 4096 + 1.
 * ``llama_k4v4_pt``  -- the same shapes, draws and seed with per-token keys
   (third pair field 1: the per-token-asym key mode).
+* ``llama_fp8_bf16``  -- the worked example's split of 32 layers: 8 kept in
+  BF16 (the four boundary layers at each end) and 24 FP8 e4m3 layers (pair
+  (8, 8, 0, 1)) with fixed per-KV-head scales; llama shapes, batch 16,
+  context 4096 + 1, seed 5.
 * ``llama_mixed325`` -- layers 0,1,2,31 K4V8; 3-26 K4V2; 27-30 K2V2; batch 64,
   prefill 128 then 512 decode steps.
 * ``qwen_mixed40``   -- 28 layers: 0-3 K8V4, 4-19 K4V4, 20-27 K4V2; batch 32,
@@ -51,6 +55,7 @@ class Workload:
     seed: int
     ragged: tuple = ()          # (lo, hi) per-sequence context range, or ()
     notes: str = field(default="")
+    fp8_scales: tuple = ()      # fp8 layers: ((k scale per KV head), (v scale per KV head)), or ()
 
     @property
     def n_layers(self) -> int:
@@ -73,6 +78,10 @@ def _llama_mixed_map():
     return tuple(m)
 
 
+def _fp8_bf16_map():
+    return tuple((16, 16) if (layer < 4 or layer >= 28) else (8, 8, 0, 1) for layer in range(32))
+
+
 def _qwen_map():
     m = []
     for layer in range(28):
@@ -93,6 +102,10 @@ WORKLOADS = {
     "tiny_k8v4": Workload("tiny_k8v4", ((8, 4),), 1, 2, 2, 64, 256, 1, "normal", 2, 10.0, "f32", 0),
     "llama_k4v4": Workload("llama_k4v4", tuple([(4, 4)] * 32), 16, 32, 8, 128, 4096, 1, "normal", 4,
                            8.0, "bf16", 1),
+    "llama_fp8_bf16": Workload("llama_fp8_bf16", _fp8_bf16_map(), 16, 32, 8, 128, 4096, 1, "normal", 4,
+                               8.0, "bf16", 5,
+                               fp8_scales=(tuple(0.0625 * (1 + h / 8) for h in range(8)),
+                                           tuple(0.03125 * (1 + h / 16) for h in range(8)))),
     "llama_k4v4_pt": Workload("llama_k4v4_pt", tuple([(4, 4, 1)] * 32), 16, 32, 8, 128, 4096, 1, "normal", 4,
                               8.0, "bf16", 1),
     "llama_mixed325": Workload("llama_mixed325", _llama_mixed_map(), 64, 32, 8, 128, 128, 512, "normal",

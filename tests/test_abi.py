@@ -20,7 +20,7 @@ def kvq():
 def _declared_symbols():
     src = open(os.path.join(ROOT, "include", "kvq.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_boundary():
@@ -65,12 +65,21 @@ def test_page_bytes_per_token_keys(kvq):
                 assert kvq.kvq_page_bytes((k, v, kvq.KVQ_KEY_PER_TOKEN), D) == 4 * D * (k + v) + 256
     assert kvq.kvq_page_bytes((16, 16, kvq.KVQ_KEY_PER_TOKEN), 128) == 0   # bf16 layers have no key mode
     assert kvq.kvq_page_bytes((4, 4, 2), 128) == 0                         # unknown mode
-    bad = kvq.kvq_pair(4, 4, 0, 1)                                          # reserved byte set
-    assert kvq.lib.kvq_page_bytes(bad, 128) == 0
+    assert kvq.kvq_page_bytes((4, 4, 0, 1), 128) == 0                      # fp8 needs 8/8 bits
+    assert kvq.kvq_page_bytes((8, 8, 1, 1), 128) == 0                      # fp8 has no key mode
+    assert kvq.kvq_page_bytes((8, 8, 0, 2), 128) == 0                      # unknown format
     assert kvq.kvq_equiv_bits([(4, 4, 1), (4, 2, 0)]) == 3.5               # the mode does not change bits
     pc = kvq.kvq_cache_pool_bytes([(4, 4)] * 2, 32, 8, 128, 16, 4097)
     pt = kvq.kvq_cache_pool_bytes([(4, 4, 1)] * 2, 32, 8, 128, 16, 4097)
     assert 0 < pt < pc
+
+
+def test_fp8_pairs(kvq):
+    for D in (64, 128):
+        assert kvq.kvq_page_bytes((8, 8, 0, kvq.KVQ_FMT_FP8), D) == 64 * D   # e4m3 elements, no page metadata
+    assert kvq.kvq_equiv_bits([(16, 16)] * 8 + [(8, 8, 0, 1)] * 24) == 10.0
+    with pytest.raises(kvq.KVQError):
+        kvq.kvq_cache_create([(8, 8, 1, 1)], 8, 8, 128, 4, 1024)
 
 
 def test_pool_bytes_validation(kvq):

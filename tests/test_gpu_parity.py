@@ -40,11 +40,17 @@ def _check_attention(got, ref, what=""):
 class Pair:
     """A one-layer GPU cache and its oracle twin, fed the same inputs."""
 
-    def __init__(self, kvq, oracle, pair, batch, hq, hkv, D, max_tokens, dtype=torch.bfloat16):
+    def __init__(self, kvq, oracle, pair, batch, hq, hkv, D, max_tokens, dtype=torch.bfloat16, fp8_scales=None):
         self.kvq, self.pair, self.batch, self.hq, self.hkv, self.D = kvq, pair, batch, hq, hkv, D
         self.dtype = dtype
         self.cache = kvq.kvq_cache_create([pair], hq, hkv, D, batch, max_tokens)
-        self.ref = oracle.OracleLayer(pair[0], pair[1], batch, hkv, D, key_mode=pair[2] if len(pair) > 2 else 0)
+        fmt = pair[3] if len(pair) > 3 else 0
+        ks = vs = None
+        if fmt:
+            ks, vs = fp8_scales if fp8_scales is not None else ([1.0] * hkv, [1.0] * hkv)
+            kvq.kvq_set_fp8_scales(self.cache, 0, ks, vs)
+        self.ref = oracle.OracleLayer(pair[0], pair[1], batch, hkv, D, key_mode=pair[2] if len(pair) > 2 else 0,
+                                      fmt=fmt, k_scales=ks, v_scales=vs)
 
     def close(self):
         self.kvq.kvq_cache_destroy(self.cache)
