@@ -287,28 +287,39 @@ __device__ __forceinline__ void tile_frags(const uint32_t (&w)[TileWords<BITS>::
   }
 }
 
-// Two e4m3 values (low, high byte of v) -> f16x2, exact (e4m3 is a subset of f16).
-__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t v) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v & 0xFFFFu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Two e4m3 bytes of x (bytes 0, 1 for kSelLo; 2, 3 for kSelHi) -> f16x2 whose
+// values are the e4m3 values times 2^-8, exactly. prmt puts each byte in the
+// low half of a 16-bit lane with its sign replicated into the high byte; a
+// shift by 7 moves the seven magnitude bits (4 exponent, 3 mantissa) to f16
+// bits 7..13 and a sign copy to bit 15; the mask keeps those. The f16 exponent
+// bias (15) exceeds e4m3's (7) by 8, which gives the 2^-8 for normal and
+// subnormal codes alike (a subnormal e4m3 m*2^-9 becomes the f16 subnormal
+// m*2^7*2^-24).
+constexpr uint32_t kSelLo = 0x9180u, kSelHi = 0xB3A2u;
+constexpr float kF8Unit = 256.0f;  // true value = f16 value * 2^8
+
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t x, uint32_t sel) {
+  uint32_t t;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(x), "r"(sel));
+  return (t << 7) & 0xBF80BF80u;
 }
 
-// fp8 counterparts of the 8-bit A and B fragments: the same bytes, converted
-// to their f16 values instead of being spread as integer codes.
+// fp8 counterparts of the 8-bit A and B fragments: the same bytes, as f16
+// values (times 2^-8) instead of integer codes.
 __device__ __forceinline__ void tile_afrag_f8(const uint32_t (&w)[TileWords<8>::N], int tt, uint32_t (&a)[4]) {
   const uint32_t x = w[2 * tt], y = w[2 * tt + 1];
-  a[0] = e4m3x2_f16x2(x);
-  a[1] = e4m3x2_f16x2(x >> 16);
-  a[2] = e4m3x2_f16x2(y);
-  a[3] = e4m3x2_f16x2(y >> 16);
+  a[0] = e4m3x2_f16x2(x, kSelLo);
+  a[1] = e4m3x2_f16x2(x, kSelHi);
+  a[2] = e4m3x2_f16x2(y, kSelLo);
+  a[3] = e4m3x2_f16x2(y, kSelHi);
 }
 
 __device__ __forceinline__ void tile_frags_f8(const uint32_t (&w)[TileWords<8>::N], int tt, uint32_t (&b)[4]) {
   const uint32_t x = w[2 * tt], y = w[2 * tt + 1];
-  b[0] = e4m3x2_f16x2(x);
-  b[1] = e4m3x2_f16x2(y);
-  b[2] = e4m3x2_f16x2(x >> 16);
-  b[3] = e4m3x2_f16x2(y >> 16);
+  b[0] = e4m3x2_f16x2(x, kSelLo);
+  b[1] = e4m3x2_f16x2(y, kSelLo);
+  b[2] = e4m3x2_f16x2(x, kSelHi);
+  b[3] = e4m3x2_f16x2(y, kSelHi);
 }
 
 // Online-softmax update with this page's scores sc[8] (log2 domain; tokens
@@ -527,8 +538,9 @@ __device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D
 }
 
 // fp8 page, head rows: A = the segment's q' hi/lo fragments with the KV head's
-// key scale folded in, B = e4m3 keys as f16; p hi/lo against e4m3 values (the
-// value scale is applied once, to the accumulators).
+// key scale folded in, B = e4m3 keys as f16 (times 2^-8, undone on the scores);
+// p hi/lo against e4m3 values (the value scale and 2^8 are applied once, to
+// the accumulators).
 template <int D>
 __device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>& st, const uint32_t* qz, int lane) {
   constexpr int KS = D / 16;
@@ -553,8 +565,8 @@ __device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>&
   float sc[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    sc[2 * j] = s4[j][0] + s4[j][2];
-    sc[2 * j + 1] = s4[j][1] + s4[j][3];
+    sc[2 * j] = (s4[j][0] + s4[j][2]) * kF8Unit;
+    sc[2 * j + 1] = (s4[j][1] + s4[j][3]) * kF8Unit;
   }
   softmax_update<D>(st, sc, kTau);
   uint32_t pa[2][4];
@@ -991,7 +1003,7 @@ __device__ __forceinline__ void attend_f8page_tok(const uint8_t* page, TokState<
   }
   float sc[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) sc[i] = s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1];
+  for (int i = 0; i < 4; ++i) sc[i] = (s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1]) * kF8Unit;
   tok_rescale_update<D>(st, sc, kTau);
   uint32_t pb[2][2];
   tok_pfrags<false>(ptr, sc, lane, partf, pb);
@@ -1373,7 +1385,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     // bit 3 set); fp8: acc * the KV head's value scale
     auto to_true_units = [&]() {
       if constexpr (F8) {
-        const float vsc = p.fp8_scales[H + sg.h];
+        const float vsc = p.fp8_scales[H + sg.h] * kF8Unit;
 #pragma unroll
         for (int j = 0; j < (TOK ? D / 16 : D / 8); ++j)
 #pragma unroll
