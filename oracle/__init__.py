@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "oracle_layer_set_fp8_scales": (None, [P, P, P]),
             "oracle_layer_free": (None, [P]),
             "oracle_layer_len": (c.c_int64, [P, c.c_int]),
+            "oracle_layer_error": (c.c_int64, [P, P]),
             "oracle_layer_append": (None, [P, P, P, P, c.c_int]),
             "oracle_layer_export_bytes": (c.c_int64, [P, c.c_int]),
             "oracle_layer_export": (None, [P, c.c_int, P]),
@@ -211,6 +212,12 @@ class OracleLayer:
 
     def length(self, b: int) -> int:
         return int(lib().oracle_layer_len(self._h, b))
+
+    def error(self):
+        """(sum (k-k^)^2, sum k^2, sum (v-v^)^2, sum v^2, quantized elements per K and per V)."""
+        out = np.zeros(4, dtype=np.float64)
+        n = int(lib().oracle_layer_error(self._h, _ptr(out)))
+        return (*[float(x) for x in out], n)
 
     def append(self, K: np.ndarray, V: np.ndarray, n_new) -> None:
         """K, V: [sum(n_new), n_kv_heads, head_dim] values (fp32 or bf16-valued)."""

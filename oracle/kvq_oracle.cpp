@@ -41,6 +41,11 @@
 //  * empty sequence: output 0.
 //  * per-token key mode keeps the same 32-token pages and bf16 residual window:
 //    a key token is quantized when its page fills, like a value token.
+//  * per-layer quantization error report (OpenReview rebuttal, Table 3 and the
+//    layer-wise error figures the pages cite: quantization error is tracked
+//    per layer): sums over every element a page flush quantizes of
+//    (x - x_hat)^2 and x^2, keys and values separately, in fp64, plus the
+//    element counts; bf16 layers add nothing.
 //  * FP8 layer format (llms-explorer facts page: vLLM-style FP8 KV cache with
 //    per-attention-head scales and BF16 skip layers; machinoai Q&A section 2
 //    worked example of BF16 and FP8 layers): each key/value element of KV head
@@ -456,6 +461,8 @@ struct Layer {
   int kb, vb, key_mode, fmt, batch, hkv, D;
   std::vector<Seq> seqs;
   std::vector<float> kscale, vscale;  // fp8 format: per KV head
+  double err[4] = {0, 0, 0, 0};       // sum (k - k_hat)^2, sum k^2, sum (v - v_hat)^2, sum v^2
+  int64_t elements = 0;               // quantized elements of K (= of V)
 };
 
 }  // namespace
@@ -544,6 +551,14 @@ void oracle_layer_set_fp8_scales(void* p, const float* kscale, const float* vsca
 
 int64_t oracle_layer_len(void* p, int b) { return static_cast<Layer*>(p)->seqs[b].len; }
 
+// Quantization error report: out = {sum (k - k_hat)^2, sum k^2, sum (v - v_hat)^2,
+// sum v^2}; returns the number of quantized key (= value) elements.
+int64_t oracle_layer_error(void* p, double* out) {
+  Layer* L = static_cast<Layer*>(p);
+  for (int i = 0; i < 4; ++i) out[i] = L->err[i];
+  return L->elements;
+}
+
 // Append n_new[b] tokens to every sequence b < batch. K and V are packed
 // [sum(n_new)][n_kv_heads][D] fp32 (rounded to bf16 on entry). Tokens enter the
 // window one at a time; the window is quantized as one page the moment it
@@ -568,6 +583,20 @@ void oracle_layer_append(void* p, const float* K, const float* V, const int32_t*
           s.pages[h].resize(off + pb);
           build_page(s.pages[h].data() + off, s.wk[h].data(), s.wv[h].data(), D, L->kb, L->vb, L->key_mode, L->fmt,
                      L->kscale[h], L->vscale[h]);
+          if (L->kb != 16) {
+            // quantization error of this flush against its bf16 inputs
+            std::vector<double> Kh(32 * D), Vh(32 * D);
+            dequant_page(s.pages[h].data() + off, D, L->kb, L->vb, L->key_mode, L->fmt, L->kscale[h], L->vscale[h],
+                         Kh.data(), Vh.data());
+            for (int i = 0; i < 32 * D; ++i) {
+              double k = bf16_to_f32(s.wk[h][i]), v = bf16_to_f32(s.wv[h][i]);
+              L->err[0] += (k - Kh[i]) * (k - Kh[i]);
+              L->err[1] += k * k;
+              L->err[2] += (v - Vh[i]) * (v - Vh[i]);
+              L->err[3] += v * v;
+            }
+            L->elements += 32LL * D;
+          }
           s.wk[h].clear();
           s.wv[h].clear();
         }
