@@ -148,7 +148,8 @@ kvq_status kvq_cache_create(const kvq_pair* layer_map, int n_layers, int n_q_hea
 /* Release the cache (synchronises the device first). NULL is a no-op. */
 void kvq_cache_destroy(kvq_cache* cache);
 
-/* Empty every sequence of every layer (enqueued on `stream`). */
+/* Empty every sequence of every layer and zero the error reports (enqueued on
+ * `stream`). */
 kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
 
 /* Append n_new[b] tokens to sequence b of `layer`, for b < batch ([rebut]
@@ -216,6 +217,21 @@ kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n_q_heads, i
                                    const int32_t* seq_len, int64_t max_seq_len, const void* Q,
                                    int batch, float* out, void* stream);
 
+/* Per-layer quantization error report ([rebut] Table 3 and the layer-wise
+ * error figures: quantization error is tracked layer by layer). Sums over every
+ * element that a page flush of `layer` has quantized since creation or the last
+ * reset, in fp64: (k - k_hat)^2, k^2, (v - v_hat)^2, v^2, with k, v the bf16
+ * inputs and k_hat, v_hat their dequantized values; `elements` counts the
+ * quantized key (= value) elements. Window tokens and bf16 layers add nothing.
+ * The relative errors are k_sq_err / k_sq and v_sq_err / v_sq. */
+typedef struct {
+  double k_sq_err, k_sq, v_sq_err, v_sq;
+  int64_t elements;
+} kvq_error_stats;
+
+/* Read `layer`'s report (synchronises the device). */
+kvq_status kvq_layer_error(const kvq_cache* cache, int layer, kvq_error_stats* out);
+
 /* Set the per-KV-head fp32 scales of an fp8 layer (host arrays of n_kv_heads
  * values, each finite and > 0; every head defaults to 1.0). Stored elements are
  * e4m3(x / scale) and read back as e4m3 * scale. The layer must be empty (no
@@ -246,8 +262,20 @@ int64_t kvq_export_bytes(const kvq_cache* cache, int layer, int batch);
 kvq_status kvq_export_layer(const kvq_cache* cache, int layer, int batch, void* host_dst,
                             size_t bytes);
 
-/* Wait for the cache's work and report any asynchronous CUDA error. */
+/* Wait for the cache's work and report any asynchronous CUDA error, or
+ * KVQ_ECAPACITY if a one-token append launched from a replayed CUDA graph met a
+ * full sequence (that sequence was left unchanged). */
 kvq_status kvq_sync(kvq_cache* cache);
+
+/* CUDA graphs. A decode step -- kvq_append with one token for every sequence,
+ * then kvq_decode_attn -- can be captured on a stream and replayed: those two
+ * calls enqueue kernels only (no host synchronisation, no host-to-device copy),
+ * and the kernels read the sequence lengths on the device. Replays do not run
+ * host code, so the host's mirror of the lengths (kvq_seq_len, kvq_bytes,
+ * kvq_export_layer, capacity checks) lags until this call copies the device
+ * lengths back (synchronises the device). Multi-token appends copy a plan from
+ * the host and must not be captured. */
+kvq_status kvq_refresh_lengths(kvq_cache* cache);
 
 /* Number of kernels the library has launched on this cache so far. */
 int64_t kvq_launch_count(const kvq_cache* cache);

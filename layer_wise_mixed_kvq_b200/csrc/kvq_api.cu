@@ -83,7 +83,7 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
     size_t wr = round_up((size_t)max_batch * n_kv_heads * 2 * kvq::kPageTokens * head_dim * 2);
     g.page_region.push_back(pr);
     g.window_region.push_back(wr);
-    total += pr + wr + round_up((size_t)max_batch * 4) + round_up((size_t)n_kv_heads * 2 * 4);
+    total += pr + wr + round_up((size_t)max_batch * 4) + round_up((size_t)n_kv_heads * 2 * 4) + round_up(5 * 8);
   }
   g.len_region = round_up((size_t)max_batch * 4);
   g.partial_slots = partial_slots_for(max_batch, n_kv_heads);
@@ -232,6 +232,8 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     p += g.len_region;
     L.fp8_scales = reinterpret_cast<float*>(p);
     p += round_up((size_t)n_kv_heads * 2 * 4);
+    L.err_stats = reinterpret_cast<double*>(p);
+    p += round_up(5 * 8);
     L.host_len.assign(max_batch, 0);
   }
   c->partials = reinterpret_cast<float*>(p);
@@ -253,6 +255,7 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     e = cudaMemset(c->layers[l].len, 0, (size_t)max_batch * 4);
     if (e == cudaSuccess)
       e = cudaMemcpy(c->layers[l].fp8_scales, ones.data(), ones.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(c->layers[l].err_stats, 0, 5 * 8);
   }
   if (e == cudaSuccess) e = cudaMemset(c->merge_ctr, 0, (size_t)max_batch * n_kv_heads * 4);
   if (e == cudaSuccess) e = cudaMemset(c->append_ctr, 0, (size_t)max_batch * 4);
@@ -281,9 +284,26 @@ kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (auto& L : c->layers) {
     cudaError_t e = cudaMemsetAsync(L.len, 0, (size_t)c->max_batch * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.err_stats, 0, 5 * 8, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     std::fill(L.host_len.begin(), L.host_len.end(), 0);
   }
+  return KVQ_OK;
+}
+
+kvq_status kvq_layer_error(const kvq_cache* c, int layer, kvq_error_stats* out) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (!out) return fail(KVQ_EINVAL, "out is null");
+  double h[5];
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(h, c->layers[layer].err_stats, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error report)");
+  out->k_sq_err = h[0];
+  out->k_sq = h[1];
+  out->v_sq_err = h[2];
+  out->v_sq = h[3];
+  out->elements = (int64_t)h[4];
   return KVQ_OK;
 }
 
@@ -354,6 +374,9 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
   p.key_mode = L.km;
   p.fmt = L.fmt;
   p.fp8_scales = L.fp8_scales;
+  p.err_stats = L.err_stats;
+  p.max_tokens = c->max_tokens;
+  p.err = c->err;
   p.plan = nullptr;
   if (!all_one) {
     // multi-token append: per-sequence plan (start, count, row offset, items)
@@ -518,8 +541,24 @@ kvq_status kvq_sync(kvq_cache* c) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(err)");
   if (flag) {
     cudaMemset(c->err, 0, 4);
+    if (flag == 2)
+      return fail(KVQ_ECAPACITY, "a one-token append (replayed graph) found a sequence at max_tokens; "
+                                 "that sequence was left unchanged");
     return fail(KVQ_ECUDA, "decode attention: a page copy did not complete within its wait limit");
   }
+  return KVQ_OK;
+}
+
+kvq_status kvq_refresh_lengths(kvq_cache* c) {
+  if (!c) return fail(KVQ_EINVAL, "cache is null");
+  cudaError_t e = cudaDeviceSynchronize();
+  std::vector<int32_t> tmp((size_t)c->max_batch);
+  for (auto& L : c->layers) {
+    if (e == cudaSuccess) e = cudaMemcpy(tmp.data(), L.len, tmp.size() * 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) break;
+    for (int b = 0; b < c->max_batch; ++b) L.host_len[b] = tmp[b];
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "kvq_refresh_lengths");
   return KVQ_OK;
 }
 

@@ -24,6 +24,9 @@
 // FP8 layers (e4m3 elements, per-KV-head scale s_h; llms-explorer facts page on
 // vLLM FP8 KV caches): code = e4m3(x / s_h), one IEEE division, then round to
 // nearest even with saturation at 448.
+// Every flush also adds its quantization error to the layer's report: sums of
+// (x - x_hat)^2 and x^2 for keys and values, in fp64 (x_hat = code * s + z, or
+// e4m3 value * s_h, is exact in fp64).
 
 #include <cuda_fp8.h>
 
@@ -163,7 +166,10 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
     if (item == 0 && h == 0 && threadIdx.x == 0) a.len[b] = T0 + n;
   } else {
     // One token per sequence; every CTA of sequence b reads the old length,
-    // and the last one to have read it publishes the new length.
+    // and the last one to have read it publishes the new length. The host
+    // checks capacity before launching, but a replayed CUDA graph does not run
+    // host code: a full sequence is left unchanged here and the cache's error
+    // flag is raised.
     if (threadIdx.x == 0) {
       int t0 = a.len[b];
       s_T0 = t0;
@@ -171,11 +177,15 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
       if (atomicAdd(&a.ctr[b], 1) == H - 1) {
         a.ctr[b] = 0;
         __threadfence();
-        a.len[b] = t0 + 1;
+        if (t0 < a.max_tokens) a.len[b] = t0 + 1;
       }
     }
     __syncthreads();
     T0 = s_T0;
+    if (T0 >= a.max_tokens) {
+      if (threadIdx.x == 0 && a.err) atomicExch(a.err, 2);
+      return;
+    }
     n = 1;
     off = b;
     items = 1;
@@ -230,13 +240,23 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         xs[1][t][d] = __bfloat162float(vx);
       }
       __syncthreads();
+      double err[4] = {0.0, 0.0, 0.0, 0.0};  // this thread's share of the error report
+      auto add_err = [&](int r, float x, double xh) {
+        const double dx = (double)x - xh;
+        err[2 * r] += dx * dx;
+        err[2 * r + 1] += (double)x * (double)x;
+      };
       if (a.fmt != 0) {
         if constexpr (KB == 8 && VB == 8) {
           const float ksc = a.fp8_scales[h], vsc = a.fp8_scales[H + h];
           for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
             const int t = idx / D, d = idx % D;
-            cs[0][t][d] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(xs[0][t][d], ksc), __NV_SATFINITE, __NV_E4M3);
-            cs[1][t][d] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(xs[1][t][d], vsc), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8_storage_t ck = __nv_cvt_float_to_fp8(__fdiv_rn(xs[0][t][d], ksc), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8_storage_t cv = __nv_cvt_float_to_fp8(__fdiv_rn(xs[1][t][d], vsc), __NV_SATFINITE, __NV_E4M3);
+            cs[0][t][d] = (uint8_t)ck;
+            cs[1][t][d] = (uint8_t)cv;
+            add_err(0, xs[0][t][d], (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(ck, __NV_E4M3))) * ksc);
+            add_err(1, xs[1][t][d], (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(cv, __NV_E4M3))) * vsc);
           }
           __syncthreads();
           store_block<8, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
@@ -267,9 +287,14 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           }
           QParams q = make_qparams(mn, mx, qmax);
+          const double s = (double)__half2float(q.s_h), z = (double)q.z;
 #pragma unroll
-          for (int k = 0; k < D / 32; ++k)
-            cs[r][t][lane + 32 * k] = (uint8_t)quant_code(xs[r][t][lane + 32 * k], q, qmax);
+          for (int k = 0; k < D / 32; ++k) {
+            const float x = xs[r][t][lane + 32 * k];
+            const uint32_t c = quant_code(x, q, qmax);
+            cs[r][t][lane + 32 * k] = (uint8_t)c;
+            add_err(r, x, (double)c * s + z);
+          }
           if (lane == 0) {
             sdst[t] = q.s_h;
             zdst[t] = q.z_h;
@@ -288,8 +313,13 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
           mx = fmaxf(mx, x);
         }
         QParams q = make_qparams(mn, mx, qmax);
+        const double s = (double)__half2float(q.s_h), z = (double)q.z;
 #pragma unroll 8
-        for (int t = 0; t < kPageTokens; ++t) cs[0][t][d] = (uint8_t)quant_code(xs[0][t][d], q, qmax);
+        for (int t = 0; t < kPageTokens; ++t) {
+          const uint32_t c = quant_code(xs[0][t][d], q, qmax);
+          cs[0][t][d] = (uint8_t)c;
+          add_err(0, xs[0][t][d], (double)c * s + z);
+        }
         int slot = kmeta_slot<D>(d);
         kscale[slot] = q.s_h;
         kzero[slot] = q.z_h;
@@ -300,6 +330,24 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
       store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
       store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
       }
+      // this flush's error sums: warp shuffles, then one fp64 atomic per sum
+      __shared__ double red[kThreads / 32][4];
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        double v = err[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp][i] = v;
+      }
+      __syncthreads();
+      if (a.err_stats && threadIdx.x < 4) {
+        double v = 0.0;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) v += red[w][threadIdx.x];
+        atomicAdd(&a.err_stats[threadIdx.x], v);
+      }
+      if (a.err_stats && threadIdx.x == 4) atomicAdd(&a.err_stats[4], (double)(kPageTokens * D));
     }
   }
 

@@ -44,6 +44,7 @@ __host__ __device__ constexpr int split_record_floats(int G, int D) { return G *
 struct LayerState {
   int kb = 0, vb = 0, km = 0, fmt = 0;
   float* fp8_scales = nullptr;   // fp8 layers: [2][n_kv_heads] key then value scales (device)
+  double* err_stats = nullptr;   // [4] sums (k-k^)^2, k^2, (v-v^)^2, v^2, then [1] element count (device)
   int64_t page_bytes = 0;
   uint8_t* pages = nullptr;
   __nv_bfloat16* window = nullptr;
@@ -66,6 +67,9 @@ struct AppendParams {
   int key_mode;          // 0 = per-channel keys, 1 = per-token keys
   int fmt;               // 0 = integer codes, 1 = fp8 e4m3
   const float* fp8_scales;  // fmt 1: [2][n_kv_heads] key then value scales
+  double* err_stats;     // quantization error sums of the layer, see LayerState
+  int64_t max_tokens;    // one-token mode: a full sequence is left unchanged and flags err
+  int32_t* err;          // cache error flag (2 = one-token append past max_tokens)
 };
 
 // Parameters of the decode attention kernel.

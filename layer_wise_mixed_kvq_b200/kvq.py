@@ -24,7 +24,7 @@ EXPORTS = (
     "kvq_page_bytes", "kvq_equiv_bits", "kvq_cache_pool_bytes", "kvq_cache_create", "kvq_cache_destroy",
     "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
     "kvq_export_bytes", "kvq_export_layer", "kvq_sync", "kvq_launch_count", "kvq_last_error",
-    "kvq_status_string", "kvq_set_fp8_scales",
+    "kvq_status_string", "kvq_set_fp8_scales", "kvq_layer_error", "kvq_refresh_lengths",
 )
 
 
@@ -37,6 +37,11 @@ def _pair(p) -> kvq_pair:
     """(k_bits, v_bits[, key_mode[, format]]) -> kvq_pair."""
     return kvq_pair(int(p[0]), int(p[1]), int(p[2]) if len(p) > 2 else KVQ_KEY_PER_CHANNEL,
                     int(p[3]) if len(p) > 3 else KVQ_FMT_INT)
+
+
+class kvq_error_stats(ctypes.Structure):
+    _fields_ = [("k_sq_err", ctypes.c_double), ("k_sq", ctypes.c_double), ("v_sq_err", ctypes.c_double),
+                ("v_sq", ctypes.c_double), ("elements", ctypes.c_int64)]
 
 
 class KVQError(RuntimeError):
@@ -74,6 +79,8 @@ def _load() -> ctypes.CDLL:
         "kvq_last_error": (c.c_char_p, []),
         "kvq_status_string": (c.c_char_p, [c.c_int]),
         "kvq_set_fp8_scales": (c.c_int, [P, c.c_int, P, P]),
+        "kvq_layer_error": (c.c_int, [P, c.c_int, c.POINTER(kvq_error_stats)]),
+        "kvq_refresh_lengths": (c.c_int, [P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -194,6 +201,13 @@ def kvq_decode_attn_noalloc(pair, head_dim, n_q_heads, n_kv_heads, pages, max_pa
                                        _dev_ptr(out), _stream(stream)))
 
 
+def kvq_layer_error(cache, layer):
+    """(sum (k-k^)^2, sum k^2, sum (v-v^)^2, sum v^2, quantized elements) of `layer` (synchronises)."""
+    out = kvq_error_stats()
+    _check(lib.kvq_layer_error(ctypes.c_void_p(cache), int(layer), ctypes.byref(out)))
+    return (out.k_sq_err, out.k_sq, out.v_sq_err, out.v_sq, int(out.elements))
+
+
 def kvq_set_fp8_scales(cache, layer, k_scale, v_scale) -> None:
     """Per-KV-head scales of an fp8 layer (sequences of n_kv_heads floats; host)."""
     ks = (ctypes.c_float * len(k_scale))(*[float(x) for x in k_scale])
@@ -228,6 +242,10 @@ def kvq_export_layer(cache, layer, batch):
     _check(lib.kvq_export_layer(ctypes.c_void_p(cache), int(layer), int(batch),
                                 ctypes.c_void_p(buf.ctypes.data), buf.size))
     return buf[:n]
+
+
+def kvq_refresh_lengths(cache) -> None:
+    _check(lib.kvq_refresh_lengths(ctypes.c_void_p(cache)))
 
 
 def kvq_sync(cache) -> None:

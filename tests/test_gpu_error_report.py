@@ -1,0 +1,43 @@
+"""GPU parity of the per-layer quantization error report (kvq_layer_error)
+with the oracle's: same element counts, sums within fp64 summation-order
+rounding."""
+
+import numpy as np
+import pytest
+import torch
+
+from test_gpu_parity import Pair, _inputs, kvq  # noqa: F401  (kvq is a fixture)
+
+pytestmark = pytest.mark.gpu
+
+
+def _same_report(got, want):
+    assert got[4] == want[4]
+    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-9, atol=0)
+
+
+@pytest.mark.parametrize("pair", [(2, 2), (4, 8), (8, 4), (4, 4, 1), (2, 8, 1), (8, 8, 0, 1), (16, 16)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_error_report_matches_oracle(kvq, oracle, pair, D):
+    rng = np.random.default_rng(hash((pair, D, "err")) % 2**32)
+    batch, hkv = 3, 2
+    scales = ([0.05, 0.2], [0.02, 0.5]) if len(pair) > 3 else None
+    P = Pair(kvq, oracle, pair, batch, hkv * 4, hkv, D, 256, fp8_scales=scales)
+    try:
+        K, V = _inputs(rng, 150, hkv, D)
+        P.append(K, V, [30, 64, 56])
+        _same_report(kvq.kvq_layer_error(P.cache, 0), P.ref.error())
+        for _ in range(40):   # decode-style appends cross more page boundaries
+            K, V = _inputs(rng, batch, hkv, D)
+            P.append(K, V, [1] * batch)
+        got, want = kvq.kvq_layer_error(P.cache, 0), P.ref.error()
+        _same_report(got, want)
+        if pair == (16, 16):
+            assert got == (0.0, 0.0, 0.0, 0.0, 0)
+        else:
+            # (2-bit per-token keys on outlier channels can lose more than the signal)
+            assert got[4] > 0 and got[0] > 0 and 0 < got[2] < got[3]
+        kvq.kvq_cache_reset(P.cache)
+        assert kvq.kvq_layer_error(P.cache, 0) == (0.0, 0.0, 0.0, 0.0, 0)
+    finally:
+        P.close()
