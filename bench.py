@@ -45,7 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=0,
-                    help="profile a truncated stack (first N layers); 0 = the workload's full stack")
+                    help="profile a truncated stack (N layers from --first-layer); 0 = the workload's full stack")
+    ap.add_argument("--first-layer", type=int, default=0, help="first layer of a truncated stack")
     return ap.parse_args()
 
 
@@ -414,7 +415,7 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.layers:
         import dataclasses
-        w = dataclasses.replace(w, layer_map=w.layer_map[:args.layers])
+        w = dataclasses.replace(w, layer_map=w.layer_map[args.first_layer:args.first_layer + args.layers])
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

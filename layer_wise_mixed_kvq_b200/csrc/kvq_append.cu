@@ -150,10 +150,12 @@ __device__ __forceinline__ int kmeta_slot(int d) {
 
 template <int KB, int VB, int D, bool F32IN>
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
+  pdl_enter();
   constexpr bool kBf16Layer = (KB == 16);
   const int b = blockIdx.z, h = blockIdx.y, item = blockIdx.x;
   const int H = a.n_kv_heads;
   __shared__ int s_T0;
+  __nv_bfloat16 k_new, v_new;  // one-token mode: this thread's channel of the new row
 
   int T0, n, items;
   int64_t off;
@@ -166,17 +168,21 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
     if (item == 0 && h == 0 && threadIdx.x == 0) a.len[b] = T0 + n;
   } else {
     // One token per sequence; every CTA of sequence b reads the old length,
-    // and the last one to have read it publishes the new length. The host
-    // checks capacity before launching, but a replayed CUDA graph does not run
-    // host code: a full sequence is left unchanged here and the cache's error
-    // flag is raised.
+    // and the last one to have read it publishes the new length (the
+    // acquire-release increment orders each CTA's read before the last CTA's
+    // write). The host checks capacity before launching, but a replayed CUDA
+    // graph does not run host code: a full sequence is left unchanged here and
+    // the cache's error flag is raised. The new token's row is loaded first:
+    // its address does not depend on the length.
+    if (threadIdx.x < D) {
+      k_new = load_in<F32IN>(a.K, ((int64_t)b * H + h) * D + threadIdx.x);
+      v_new = load_in<F32IN>(a.V, ((int64_t)b * H + h) * D + threadIdx.x);
+    }
     if (threadIdx.x == 0) {
-      int t0 = a.len[b];
+      const int t0 = a.len[b];
       s_T0 = t0;
-      __threadfence();
-      if (atomicAdd(&a.ctr[b], 1) == H - 1) {
+      if (atomic_add_acq_rel(&a.ctr[b], 1) == H - 1) {
         a.ctr[b] = 0;
-        __threadfence();
         if (t0 < a.max_tokens) a.len[b] = t0 + 1;
       }
     }
@@ -356,22 +362,29 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
     const int wstart = (T1 / kPageTokens) * kPageTokens;
     const int from = wstart > T0 ? wstart : T0;
     const int cnt = T1 - from;
-    for (int idx = threadIdx.x; idx < cnt * D; idx += kThreads) {
-      int i = idx / D, d = idx % D;
-      int tau = from + i;
-      int64_t row = off + (tau - T0);
-      int slot = tau % kPageTokens;
-      win[(0 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.K, (row * H + h) * D + d);
-      win[(1 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.V, (row * H + h) * D + d);
+    if (!a.plan) {
+      if (cnt == 1 && threadIdx.x < D) {  // the new token (cnt = 0: it completed a page)
+        const int slot = T0 % kPageTokens;
+        win[(0 * kPageTokens + slot) * D + threadIdx.x] = k_new;
+        win[(1 * kPageTokens + slot) * D + threadIdx.x] = v_new;
+      }
+    } else {
+      for (int idx = threadIdx.x; idx < cnt * D; idx += kThreads) {
+        int i = idx / D, d = idx % D;
+        int tau = from + i;
+        int64_t row = off + (tau - T0);
+        int slot = tau % kPageTokens;
+        win[(0 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.K, (row * H + h) * D + d);
+        win[(1 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.V, (row * H + h) * D + d);
+      }
     }
   }
 }
 
 template <int KB, int VB, int D>
 cudaError_t launch3(kvq_dtype dt, const AppendParams& p, dim3 grid, cudaStream_t s) {
-  if (dt == KVQ_F32) append_kernel<KB, VB, D, true><<<grid, kThreads, 0, s>>>(p);
-  else append_kernel<KB, VB, D, false><<<grid, kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  if (dt == KVQ_F32) return launch_pdl(append_kernel<KB, VB, D, true>, grid, dim3(kThreads), 0, s, p);
+  return launch_pdl(append_kernel<KB, VB, D, false>, grid, dim3(kThreads), 0, s, p);
 }
 
 template <int D>

@@ -119,14 +119,6 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-// Device-scope fetch-add with acquire-release ordering: releases every write
-// this thread has observed (the CTA's partial records, via the preceding
-// barrier) and acquires the other CTAs' released records.
-__device__ __forceinline__ int atomic_add_acq_rel(int* addr, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
-  return old;
-}
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
@@ -182,7 +174,9 @@ struct Cfg {
   // small pages: 3 CTAs per SM with 3-4 stages per warp; larger ones: 2 CTAs per SM
   static constexpr int MINB = PB <= 5000 ? 3 : 2;      // head-row kernel (64 accumulators per lane)
   static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;  // token-row kernel (32 accumulators per lane)
-  static constexpr int RING_BUDGET = MINB == 3 ? 14336 : 24576;   // bytes of stages per warp
+  // bytes of stages per warp: with 3 CTAs per SM, 3 x 4 warps x 14 KB; with 2, 2 x 4 x 20 KB, leaving
+  // room for the rest of a CTA's shared memory (about 20-30 KB) inside half an SM
+  static constexpr int RING_BUDGET = MINB == 3 ? 14336 : 20480;
   static constexpr int R = (RING_BUDGET / PB) < 2 ? 2 : ((RING_BUDGET / PB) > 4 ? 4 : (RING_BUDGET / PB));
   static constexpr int STAGE = (PB + 127) / 128 * 128;
   // Power-of-two factors of the subnormal unpack (see file comment).
@@ -1191,6 +1185,7 @@ __device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p
 template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
 __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_TOK : Cfg<KB, VB, D, PT, F8>::MINB)
     decode_mma_kernel(DecodeParams p) {
+  pdl_enter();
   using C = Cfg<KB, VB, D, PT, F8>;
   using State = typename std::conditional<TOK, TokState<D>, WarpState<D>>::type;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -1598,8 +1593,8 @@ cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   grid = std::min<int64_t>(grid, p.n_units);
   grid = std::min<int64_t>(grid, p.max_ctas);
   if (grid < 1) grid = 1;
-  decode_mma_kernel<KB, VB, D, TOK, PT, F8><<<(unsigned)grid, kThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decode_mma_kernel<KB, VB, D, TOK, PT, F8>, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, s,
+                    p);
 }
 
 template <int KB, int VB, int D>

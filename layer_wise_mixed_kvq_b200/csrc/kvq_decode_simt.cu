@@ -188,6 +188,7 @@ __device__ void attend_tokens(Smem<KB, VB, D>& sm, int G, int ntok, float scale_
 
 template <int KB, int VB, int D>
 __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeParams p) {
+  pdl_enter();
   constexpr int NACC = kMaxGqa * D / kThreads;
   __shared__ Smem<KB, VB, D> sm;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeParams p) {
 template <int D>
 cudaError_t launch_d(int kb, int vb, const DecodeParams& p, dim3 grid, cudaStream_t s) {
 #define KVQ_PAIR(K_, V_) \
-  if (kb == K_ && vb == V_) { decode_simt_kernel<K_, V_, D><<<grid, kThreads, 0, s>>>(p); return cudaGetLastError(); }
+  if (kb == K_ && vb == V_) return launch_pdl(decode_simt_kernel<K_, V_, D>, grid, dim3(kThreads), 0, s, p);
   KVQ_PAIR(2, 2) KVQ_PAIR(2, 4) KVQ_PAIR(2, 8)
   KVQ_PAIR(4, 2) KVQ_PAIR(4, 4) KVQ_PAIR(4, 8)
   KVQ_PAIR(8, 2) KVQ_PAIR(8, 4) KVQ_PAIR(8, 8)

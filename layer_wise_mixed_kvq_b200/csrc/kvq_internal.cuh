@@ -17,6 +17,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <utility>
 #include <string>
 #include <vector>
 
@@ -98,6 +99,48 @@ struct DecodeParams {
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
 };
+
+// Programmatic dependent launch. Every kernel of the library starts with
+// pdl_enter(): it waits for its stream predecessor to complete (with that
+// grid's memory visible) before its first global memory access, then lets its
+// own successor begin launching. On an ordinary stream the kernels are launched
+// with programmatic stream serialization, so a successor's launch and CTA
+// placement overlap this kernel's tail; stream order is unchanged. While the
+// stream is being captured into a CUDA graph they are launched plainly
+// (measured on B200: programmatic edges inside the captured decode step made
+// replays slower), and the wait is then a no-op.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Device-scope fetch-add with acquire-release ordering: releases every memory
+// access this thread has performed or observed (through a preceding barrier)
+// and acquires those released by the other participants.
+__device__ __forceinline__ int atomic_add_acq_rel(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &capture);
+  if (e != cudaSuccess) return e;
+  cfg.attrs = attr;
+  cfg.numAttrs = capture == cudaStreamCaptureStatusNone ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launchers (defined per kernel file); return the CUDA launch error.
 // The key mode travels in the parameter blocks (AppendParams/DecodeParams::key_mode).
