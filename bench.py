@@ -171,6 +171,19 @@ def cpu_baseline(w, seconds):
             "decode_layers_per_s": samples / t_attn}
 
 
+def workload_config(w, equiv_bits, world):
+    """The `config` object both arms print (the GPU arm's workload, whatever the arm samples)."""
+    return {"workload": w.name, "layers": w.n_layers, "layer_map_equiv_bits": equiv_bits, "batch": w.batch,
+            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "context": int(synth.context_lengths(w).max()), "parallelism": f"replicas x{world}",
+            "l2": "cache larger than L2 (no flush)"}
+
+
+def oracle_equiv_bits(w):
+    import oracle
+    return oracle.equiv_bits([p[:2] for p in w.layer_map])
+
+
 def run_reference(args, w):
     rank, world, _ = replicas.world()
     if rank != 0:
@@ -185,8 +198,7 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_layer_s * w.n_layers * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": 1, "context": w.context, "layers": w.n_layers,
-                   "note": "CPU oracle on a bounded sample (single sequence per layer)"},
+        "config": workload_config(w, oracle_equiv_bits(w), 1),
         "cpu_baseline": {k: cb[k] for k in ("kind", "cores", "sample")} | {"value": value, "unit": "GB/s"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "bytes_per_layer": bytes_per_layer,
@@ -377,12 +389,10 @@ def run_gpu(args, w):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4/int2/int8 codes + bf16, fp32 accumulate",
+        "dtype": "f32",
+        "operands": "f16 tensor-core operands (integer codes and e4m3 as exact f16, q and p as hi+lo f16 pairs)",
         "data": "synthetic",
-        "config": {"workload": w.name, "layers": NL, "layer_map_equiv_bits": kvq.kvq_equiv_bits(list(w.layer_map)),
-                   "batch": B, "n_q_heads": Hq, "n_kv_heads": Hkv, "head_dim": D,
-                   "context": int(lens.max()), "parallelism": f"replicas x{world}",
-                   "l2": "cache larger than L2 (no flush)"},
+        "config": workload_config(w, kvq.kvq_equiv_bits(list(w.layer_map)), world),
         "pct_of_peak": value / peak,
         "decode_steps_per_s": 1e3 / ms_per_step,
         "tokens_per_s": B * world * 1e3 / ms_per_step,
