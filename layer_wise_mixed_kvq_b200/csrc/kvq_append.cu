@@ -269,72 +269,72 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
           store_block<8, D>(page + code_block_bytes(8, D), true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
         }
       } else {
-      const bool per_token_keys = a.key_mode != 0;
-      const int nk = per_token_keys ? kPageTokens : D;  // key scale/zero pairs
-      uint8_t* vblk = page + code_block_bytes(KB, D);
-      __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
-      __half* kzero = kscale + nk;
-      __half* vscale = kzero + nk;
-      __half* vzero = vscale + kPageTokens;
-      // one warp per token over the head dimension: row r of xs (0 keys, 1 values)
-      auto quantize_tokens = [&](int r, int qmax, __half* sdst, __half* zdst) {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        for (int t = warp; t < kPageTokens; t += kThreads / 32) {
-          float mn = xs[r][t][lane], mx = mn;
-#pragma unroll
-          for (int k = 1; k < D / 32; ++k) {
-            float x = xs[r][t][lane + 32 * k];
+        const bool per_token_keys = a.key_mode != 0;
+        const int nk = per_token_keys ? kPageTokens : D;  // key scale/zero pairs
+        uint8_t* vblk = page + code_block_bytes(KB, D);
+        __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
+        __half* kzero = kscale + nk;
+        __half* vscale = kzero + nk;
+        __half* vzero = vscale + kPageTokens;
+        // one warp per token over the head dimension: row r of xs (0 keys, 1 values)
+        auto quantize_tokens = [&](int r, int qmax, __half* sdst, __half* zdst) {
+          const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+          for (int t = warp; t < kPageTokens; t += kThreads / 32) {
+            float mn = xs[r][t][lane], mx = mn;
+  #pragma unroll
+            for (int k = 1; k < D / 32; ++k) {
+              float x = xs[r][t][lane + 32 * k];
+              mn = fminf(mn, x);
+              mx = fmaxf(mx, x);
+            }
+  #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            QParams q = make_qparams(mn, mx, qmax);
+            const double s = (double)__half2float(q.s_h), z = (double)q.z;
+  #pragma unroll
+            for (int k = 0; k < D / 32; ++k) {
+              const float x = xs[r][t][lane + 32 * k];
+              const uint32_t c = quant_code(x, q, qmax);
+              cs[r][t][lane + 32 * k] = (uint8_t)c;
+              add_err(r, x, (double)c * s + z);
+            }
+            if (lane == 0) {
+              sdst[t] = q.s_h;
+              zdst[t] = q.z_h;
+            }
+          }
+        };
+        if (per_token_keys) quantize_tokens(0, (1 << KB) - 1, kscale, kzero);
+        // keys (per-channel mode): one thread per channel, over the group's 32 tokens
+        for (int d = threadIdx.x; d < (per_token_keys ? 0 : D); d += kThreads) {
+          constexpr int qmax = (1 << KB) - 1;
+          float mn = xs[0][0][d], mx = mn;
+  #pragma unroll 8
+          for (int t = 1; t < kPageTokens; ++t) {
+            float x = xs[0][t][d];
             mn = fminf(mn, x);
             mx = fmaxf(mx, x);
           }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          }
           QParams q = make_qparams(mn, mx, qmax);
           const double s = (double)__half2float(q.s_h), z = (double)q.z;
-#pragma unroll
-          for (int k = 0; k < D / 32; ++k) {
-            const float x = xs[r][t][lane + 32 * k];
-            const uint32_t c = quant_code(x, q, qmax);
-            cs[r][t][lane + 32 * k] = (uint8_t)c;
-            add_err(r, x, (double)c * s + z);
+  #pragma unroll 8
+          for (int t = 0; t < kPageTokens; ++t) {
+            const uint32_t c = quant_code(xs[0][t][d], q, qmax);
+            cs[0][t][d] = (uint8_t)c;
+            add_err(0, xs[0][t][d], (double)c * s + z);
           }
-          if (lane == 0) {
-            sdst[t] = q.s_h;
-            zdst[t] = q.z_h;
-          }
+          int slot = kmeta_slot<D>(d);
+          kscale[slot] = q.s_h;
+          kzero[slot] = q.z_h;
         }
-      };
-      if (per_token_keys) quantize_tokens(0, (1 << KB) - 1, kscale, kzero);
-      // keys (per-channel mode): one thread per channel, over the group's 32 tokens
-      for (int d = threadIdx.x; d < (per_token_keys ? 0 : D); d += kThreads) {
-        constexpr int qmax = (1 << KB) - 1;
-        float mn = xs[0][0][d], mx = mn;
-#pragma unroll 8
-        for (int t = 1; t < kPageTokens; ++t) {
-          float x = xs[0][t][d];
-          mn = fminf(mn, x);
-          mx = fmaxf(mx, x);
-        }
-        QParams q = make_qparams(mn, mx, qmax);
-        const double s = (double)__half2float(q.s_h), z = (double)q.z;
-#pragma unroll 8
-        for (int t = 0; t < kPageTokens; ++t) {
-          const uint32_t c = quant_code(xs[0][t][d], q, qmax);
-          cs[0][t][d] = (uint8_t)c;
-          add_err(0, xs[0][t][d], (double)c * s + z);
-        }
-        int slot = kmeta_slot<D>(d);
-        kscale[slot] = q.s_h;
-        kzero[slot] = q.z_h;
-      }
-      // values: one warp per token, over the head dimension
-      quantize_tokens(1, (1 << VB) - 1, vscale, vzero);
-      __syncthreads();
-      store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
-      store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
+        // values: one warp per token, over the head dimension
+        quantize_tokens(1, (1 << VB) - 1, vscale, vzero);
+        __syncthreads();
+        store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
+        store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
       }
       // this flush's error sums: warp shuffles, then one fp64 atomic per sum
       __shared__ double red[kThreads / 32][4];
