@@ -171,12 +171,13 @@ struct Cfg {
   static constexpr bool kBf16 = (KB == 16);
   static constexpr int KS = D / 16;                       // 16-channel tiles
   static constexpr int PB = (int)page_bytes_of(KB, VB, D, PT ? 1 : 0, F8 ? 1 : 0);
-  // small pages: 3 CTAs per SM with 3-4 stages per warp; larger ones: 2 CTAs per SM
-  static constexpr int MINB = PB <= 5000 ? 3 : 2;      // head-row kernel (64 accumulators per lane)
-  static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;  // token-row kernel (32 accumulators per lane)
+  // token rows: 3 CTAs per SM for small pages (3-4 stages per warp), 2 for larger ones; head rows
+  // (64 accumulators per lane) always 2, so they get the registers they need without spilling
+  static constexpr int MINB = 2;
+  static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;
   // bytes of stages per warp: with 3 CTAs per SM, 3 x 4 warps x 14 KB; with 2, 2 x 4 x 20 KB, leaving
   // room for the rest of a CTA's shared memory (about 20-30 KB) inside half an SM
-  static constexpr int RING_BUDGET = MINB == 3 ? 14336 : 20480;
+  static constexpr int RING_BUDGET = MINB_TOK == 3 ? 14336 : 20480;
   static constexpr int R = (RING_BUDGET / PB) < 2 ? 2 : ((RING_BUDGET / PB) > 4 ? 4 : (RING_BUDGET / PB));
   static constexpr int STAGE = (PB + 127) / 128 * 128;
   // Power-of-two factors of the subnormal unpack (see file comment).

@@ -301,3 +301,25 @@ def test_simt_kernel_matches_oracle(kvq, oracle, tmp_path):
     env = dict(os.environ, KVQ_DECODE_KERNEL="simt")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_max_batch_and_gqa(kvq, oracle, mode):
+    """The largest batch (1024 sequences) at the largest GQA ratio (8 query heads
+    per KV head, head-row formulation) with ragged short contexts: exercises the
+    unit scan over many sequences, many small segments per CTA and empty ones."""
+    rng = np.random.default_rng(1024 + mode)
+    batch, hkv, G, D = 1024, 1, 8, 64
+    lens = [int(x) for x in rng.integers(0, 70, size=batch)]
+    P = Pair(kvq, oracle, (4, 2, mode), batch, hkv * G, hkv, D, 80)
+    try:
+        K, V = _inputs(rng, sum(lens), hkv, D)
+        P.append(K, V, lens)
+        K1, V1 = _inputs(rng, batch, hkv, D)
+        P.append(K1, V1, [1] * batch)
+        P.check_pages()
+        seqs = [0, 1, 511, 777, 1023] + [i for i, n in enumerate(lens) if n == 0][:3]
+        got, ref = P.attend(_q(rng, batch, hkv * G, D), seqs=seqs)
+        _check_attention(got[seqs], ref[seqs], f"batch 1024 mode {mode}")
+    finally:
+        P.close()
