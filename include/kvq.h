@@ -244,6 +244,24 @@ kvq_status kvq_set_fp8_scales(kvq_cache* cache, int layer, const float* k_scale,
  * it changes only the rounding order of the result. */
 kvq_status kvq_set_split_pages(kvq_cache* cache, int pages_per_split);
 
+/* Work split of kvq_decode_attn's tensor-core kernel when the query group has
+ * at most 4 heads (n_q_heads / n_kv_heads <= 4): either each warp attends whole
+ * (sequence, KV head) segments on its own and writes their outputs (no split
+ * records, no merge), or the CTAs of a persistent grid share each segment's
+ * pages. The first wins when sequences are short and segments many (batch 64 x
+ * 160 tokens: 10 vs 19 us per layer on B200), the second otherwise.
+ *   -1 (default): automatic -- the split a cost model fitted on B200 predicts
+ *       faster (warp split about 5 + 1.0 us per page of the longest sequence;
+ *       shared split about 11.5 + 0.01 us per segment + 0.15 us per page per SM);
+ *    0: always the shared split;
+ *    n > 0: the warp split whenever no sequence holds more than n full pages.
+ * The warp split also needs every segment to fit the resident warps, else the
+ * shared split runs. The choice is taken at launch from the host's view of the
+ * lengths, so a CUDA graph keeps the split it was captured with (both are
+ * correct at any length). It changes only the rounding order of the result.
+ * Errors: KVQ_EINVAL (null cache, value < -1). */
+kvq_status kvq_set_decode_mode(kvq_cache* cache, int max_pages_per_warp);
+
 /* Tokens currently held by sequence `seq` of `layer` (host mirror), -1 if invalid. */
 int64_t kvq_seq_len(const kvq_cache* cache, int layer, int seq);
 

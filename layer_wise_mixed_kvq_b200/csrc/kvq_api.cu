@@ -334,6 +334,13 @@ kvq_status kvq_set_split_pages(kvq_cache* c, int pages_per_split) {
   return KVQ_OK;
 }
 
+kvq_status kvq_set_decode_mode(kvq_cache* c, int max_pages_per_warp) {
+  if (!c) return fail(KVQ_EINVAL, "cache is null");
+  if (max_pages_per_warp < -1) return fail(KVQ_EINVAL, "max_pages_per_warp must be >= -1");
+  c->warp_pages = max_pages_per_warp;
+  return KVQ_OK;
+}
+
 kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq_dtype dtype,
                       const int32_t* n_new, int batch, void* stream) {
   kvq_status st = check_cache(c, layer);
@@ -460,6 +467,23 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.key_mode = L.km;
   p.fmt = L.fmt;
   p.fp8_scales = L.fp8_scales;
+  {
+    // One warp per (sequence, KV head) segment, or CTAs sharing each segment's pages.
+    // Automatic: the split a cost model predicts faster, fitted to both kernels' times
+    // on B200 (K4V2..K8V8 pages, batch 16 and 64, 5 to 128 pages per sequence): the
+    // warp split takes about 5 + 1.0 us per page of the longest sequence, the shared
+    // split about 11.5 + 0.01 us per segment + 0.15 us per page per SM.
+    bool warp = false;
+    if (p.gqa <= 4 && c->warp_pages > 0) {
+      warp = max_p <= c->warp_pages;
+    } else if (p.gqa <= 4 && c->warp_pages < 0) {
+      const double segs = (double)batch * c->n_kv_heads;
+      const double t_warp = 5.0 + 1.0 * (double)max_p;
+      const double t_shared = 11.5 + 0.01 * segs + 0.15 * (double)total_pages / c->sm_count;
+      warp = t_warp < t_shared;
+    }
+    p.warp_split = warp ? 1 : 0;
+  }
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

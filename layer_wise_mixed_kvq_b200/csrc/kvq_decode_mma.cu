@@ -1572,9 +1572,246 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
   }
 }
 
+// ---------------------------------------------------------- warp-segment kernel --
+// Short sequences (token rows, G <= 4): warp w of CTA c attends segments
+// s = c * kWarps + w, then s + gridDim.x * kWarps, ... on its own -- query rows
+// by bulk copy into the warp's slot, pages through the warp's ring, then the
+// window -- and writes the segment's output directly. No CTA barrier, split
+// record or merge: at a few pages per segment those fixed costs, not the page
+// bytes, are what a shared split spends its time on.
+template <int KB, int VB, int D, bool PT, bool F8>
+struct WarpCfg {
+  using C = Cfg<KB, VB, D, PT, F8>;
+  static constexpr int MBAR_OFF = C::RING;
+  static constexpr int MBAR_BYTES = ((kWarps * (C::R + 1)) * 8 + 127) / 128 * 128;  // ring + one query barrier
+  static constexpr int WSCR_OFF = MBAR_OFF + MBAR_BYTES;
+  static constexpr int QBUF_OFF = WSCR_OFF + kWarps * C::WSCR_STRIDE;
+  static constexpr int QSLOT = 4 * D * 2;                                            // [4][D] bf16 per warp
+  static constexpr int SMEM = QBUF_OFF + kWarps * QSLOT;
+};
+
+template <int KB, int VB, int D, bool PT, bool F8>
+__global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
+    decode_warp_kernel(DecodeParams p) {
+  pdl_enter();
+  using C = Cfg<KB, VB, D, PT, F8>;
+  using WC = WarpCfg<KB, VB, D, PT, F8>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int H = p.n_kv_heads, G = p.gqa;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int qh = g >> 1;  // column head of this lane
+  const float partf = (float)(g & 1);
+  uint8_t* ring = smem + warp * C::R * C::STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WC::MBAR_OFF) + warp * (C::R + 1);
+  uint64_t* qbar = bars + C::R;
+  float* wscr = reinterpret_cast<float*>(smem + WC::WSCR_OFF + warp * C::WSCR_STRIDE);
+  __nv_bfloat16* qslot = reinterpret_cast<__nv_bfloat16*>(smem + WC::QBUF_OFF + warp * WC::QSLOT);
+  if (lane == 0) {
+    for (int r = 0; r <= C::R; ++r) mbar_init(&bars[r], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  const int S = p.batch * H;
+  const int stride = (int)gridDim.x * kWarps;
+  const uint32_t qbytes = (uint32_t)(G * D * 2);
+  const uint64_t pol = l2_evict_first_policy();
+  bool ok = true;
+  int issued = 0, consumed = 0, nq = 0;
+  for (int s = blockIdx.x * kWarps + warp; s < S && ok; s += stride, ++nq) {
+    const int b = s / H, h = s % H;
+    const int T = p.len[b];
+    const int P = T / kPageTokens, W = T % kPageTokens;
+    const uint8_t* base = p.pages + ((int64_t)s * p.max_pages) * p.page_bytes;
+    const __nv_bfloat16* win = p.window + ((int64_t)s * 2) * kPageTokens * D;
+    int next = 0;  // next page of this segment to copy
+    if (lane == 0) {
+      fence_proxy_async();  // the slot's previous rows were read through the generic proxy
+      mbar_expect_tx(qbar, qbytes);
+      bulk_load(qslot, p.Q + (int64_t)s * G * D, qbytes, qbar);
+      for (; next < P && next < C::R; ++next) {
+        const int stage = (issued + next) % C::R;
+        mbar_expect_tx(&bars[stage], C::PB);
+        bulk_load_once(ring + stage * C::STAGE, base + (int64_t)next * p.page_bytes, C::PB, &bars[stage], pol);
+      }
+      if (W > 0) {
+        prefetch_l2(win, (uint32_t)(W * D * 2));
+        prefetch_l2(win + kPageTokens * D, (uint32_t)(W * D * 2));
+      }
+    }
+    next = __shfl_sync(0xffffffffu, next, 0);
+    issued += next;
+    {
+      const bool got = mbar_wait(qbar, (uint32_t)(nq & 1));
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+    }
+    const bool qvalid = qh < G;
+    const __nv_bfloat16* qrow = qslot + (qvalid ? qh : 0) * D;
+    float qf[D / 4];
+    uint32_t qb[D / 8];
+    uint32_t qzb[D / 8];
+    float qsum = 0.f;
+    auto load_qbp = [&]() {
+#pragma unroll
+      for (int dt = 0; dt < C::KS; ++dt) {
+        const uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
+        const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
+        const bool keep = qvalid && (g & 1) == 0;  // q is exact in bf16: its low part is zero
+        qb[2 * dt] = keep ? lo : 0u;
+        qb[2 * dt + 1] = keep ? hi : 0u;
+      }
+    };
+    if constexpr (C::kBf16) {
+      load_qbp();
+    } else {
+#pragma unroll
+      for (int dt = 0; dt < C::KS; ++dt) {
+        uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
+        uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
+        if (!qvalid) lo = hi = 0u;
+        const float2 l2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&lo));
+        const float2 h2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&hi));
+        qf[dt * 4 + 0] = l2.x * p.scale_log2;
+        qf[dt * 4 + 1] = l2.y * p.scale_log2;
+        qf[dt * 4 + 2] = h2.x * p.scale_log2;
+        qf[dt * 4 + 3] = h2.y * p.scale_log2;
+      }
+      const float qlo = F8 ? p.fp8_scales[h] : 1.f;
+      const float qhi = PT ? 1.f / C::tauK : qlo;
+#pragma unroll
+      for (int dt = 0; dt < C::KS; ++dt) {
+        qzb[2 * dt] = part_f16(qf[dt * 4 + 0] * qlo, qf[dt * 4 + 1] * qlo, partf);
+        qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, partf);
+      }
+      if constexpr (PT) {
+        float qs = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 4; ++i) qs += qf[i];
+        qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+        qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+        qsum = __shfl_sync(0xffffffffu, qs, 8 * t);
+      }
+    }
+
+    TokState<D> st;
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st.o[j][k] = 0.f;
+    st.m = -INFINITY;
+    st.l = 0.f;
+    st.vz = 0.f;
+    bool converted = C::kBf16;
+    auto to_true_units = [&]() {
+      if constexpr (F8) {
+        const float vsc = p.fp8_scales[H + h] * kF8Unit;
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) st.o[j][k] *= vsc;
+      } else if constexpr (!C::kBf16) {
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+          st.o[j][0] *= kTwo24;
+          st.o[j][1] *= kTwo24;
+          st.o[j][2] *= kTwo24 / C::sigmaV;
+          st.o[j][3] *= kTwo24 / C::sigmaV;
+        }
+      }
+      converted = true;
+    };
+
+    for (int k = 0; k < P; ++k) {
+      const int stage = consumed % C::R;
+      const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
+      if (!__all_sync(0xffffffffu, arrived)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* page = ring + stage * C::STAGE;
+      if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
+      else if constexpr (F8) attend_f8page_tok<D>(page, st, qzb, wscr, partf, lane);
+      else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
+      else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
+      ++consumed;
+      __syncwarp();
+      if (next < P) {
+        if (lane == 0) {
+          fence_proxy_async();
+          mbar_expect_tx(&bars[stage], C::PB);
+          bulk_load_once(ring + stage * C::STAGE, base + (int64_t)next * p.page_bytes, C::PB, &bars[stage], pol);
+        }
+        ++next;
+        ++issued;
+      }
+    }
+    if (!ok) break;
+    if (W > 0) {
+      if constexpr (!C::kBf16) {
+        to_true_units();
+        load_qbp();
+      }
+      attend_window_tok<D>(win, W, st, qb, wscr, partf, p.scale_log2, lane);
+    }
+    if (!converted) to_true_units();
+
+    // head t's sum over the warp's tokens, then the output rows of this segment
+    float l = st.l, vz = st.vz;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, o);
+      vz += __shfl_xor_sync(0xffffffffu, vz, o);
+    }
+    if (t < G) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* dst = p.out + ((int64_t)s * G + t) * D;
+#pragma unroll
+      for (int j = 0; j < D / 16; ++j) {
+        dst[16 * j + g] = (st.o[j][0] + st.o[j][1] + vz) * inv;
+        dst[16 * j + 8 + g] = (st.o[j][2] + st.o[j][3] + vz) * inv;
+      }
+    }
+    __syncwarp();  // every lane has read the query slot before the next segment's copy lands
+  }
+
+  if (!ok) {
+    // a copy never completed: report it, then let the copies in flight land
+    // (each wait bounded again) before this CTA's shared memory goes away
+    if (lane == 0 && p.err) atomicExch(p.err, 1);
+    for (int i = consumed; i < issued; ++i) mbar_wait(&bars[i % C::R], (uint32_t)((i / C::R) & 1));
+    mbar_wait(qbar, (uint32_t)(nq & 1));
+  }
+}
+
 template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
 cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   using C = Cfg<KB, VB, D, PT, F8>;
+  if constexpr (TOK) {
+    // short sequences: one warp per segment when every segment fits in one resident wave
+    if (p.warp_split) {
+      using WC = WarpCfg<KB, VB, D, PT, F8>;
+      static bool configured = false;
+      static int occ_w = 0;
+      if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_w, decode_warp_kernel<KB, VB, D, PT, F8>, kThreads,
+                                                          WC::SMEM);
+        if (e != cudaSuccess) return e;
+        configured = true;
+      }
+      const int64_t segs = (int64_t)p.batch * p.n_kv_heads;
+      const int64_t ctas = (segs + kWarps - 1) / kWarps;
+      if (ctas >= 1 && ctas <= (int64_t)occ_w * p.sm_count)
+        return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8>, dim3((unsigned)ctas), dim3(kThreads),
+                          (size_t)WC::SMEM, s, p);
+    }
+  }
   static int configured_smem = 0;
   static int occ_smem = -1, occ_blocks = 0;
   const int smem = C::smem_bytes(TOK, p.gqa, p.batch);

@@ -98,6 +98,8 @@ struct DecodeParams {
   const float* fp8_scales;  // fmt 1: [2][n_kv_heads] key then value scales
   float scale_log2;      // log2(e) / sqrt(head_dim)
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
+  int warp_split;        // tensor-core kernel, G <= 4: one warp per segment (if the segments fit the
+                         // resident warps) instead of CTAs sharing each segment's pages
 };
 
 // Programmatic dependent launch. Every kernel of the library starts with
@@ -181,5 +183,6 @@ struct kvq_cache {
   size_t pool_bytes = 0;
   bool owns_pool = false;
   int split_pages = 0;
+  int warp_pages = -1;               // kvq_set_decode_mode: -1 automatic, 0 never, n > 0 up to n pages
   int64_t launches = 0;
 };

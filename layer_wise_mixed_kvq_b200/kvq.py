@@ -25,6 +25,7 @@ EXPORTS = (
     "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
     "kvq_export_bytes", "kvq_export_layer", "kvq_sync", "kvq_launch_count", "kvq_last_error",
     "kvq_status_string", "kvq_set_fp8_scales", "kvq_layer_error", "kvq_refresh_lengths",
+    "kvq_set_decode_mode",
 )
 
 
@@ -70,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "kvq_decode_attn_noalloc": (c.c_int, [kvq_pair, c.c_int, c.c_int, c.c_int, P, c.c_int64, P, P, c.c_int64, P,
                                               c.c_int, P, P]),
         "kvq_set_split_pages": (c.c_int, [P, c.c_int]),
+        "kvq_set_decode_mode": (c.c_int, [P, c.c_int]),
         "kvq_seq_len": (c.c_int64, [P, c.c_int, c.c_int]),
         "kvq_bytes": (c.c_int64, [P, c.c_int, c.c_int, c.c_int]),
         "kvq_export_bytes": (c.c_int64, [P, c.c_int, c.c_int]),
@@ -218,6 +220,10 @@ def kvq_set_fp8_scales(cache, layer, k_scale, v_scale) -> None:
 
 def kvq_set_split_pages(cache, pages_per_split: int) -> None:
     _check(lib.kvq_set_split_pages(ctypes.c_void_p(cache), int(pages_per_split)))
+
+
+def kvq_set_decode_mode(cache, max_pages_per_warp: int) -> None:
+    _check(lib.kvq_set_decode_mode(ctypes.c_void_p(cache), int(max_pages_per_warp)))
 
 
 def kvq_seq_len(cache, layer, seq) -> int:
