@@ -186,6 +186,27 @@ kvq_status kvq_append(kvq_cache* cache, int layer, const void* K, const void* V,
 kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch, float* out,
                            void* stream);
 
+/* One decode step of `layer`: append one new token to every sequence b < batch,
+ * then attend over all tokens including it -- the same result as
+ * kvq_append(n_new = 1 for each b) followed by kvq_decode_attn, with the same
+ * pages, window, lengths and error report afterwards.
+ *   K, V: device bf16 [batch, n_kv_heads, head_dim], the new token of each
+ *         sequence, 16-byte aligned.
+ *   Q, out: as for kvq_decode_attn.
+ * Where kvq_decode_attn would take the one-warp-per-segment split (short
+ * sequences, at most 4 query heads per KV head; see kvq_set_decode_mode) this is
+ * ONE kernel launch: the warp that attends segment (b, h) first writes its new
+ * token into the window or, when the token completes a 32-token group,
+ * quantizes and packs that group into the next page and attends it from there.
+ * Otherwise it runs the two kernels. The KVTuner pages warn that per-layer
+ * dispatch overhead can erase the savings of a small KV cache; at short
+ * sequences the append kernel costs about as much as the attention itself.
+ * A CUDA graph keeps the form it was captured with; inside a graph the one-
+ * token capacity guard of kvq_append applies (see kvq_refresh_lengths).
+ * Errors: KVQ_EINVAL, KVQ_ECAPACITY (some sequence is full; nothing changes). */
+kvq_status kvq_decode_step(kvq_cache* cache, int layer, const void* K, const void* V, const void* Q, int batch,
+                           float* out, void* stream);
+
 /* kvq_decode_attn for callers that cannot allocate device memory. The KVTuner
  * pages have no counterpart of this call; it exists for programs whose device
  * memory belongs to someone else (a serving engine that reserves all of HBM for

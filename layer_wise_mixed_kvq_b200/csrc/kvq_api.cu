@@ -111,12 +111,16 @@ void set_last_error(const std::string& msg) { g_last_error = msg; }
 
 // The tensor-core kernel serves every pair; KVQ_DECODE_KERNEL=simt selects the
 // CUDA-core kernel instead (a second, independent implementation for checks).
-cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s) {
+bool decode_uses_simt() {
   static const bool simt = [] {
     const char* e = std::getenv("KVQ_DECODE_KERNEL");
     return e && std::string(e) == "simt";
   }();
-  return simt ? launch_decode_simt(kb, vb, D, p, grid, s) : launch_decode_mma(kb, vb, D, p, s);
+  return simt;
+}
+
+cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  return decode_uses_simt() ? launch_decode_simt(kb, vb, D, p, grid, s) : launch_decode_mma(kb, vb, D, p, s);
 }
 
 int seg_overhead_units() {
@@ -415,6 +419,20 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
   return KVQ_OK;
 }
 
+// One warp per (sequence, KV head) segment, or CTAs sharing each segment's pages.
+// Automatic: the split a cost model predicts faster, fitted to both kernels' times
+// on B200 (K4V2..K8V8 pages, batch 16 and 64, 5 to 128 pages per sequence): the
+// warp split takes about 5 + 1.0 us per page of the longest sequence, the shared
+// split about 11.5 + 0.01 us per segment + 0.15 us per page per SM.
+static bool choose_warp_split(const kvq_cache* c, int gqa, int batch, int64_t max_p, int64_t total_pages) {
+  if (gqa > 4 || c->warp_pages == 0) return false;
+  if (c->warp_pages > 0) return max_p <= c->warp_pages;
+  const double segs = (double)batch * c->n_kv_heads;
+  const double t_warp = 5.0 + 1.0 * (double)max_p;
+  const double t_shared = 11.5 + 0.01 * segs + 0.15 * (double)total_pages / c->sm_count;
+  return t_warp < t_shared;
+}
+
 kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, float* out, void* stream) {
   kvq_status st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
@@ -467,26 +485,73 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.key_mode = L.km;
   p.fmt = L.fmt;
   p.fp8_scales = L.fp8_scales;
-  {
-    // One warp per (sequence, KV head) segment, or CTAs sharing each segment's pages.
-    // Automatic: the split a cost model predicts faster, fitted to both kernels' times
-    // on B200 (K4V2..K8V8 pages, batch 16 and 64, 5 to 128 pages per sequence): the
-    // warp split takes about 5 + 1.0 us per page of the longest sequence, the shared
-    // split about 11.5 + 0.01 us per segment + 0.15 us per page per SM.
-    bool warp = false;
-    if (p.gqa <= 4 && c->warp_pages > 0) {
-      warp = max_p <= c->warp_pages;
-    } else if (p.gqa <= 4 && c->warp_pages < 0) {
-      const double segs = (double)batch * c->n_kv_heads;
-      const double t_warp = 5.0 + 1.0 * (double)max_p;
-      const double t_shared = 11.5 + 0.01 * segs + 0.15 * (double)total_pages / c->sm_count;
-      warp = t_warp < t_shared;
-    }
-    p.warp_split = warp ? 1 : 0;
-  }
+  p.warp_split = choose_warp_split(c, p.gqa, batch, max_p, total_pages) ? 1 : 0;
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  c->launches += 1;
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_step(kvq_cache* c, int layer, const void* K, const void* V, const void* Q, int batch,
+                           float* out, void* stream) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (batch <= 0 || batch > c->max_batch) return fail(KVQ_EINVAL, "batch must be in [1, max_batch]");
+  if (!K || !V || !Q || !out) return fail(KVQ_EINVAL, "K, V, Q or out is null");
+  if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out))
+    return fail(KVQ_EINVAL, "K, V, Q and out must be 16-byte aligned");
+  kvq::LayerState& L = c->layers[layer];
+  int64_t total_pages = 0, max_p = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (L.host_len[b] + 1 > c->max_tokens)
+      return fail(KVQ_ECAPACITY, "append would exceed max_tokens for sequence " + std::to_string(b));
+    const int64_t P = (L.host_len[b] + 1) / kvq::kPageTokens;
+    total_pages += P;
+    max_p = std::max(max_p, P);
+  }
+  total_pages *= c->n_kv_heads;
+  const int gqa = c->n_q_heads / c->n_kv_heads;
+  auto two_launches = [&]() -> kvq_status {
+    std::vector<int32_t> ones((size_t)batch, 1);
+    kvq_status r = kvq_append(c, layer, K, V, KVQ_BF16, ones.data(), batch, stream);
+    return r != KVQ_OK ? r : kvq_decode_attn(c, layer, Q, batch, out, stream);
+  };
+  if (kvq::decode_uses_simt() || !choose_warp_split(c, gqa, batch, max_p, total_pages)) return two_launches();
+
+  kvq::DecodeParams p{};
+  p.pages = L.pages;
+  p.window = L.window;
+  p.len = L.len;
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.out = out;
+  p.page_bytes = L.page_bytes;
+  p.max_pages = (int)c->max_pages;
+  p.n_kv_heads = c->n_kv_heads;
+  p.gqa = gqa;
+  p.batch = batch;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
+  p.err = c->err;
+  p.sm_count = c->sm_count;
+  p.key_mode = L.km;
+  p.fmt = L.fmt;
+  p.fp8_scales = L.fp8_scales;
+  p.warp_split = 1;
+  p.step_pages = L.pages;
+  p.step_window = L.window;
+  p.step_len = L.len;
+  p.append_ctr = c->append_ctr;
+  p.k_new = static_cast<const __nv_bfloat16*>(K);
+  p.v_new = static_cast<const __nv_bfloat16*>(V);
+  p.err_stats = L.err_stats;
+  p.max_tokens = (int)std::min<int64_t>(c->max_tokens, INT32_MAX);
+  cudaError_t e = kvq::launch_decode_step(L.kb, L.vb, c->head_dim, p, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    return two_launches();
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode step kernel launch");
+  for (int b = 0; b < batch; ++b) L.host_len[b] += 1;
   c->launches += 1;
   return KVQ_OK;
 }

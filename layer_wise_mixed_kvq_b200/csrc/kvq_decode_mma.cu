@@ -36,6 +36,7 @@
 #include <cuda_fp8.h>
 
 #include "kvq_internal.cuh"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 namespace {
@@ -1572,6 +1573,189 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
   }
 }
 
+// ------------------------------------------------------------ fused append --
+// Warp-level flush of one completed 32-token group (the window's 31 tokens and
+// the new token) into `page`, bit-identical to the append kernel's CTA-wide
+// flush: the same quantizer and packing (kvq_quant.cuh), only the work split
+// differs. `scr` is this warp's ring (free at a segment's start) and holds the
+// codes as bytes, [2][32][D] (bf16 layers: the rows themselves), before they
+// are packed in fragment order.
+template <int BITS, int D, typename Get>
+__device__ __forceinline__ void pack_block_warp(uint8_t* blk, bool is_value, int lane, Get vals) {
+  constexpr int kPerLane = (int)(code_block_bytes(BITS, D) / 16) / 32;  // 16-byte vectors per lane
+#pragma unroll 1
+  for (int vi = 0; vi < kPerLane; ++vi) {
+    uint4 q;
+    q.x = lane_word<BITS>(lane, 4 * vi + 0, is_value, vals);
+    q.y = lane_word<BITS>(lane, 4 * vi + 1, is_value, vals);
+    q.z = lane_word<BITS>(lane, 4 * vi + 2, is_value, vals);
+    q.w = lane_word<BITS>(lane, 4 * vi + 3, is_value, vals);
+    reinterpret_cast<uint4*>(blk)[vi * 32 + lane] = q;
+  }
+}
+
+template <int KB, int VB, int D, bool PT, bool F8>
+__device__ __noinline__ void warp_flush(uint8_t* page, const __nv_bfloat16* win, const __nv_bfloat16* kn,
+                                        const __nv_bfloat16* vn, uint8_t* scr, float ksc, float vsc,
+                                        double* err_stats, int lane) {
+  // row of token tok (0..31) of keys (r = 0) or values (r = 1)
+  auto row = [&](int r, int tok) -> const __nv_bfloat16* {
+    return tok < kPageTokens - 1 ? win + (r * kPageTokens + tok) * D : (r ? vn : kn);
+  };
+  if constexpr (KB == 16) {
+    // bf16 layer: stage the 32 rows of keys and values, then pack their bit patterns
+    uint16_t* sb = reinterpret_cast<uint16_t*>(scr);  // [2][32][D]
+#pragma unroll 1
+    for (int i = lane; i < 2 * kPageTokens * D / 8; i += 32) {
+      const int r = i / (kPageTokens * D / 8), rem = i % (kPageTokens * D / 8);
+      const int tok = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
+      *reinterpret_cast<uint4*>(sb + (r * kPageTokens + tok) * D + c8) =
+          *reinterpret_cast<const uint4*>(row(r, tok) + c8);
+    }
+    __syncwarp();
+    pack_block_warp<16, D>(page, false, lane, [&](int tok, int dim) { return (uint32_t)sb[tok * D + dim]; });
+    pack_block_warp<16, D>(page + code_block_bytes(16, D), true, lane,
+                           [&](int tok, int dim) { return (uint32_t)sb[(kPageTokens + tok) * D + dim]; });
+    return;
+  } else {
+    uint8_t* cs = scr;  // [2][32][D] codes
+    double err[4] = {0.0, 0.0, 0.0, 0.0};
+    auto add_err = [&](int r, float x, double xh) {
+      const double dx = (double)x - xh;
+      err[2 * r] += dx * dx;
+      err[2 * r + 1] += (double)x * (double)x;
+    };
+    if constexpr (F8) {
+      // lane = token: every element is e4m3(x / s_h) of its KV head's scale
+#pragma unroll 1
+      for (int r = 0; r < 2; ++r) {
+        const float sc = r ? vsc : ksc;
+        const __nv_bfloat16* src = row(r, lane);
+#pragma unroll 1
+        for (int c8 = 0; c8 < D; c8 += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
+          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+          uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = __bfloat162float(xv[j]);
+            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(__fdiv_rn(x, sc), __NV_SATFINITE, __NV_E4M3);
+            packed[j >> 2] |= (uint32_t)c << (8 * (j & 3));
+            add_err(r, x, (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3))) * sc);
+          }
+          *reinterpret_cast<uint2*>(cs + (r * kPageTokens + lane) * D + c8) = make_uint2(packed[0], packed[1]);
+        }
+      }
+      __syncwarp();
+      pack_block_warp<8, D>(page, false, lane, [&](int tok, int dim) { return (uint32_t)cs[tok * D + dim]; });
+      pack_block_warp<8, D>(page + code_block_bytes(8, D), true, lane,
+                            [&](int tok, int dim) { return (uint32_t)cs[(kPageTokens + tok) * D + dim]; });
+    } else {
+      constexpr int nk = PT ? kPageTokens : D;  // key scale/zero pairs
+      uint8_t* vblk = page + code_block_bytes(KB, D);
+      __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
+      __half* kzero = kscale + nk;
+      __half* vscale = kzero + nk;
+      __half* vzero = vscale + kPageTokens;
+      // per token over head_dim (values; keys in per-token mode): lane = token
+      auto per_token = [&](int r, int qmax, __half* sdst, __half* zdst) {
+        const __nv_bfloat16* src = row(r, lane);
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll 1
+        for (int c8 = 0; c8 < D; c8 += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
+          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = __bfloat162float(xv[j]);
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+        }
+        const QParams q = make_qparams(mn, mx, qmax);
+        const double s = (double)__half2float(q.s_h), z = (double)q.z;
+#pragma unroll 1
+        for (int c8 = 0; c8 < D; c8 += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
+          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+          uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = __bfloat162float(xv[j]);
+            const uint32_t c = quant_code(x, q, qmax);
+            packed[j >> 2] |= c << (8 * (j & 3));
+            add_err(r, x, (double)c * s + z);
+          }
+          *reinterpret_cast<uint2*>(cs + (r * kPageTokens + lane) * D + c8) = make_uint2(packed[0], packed[1]);
+        }
+        sdst[lane] = q.s_h;
+        zdst[lane] = q.z_h;
+      };
+      if constexpr (PT) {
+        per_token(0, (1 << KB) - 1, kscale, kzero);
+      } else {
+        // keys per channel over the 32 tokens: lane owns channels lane * NC .. + NC - 1
+        constexpr int NC = D / 32;
+        constexpr int qmax = (1 << KB) - 1;
+        const int c0 = lane * NC;
+        float mn[NC], mx[NC];
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+          mn[j] = INFINITY;
+          mx[j] = -INFINITY;
+        }
+#pragma unroll 1
+        for (int tok = 0; tok < kPageTokens; ++tok) {
+          const __nv_bfloat16* src = row(0, tok) + c0;
+#pragma unroll
+          for (int j = 0; j < NC; ++j) {
+            const float x = __bfloat162float(src[j]);
+            mn[j] = fminf(mn[j], x);
+            mx[j] = fmaxf(mx[j], x);
+          }
+        }
+        QParams q[NC];
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+          q[j] = make_qparams(mn[j], mx[j], qmax);
+          const int slot = kmeta_slot<D>(c0 + j);
+          kscale[slot] = q[j].s_h;
+          kzero[slot] = q[j].z_h;
+        }
+#pragma unroll 1
+        for (int tok = 0; tok < kPageTokens; ++tok) {
+          const __nv_bfloat16* src = row(0, tok) + c0;
+#pragma unroll
+          for (int j = 0; j < NC; ++j) {
+            const float x = __bfloat162float(src[j]);
+            const uint32_t c = quant_code(x, q[j], qmax);
+            cs[tok * D + c0 + j] = (uint8_t)c;
+            add_err(0, x, (double)c * (double)__half2float(q[j].s_h) + (double)q[j].z);
+          }
+        }
+      }
+      per_token(1, (1 << VB) - 1, vscale, vzero);
+      __syncwarp();
+      pack_block_warp<KB, D>(page, false, lane, [&](int tok, int dim) { return (uint32_t)cs[tok * D + dim]; });
+      pack_block_warp<VB, D>(vblk, true, lane,
+                             [&](int tok, int dim) { return (uint32_t)cs[(kPageTokens + tok) * D + dim]; });
+    }
+    // this flush's error sums: warp shuffles, then one fp64 atomic per sum
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      double v = err[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      err[i] = v;
+    }
+    if (err_stats && lane == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) atomicAdd(&err_stats[i], err[i]);
+      atomicAdd(&err_stats[4], (double)(kPageTokens * D));
+    }
+  }
+}
+
 // ---------------------------------------------------------- warp-segment kernel --
 // Short sequences (token rows, G <= 4): warp w of CTA c attends segments
 // s = c * kWarps + w, then s + gridDim.x * kWarps, ... on its own -- query rows
@@ -1590,12 +1774,18 @@ struct WarpCfg {
   static constexpr int SMEM = QBUF_OFF + kWarps * QSLOT;
 };
 
-template <int KB, int VB, int D, bool PT, bool F8>
+// AP (kvq_decode_step): before attending segment (b, h) the warp appends its new
+// token -- into the window, or, when it completes a group, quantized into the
+// next page, which the warp then attends from global memory -- and the last of
+// sequence b's H warps to have read the old length publishes the new one (the
+// acquire-release increment orders every read before that write).
+template <int KB, int VB, int D, bool PT, bool F8, bool AP = false>
 __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
     decode_warp_kernel(DecodeParams p) {
   pdl_enter();
   using C = Cfg<KB, VB, D, PT, F8>;
   using WC = WarpCfg<KB, VB, D, PT, F8>;
+  static_assert(C::R * C::STAGE >= 2 * kPageTokens * D * (C::kBf16 ? 2 : 1), "flush scratch fits the warp's ring");
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = p.n_kv_heads, G = p.gqa;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1621,8 +1811,48 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
   int issued = 0, consumed = 0, nq = 0;
   for (int s = blockIdx.x * kWarps + warp; s < S && ok; s += stride, ++nq) {
     const int b = s / H, h = s % H;
-    const int T = p.len[b];
-    const int P = T / kPageTokens, W = T % kPageTokens;
+    int T, P;              // tokens attended; pages read through the ring
+    bool flushed = false;  // AP: page P, just written, is attended too
+    if constexpr (AP) {
+      int t0 = 0;
+      if (lane == 0) {
+        t0 = p.step_len[b];
+        if (atomic_add_acq_rel(&p.append_ctr[b], 1) == H - 1) {
+          p.append_ctr[b] = 0;
+          if (t0 < p.max_tokens) p.step_len[b] = t0 + 1;
+        }
+      }
+      t0 = __shfl_sync(0xffffffffu, t0, 0);
+      P = t0 / kPageTokens;
+      if (t0 < p.max_tokens) {
+        T = t0 + 1;
+        __nv_bfloat16* wwin = p.step_window + ((int64_t)s * 2) * kPageTokens * D;
+        const __nv_bfloat16* kn = p.k_new + (int64_t)s * D;
+        const __nv_bfloat16* vn = p.v_new + (int64_t)s * D;
+        if (T % kPageTokens != 0) {
+          // the new token into window slot t0 mod 32
+          const int slot = t0 % kPageTokens;
+          for (int d = 2 * lane; d < D; d += 64) {
+            *reinterpret_cast<uint32_t*>(wwin + slot * D + d) = *reinterpret_cast<const uint32_t*>(kn + d);
+            *reinterpret_cast<uint32_t*>(wwin + (kPageTokens + slot) * D + d) =
+                *reinterpret_cast<const uint32_t*>(vn + d);
+          }
+        } else {
+          flushed = true;
+          warp_flush<KB, VB, D, PT, F8>(p.step_pages + ((int64_t)s * p.max_pages + P) * p.page_bytes, wwin, kn, vn,
+                                        ring, F8 ? p.fp8_scales[h] : 1.f, F8 ? p.fp8_scales[H + h] : 1.f,
+                                        p.err_stats, lane);
+        }
+        __syncwarp();  // the window row or page and the ring scratch are complete for every lane
+      } else {
+        T = t0;  // a full sequence is left unchanged and the cache's error flag raised
+        if (lane == 0 && p.err) atomicExch(p.err, 2);
+      }
+    } else {
+      T = p.len[b];
+      P = T / kPageTokens;
+    }
+    const int W = T % kPageTokens;
     const uint8_t* base = p.pages + ((int64_t)s * p.max_pages) * p.page_bytes;
     const __nv_bfloat16* win = p.window + ((int64_t)s * 2) * kPageTokens * D;
     int next = 0;  // next page of this segment to copy
@@ -1750,6 +1980,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
       }
     }
     if (!ok) break;
+    if (flushed) {
+      // the page this warp has just written (generic loads: it never went through the async proxy)
+      const uint8_t* page = base + (int64_t)P * p.page_bytes;
+      if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
+      else if constexpr (F8) attend_f8page_tok<D>(page, st, qzb, wscr, partf, lane);
+      else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
+      else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
+    }
     if (W > 0) {
       if constexpr (!C::kBf16) {
         to_true_units();
@@ -1861,11 +2099,63 @@ cudaError_t launch_d(int kb, int vb, const DecodeParams& p, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
+// fused append + decode (one warp per segment); not launched when the segments
+// do not fit one resident wave of warps
+template <int KB, int VB, int D, bool PT, bool F8>
+cudaError_t launch_step4(const DecodeParams& p, cudaStream_t s) {
+  using WC = WarpCfg<KB, VB, D, PT, F8>;
+  static bool configured = false;
+  static int occ = 0;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_warp_kernel<KB, VB, D, PT, F8, true>, kThreads,
+                                                      WC::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int64_t ctas = ((int64_t)p.batch * p.n_kv_heads + kWarps - 1) / kWarps;
+  if (ctas < 1 || ctas > (int64_t)occ * p.sm_count) return cudaErrorNotSupported;
+  return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8, true>, dim3((unsigned)ctas), dim3(kThreads),
+                    (size_t)WC::SMEM, s, p);
+}
+
+template <int KB, int VB, int D>
+cudaError_t launch_step3(const DecodeParams& p, cudaStream_t s) {
+  if (p.gqa > 4) return cudaErrorNotSupported;
+  if constexpr (KB == 8 && VB == 8) {
+    if (p.fmt != 0) return launch_step4<KB, VB, D, false, true>(p, s);
+  }
+  if constexpr (KB != 16) {
+    if (p.key_mode != 0) return launch_step4<KB, VB, D, true, false>(p, s);
+  }
+  return launch_step4<KB, VB, D, false, false>(p, s);
+}
+
+template <int D>
+cudaError_t launch_step_d(int kb, int vb, const DecodeParams& p, cudaStream_t s) {
+#define KVQ_PAIR(K_, V_) \
+  if (kb == K_ && vb == V_) return launch_step3<K_, V_, D>(p, s);
+  KVQ_PAIR(2, 2) KVQ_PAIR(2, 4) KVQ_PAIR(2, 8)
+  KVQ_PAIR(4, 2) KVQ_PAIR(4, 4) KVQ_PAIR(4, 8)
+  KVQ_PAIR(8, 2) KVQ_PAIR(8, 4) KVQ_PAIR(8, 8)
+  KVQ_PAIR(16, 16)
+#undef KVQ_PAIR
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s) {
   if (D == 64) return launch_d<64>(kb, vb, p, s);
   if (D == 128) return launch_d<128>(kb, vb, p, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_step(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s) {
+  if (D == 64) return launch_step_d<64>(kb, vb, p, s);
+  if (D == 128) return launch_step_d<128>(kb, vb, p, s);
   return cudaErrorInvalidValue;
 }
 

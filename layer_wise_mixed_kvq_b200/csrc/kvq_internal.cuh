@@ -100,6 +100,16 @@ struct DecodeParams {
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
   int warp_split;        // tensor-core kernel, G <= 4: one warp per segment (if the segments fit the
                          // resident warps) instead of CTAs sharing each segment's pages
+  // fused decode step (kvq_decode_step): the warp attending segment (b, h) first
+  // appends that segment's new token; the same buffers as above, writable
+  uint8_t* step_pages;
+  __nv_bfloat16* step_window;
+  int32_t* step_len;
+  int32_t* append_ctr;           // [batch], zero between launches
+  const __nv_bfloat16* k_new;    // [batch][n_kv_heads][head_dim]
+  const __nv_bfloat16* v_new;
+  double* err_stats;
+  int max_tokens;
 };
 
 // Programmatic dependent launch. Every kernel of the library starts with
@@ -159,8 +169,15 @@ int choose_chunk(int sm_count, int64_t total_pages, int64_t max_pages_per_seq, i
 int seg_overhead_units();
 // Message returned by kvq_last_error() on this thread.
 void set_last_error(const std::string& msg);
+// KVQ_DECODE_KERNEL=simt: the CUDA-core decode kernel instead of the tensor-core one.
+bool decode_uses_simt();
+
 // Layer-map dispatcher: the kernel instance for a layer's pair.
 cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
+// Fused one-token append + decode attention with one warp per segment (query
+// groups of at most 4 heads). cudaErrorNotSupported when the segments do not fit
+// the resident warps (nothing launched: the caller runs the two kernels).
+cudaError_t launch_decode_step(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s);
 
 }  // namespace kvq
 

@@ -25,7 +25,7 @@ EXPORTS = (
     "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
     "kvq_export_bytes", "kvq_export_layer", "kvq_sync", "kvq_launch_count", "kvq_last_error",
     "kvq_status_string", "kvq_set_fp8_scales", "kvq_layer_error", "kvq_refresh_lengths",
-    "kvq_set_decode_mode",
+    "kvq_set_decode_mode", "kvq_decode_step",
 )
 
 
@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
                                               c.c_int, P, P]),
         "kvq_set_split_pages": (c.c_int, [P, c.c_int]),
         "kvq_set_decode_mode": (c.c_int, [P, c.c_int]),
+        "kvq_decode_step": (c.c_int, [P, c.c_int, P, P, P, c.c_int, P, P]),
         "kvq_seq_len": (c.c_int64, [P, c.c_int, c.c_int]),
         "kvq_bytes": (c.c_int64, [P, c.c_int, c.c_int, c.c_int]),
         "kvq_export_bytes": (c.c_int64, [P, c.c_int, c.c_int]),
@@ -185,6 +186,20 @@ def kvq_decode_attn(cache, layer, Q, out, stream=None) -> None:
         raise ValueError("Q must be bfloat16 and out float32")
     _check(lib.kvq_decode_attn(ctypes.c_void_p(cache), int(layer), _dev_ptr(Q), int(Q.shape[0]), _dev_ptr(out),
                                _stream(stream)))
+
+
+def kvq_decode_step(cache, layer, K, V, Q, out, stream=None) -> None:
+    """Append one token per sequence (K, V: bf16 CUDA [batch, n_kv_heads, head_dim]) and attend
+    (Q: bf16 CUDA [batch, n_q_heads, head_dim]; out: fp32 CUDA, same shape)."""
+    import torch
+    if K.dtype != torch.bfloat16 or V.dtype != torch.bfloat16 or Q.dtype != torch.bfloat16:
+        raise ValueError("K, V and Q must be bfloat16")
+    if out.dtype != torch.float32:
+        raise ValueError("out must be float32")
+    if K.shape[0] != Q.shape[0] or V.shape[0] != Q.shape[0]:
+        raise ValueError("K, V and Q must have the same batch")
+    _check(lib.kvq_decode_step(ctypes.c_void_p(cache), int(layer), _dev_ptr(K), _dev_ptr(V), _dev_ptr(Q),
+                               int(Q.shape[0]), _dev_ptr(out), _stream(stream)))
 
 
 def kvq_decode_attn_noalloc(pair, head_dim, n_q_heads, n_kv_heads, pages, max_pages, window, seq_len,
