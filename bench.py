@@ -1,8 +1,9 @@
 """Benchmark of the mixed-precision KV decode step on B200.
 
 One step = for every layer of the stack: append one new token per sequence
-(kvq_append) and decode attention for every query head (kvq_decode_attn), over
-a cache prefilled to the workload's context. Default workload: the
+and decode attention for every query head (kvq_decode_step: one fused kernel
+where the one-warp-per-segment split applies, else kvq_append then
+kvq_decode_attn), over a cache prefilled to the workload's context. Default workload: the
 Llama-3.1-8B-shaped uniform K4V4 stack (32 layers, 32 query / 8 KV heads,
 head_dim 128, batch 16, context 4096).
 
@@ -262,13 +263,19 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream()
 
     def step(s, events=None):
+        # one decode step per layer through the public call (kvq_decode_step: the
+        # append fused into the attention kernel where the one-warp-per-segment
+        # split applies, the two kernels otherwise); the kernel-timing pass calls
+        # them separately so the events bracket the decode attention kernel alone
         for layer in range(NL):
+            if events is None:
+                kvq.kvq_decode_step(cache, layer, steps_K[s][layer], steps_V[s][layer], steps_Q[s][layer],
+                                    outs[layer], stream)
+                continue
             kvq.kvq_append(cache, layer, steps_K[s][layer], steps_V[s][layer], ones, stream)
-            if events is not None:
-                events[layer][0].record(stream)
+            events[layer][0].record(stream)
             kvq.kvq_decode_attn(cache, layer, steps_Q[s][layer], outs[layer], stream)
-            if events is not None:
-                events[layer][1].record(stream)
+            events[layer][1].record(stream)
 
     for s in range(args.warmup):
         step(s)
@@ -347,8 +354,7 @@ def run_gpu(args, w):
     for s in range(e2e_steps):
         dstage.copy_(hstage[s], non_blocking=True)
         for layer in range(NL):
-            kvq.kvq_append(cache, layer, dK[layer], dV[layer], ones, stream)
-            kvq.kvq_decode_attn(cache, layer, dQ[layer], douts[layer], stream)
+            kvq.kvq_decode_step(cache, layer, dK[layer], dV[layer], dQ[layer], douts[layer], stream)
         hout.copy_(douts, non_blocking=True)
     b_.record(stream)
     torch.cuda.synchronize()
@@ -369,8 +375,7 @@ def run_gpu(args, w):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=gstream):
         for layer in range(NL):
-            kvq.kvq_append(cache, layer, gK[layer], gV[layer], ones)
-            kvq.kvq_decode_attn(cache, layer, gQ[layer], outs[layer])
+            kvq.kvq_decode_step(cache, layer, gK[layer], gV[layer], gQ[layer], outs[layer])
     stream.wait_stream(gstream)
     graph.replay()                      # warm-up replay
     torch.cuda.synchronize()
@@ -392,7 +397,7 @@ def run_gpu(args, w):
     del graph
     graph_result = {"value": g_total / (g_max / 1e3) / 1e9, "unit": "GB/s", "steps": graph_steps,
                     "ms_per_step": g_max / graph_steps, "decode_steps_per_s": graph_steps / (g_max / 1e3) * world,
-                    "note": "same step (append + decode per layer) captured in one CUDA graph, inputs resident"}
+                    "note": "same step (kvq_decode_step per layer) captured in one CUDA graph, inputs resident"}
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
