@@ -7,12 +7,18 @@
 // dequantized per channel (x = code * s_c + z_c over each 32-token page) and
 // values per token (x = code * s_t + z_t).
 //
-// Work split: grid (splits, n_kv_heads, batch), 4 warps per CTA. Each warp
-// streams its own pages (p0 + warp, p0 + warp + 4, ...) through a private ring
-// of shared-memory stages filled by bulk copies (cp.async.bulk, one copy per
-// page, mbarrier completion) and keeps its own online-softmax state. The CTA
-// merges its warps, then either writes the output (one split) or a partial
-// (acc, m, l) that the last CTA of the (sequence, head) merges.
+// Work splits, 4 warps per CTA, each warp streaming pages through a private
+// ring of shared-memory stages filled by bulk copies (cp.async.bulk, one copy
+// per page, mbarrier completion) with its own online-softmax state:
+//  * shared split (decode_mma_kernel): a persistent grid cuts all (sequence,
+//    KV head) segments' pages into balanced contiguous slices, one per CTA; the
+//    CTA's warps take a segment part's pages in turn, merge in shared memory,
+//    and either write the output or leave a split record that the last CTA of
+//    the segment merges;
+//  * warp split (decode_warp_kernel, short sequences, G <= 4): each warp
+//    attends whole segments alone and writes their outputs; its fused form
+//    first appends the segment's new token (window slot, or a warp-level
+//    flush of the completed group into the next page).
 //
 // Per page (32 tokens), with MMA rows = query heads: row g holds the high f16
 // part of head g's operand and row g + 8 the low part (hi + lo carries ~22
