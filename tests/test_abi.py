@@ -112,4 +112,6 @@ def test_null_cache_calls_fail_cleanly(kvq):
     assert kvq.lib.kvq_decode_attn(None, 0, None, 1, None, None) == kvq.KVQ_EINVAL
     n = (ctypes.c_int32 * 1)(1)
     assert kvq.lib.kvq_append(None, 0, None, None, 0, n, 1, None) == kvq.KVQ_EINVAL
+    assert kvq.lib.kvq_decode_step(None, 0, None, None, None, 1, None, None) == kvq.KVQ_EINVAL
+    assert kvq.lib.kvq_set_decode_mode(None, -1) == kvq.KVQ_EINVAL
     kvq.kvq_cache_destroy(None)
