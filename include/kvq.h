@@ -180,9 +180,11 @@ kvq_status kvq_append(kvq_cache* cache, int layer, const void* K, const void* V,
  *   exact bf16), q head hq reading KV head hq / (n_q_heads/n_kv_heads).
  *   Q:   device bf16 [batch, n_q_heads, head_dim], 16-byte aligned.
  *   out: device fp32 [batch, n_q_heads, head_dim], 16-byte aligned.
- * An empty sequence gives zeros. One kernel launch: the sequence is split
- * across CTAs and the last CTA of each (sequence, KV head) merges the partial
- * softmax states. Errors: KVQ_EINVAL. */
+ * An empty sequence gives zeros. One kernel launch: either the CTAs of a
+ * persistent grid share each (sequence, KV head) segment's pages and the last
+ * CTA of a split segment merges the partial softmax states, or, for short
+ * sequences (see kvq_set_decode_mode), one warp attends each segment whole.
+ * Errors: KVQ_EINVAL. */
 kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch, float* out,
                            void* stream);
 
