@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default="llama_k4v4", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--layers", type=int, default=0,
                     help="profile a truncated stack (N layers from --first-layer); 0 = the workload's full stack")
     ap.add_argument("--first-layer", type=int, default=0, help="first layer of a truncated stack")
@@ -137,39 +137,74 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------- CPU oracle --
-def cpu_baseline(w, seconds):
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, seconds, threads=(1,)):
     """The oracle, as it stands, timed on this host on a bounded sample of the
-    workload: whole layers (every KV head) of single sequences at the
-    workload's context, prefill appends untimed, decode attention timed."""
+    workload. One oracle layer per distinct pair of the layer map, holding the
+    workload's whole batch at its context (+1, the step's token; prefill appends
+    untimed); each is attended repeatedly with fresh queries for its share of
+    `seconds` per thread count, the (sequence, KV head) units shared out over
+    that many host threads. The stack's rate weights every pair by its layer
+    count: GB/s = sum of layer bytes / sum of layer times. One result per entry
+    of `threads`."""
     import oracle
     oracle.build()
-    done_bytes, t_attn, samples = 0, 0.0, 0
-    layer = 0
-    ctx = int(synth.context_lengths(w, 1)[0])
-    while t_attn < seconds and samples < 1024:
-        pair = w.layer_map[layer % w.n_layers]
+    lens = synth.context_lengths(w) + 1
+    pairs = []
+    for layer, pair in enumerate(w.layer_map):
+        if pair not in [p for p, _, _ in pairs]:
+            pairs.append((pair, layer, sum(1 for q in w.layer_map if q == pair)))
+    per_pair = seconds / len(pairs) / len(threads)
+    acc = {n: {"stack_s": 0.0, "reps": 0, "t": 0.0} for n in threads}
+    stack_bytes = 0.0
+    for pair, layer, count in pairs:
         key_mode = pair[2] if len(pair) > 2 else 0
         fmt = pair[3] if len(pair) > 3 else 0
         scales = w.fp8_scales if fmt else (None, None)
-        L = oracle.OracleLayer(pair[0], pair[1], 1, w.n_kv_heads, w.head_dim, key_mode=key_mode, fmt=fmt,
+        L = oracle.OracleLayer(pair[0], pair[1], w.batch, w.n_kv_heads, w.head_dim, key_mode=key_mode, fmt=fmt,
                                k_scales=scales[0], v_scales=scales[1])
-        K, V = synth.kv_tokens(w, layer, ctx + 1)
-        L.append(K, V, [ctx + 1])
-        Q = synth.queries(w, layer, batch=1)
-        t0 = time.perf_counter()
-        L.attend(Q)
-        t_attn += time.perf_counter() - t0
-        T = ctx + 1
-        P, W = T // 32, T % 32
+        K, V = synth.kv_tokens(w, layer, int(lens.sum()))
+        L.append(K, V, [int(x) for x in lens])
+        del K, V
         page = oracle.page_bytes(pair[0], pair[1], w.head_dim, key_mode, fmt)
-        done_bytes += w.n_kv_heads * (P * page + W * w.head_dim * 4)
-        samples += 1
-        layer += 1
-    gbs = done_bytes / t_attn / 1e9
-    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{samples} single-sequence layer(s) of {w.name} at context {ctx + 1}, all "
-                      f"{w.n_q_heads} query heads, fp64 attention; {t_attn:.1f} s of attention",
-            "decode_layers_per_s": samples / t_attn}
+        stack_bytes += count * w.n_kv_heads * sum((int(T) // 32) * page + (int(T) % 32) * w.head_dim * 4
+                                                  for T in lens)
+        for n in threads:
+            t, reps = 0.0, 0
+            while reps == 0 or t < per_pair:
+                Q = synth.queries(w, layer, salt=100 + reps)
+                t0 = time.perf_counter()
+                L.attend(Q, threads=n)
+                t += time.perf_counter() - t0
+                reps += 1
+            acc[n]["stack_s"] += count * t / reps
+            acc[n]["reps"] += reps
+            acc[n]["t"] += t
+        del L
+    out = []
+    for n in threads:
+        a = acc[n]
+        out.append({"value": stack_bytes / a["stack_s"] / 1e9, "unit": "GB/s", "cores": n, "kind": "oracle",
+                    "sample": f"{a['reps']} whole-layer attention(s) of {w.name} (batch {w.batch}, all "
+                              f"{w.n_q_heads} query heads, context {int(lens.min())}-{int(lens.max())}), one "
+                              f"oracle layer per distinct pair ({len(pairs)}), fp64 attention on {n} host "
+                              f"thread(s), {a['t']:.1f} s of attention; the stack rate weights the pairs by "
+                              f"layer count",
+                    "ms_per_step": a["stack_s"] * 1e3})
+    return out
+
+
+def cpu_baselines(w, seconds):
+    """All host cores (the reported baseline) with one thread beside it."""
+    allc, one = cpu_baseline(w, seconds, threads=(host_cores(), 1))
+    allc["single_thread"] = {k: one[k] for k in ("value", "unit", "cores", "sample", "ms_per_step")}
+    return allc
 
 
 def workload_config(w, equiv_bits, world):
@@ -189,20 +224,17 @@ def run_reference(args, w):
     rank, world, _ = replicas.world()
     if rank != 0:
         return 0
-    cb = cpu_baseline(w, args.cpu_seconds / 2)
-    # one "step" = one full layer stack for one sequence, bounded per step
-    per_layer_s = 1.0 / cb["decode_layers_per_s"]
-    bytes_per_layer = cb["value"] * 1e9 * per_layer_s
+    cb = cpu_baseline(w, args.cpu_seconds, threads=(host_cores(),))[0]
     value = cb["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_layer_s * w.n_layers * 1e3, "higher_is_better": True, "scaling": "weak",
+        # one step = every layer of the stack over the whole batch (the GPU arm's step)
+        "ms_per_step": cb["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, oracle_equiv_bits(w), 1),
         "cpu_baseline": {k: cb[k] for k in ("kind", "cores", "sample")} | {"value": value, "unit": "GB/s"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "bytes_per_layer": bytes_per_layer,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -401,8 +433,7 @@ def run_gpu(args, w):
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(w, args.cpu_seconds)
-        cb.pop("decode_layers_per_s", None)
+        cb = cpu_baselines(w, args.cpu_seconds)
 
     traffic = traffic_from_profile(w.name)
     clocks = clk.summary()

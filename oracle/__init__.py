@@ -20,7 +20,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kvq_oracle.cpp")
 _LIB = os.path.join(_HERE, "liboracle.so")
-_CXXFLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC"]
+_CXXFLAGS = ["-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC", "-pthread"]
 _lock = threading.Lock()
 _lib = None
 
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "oracle_layer_export": (None, [P, c.c_int, P]),
             "oracle_layer_dequant": (None, [P, c.c_int, c.c_int, P, P]),
             "oracle_layer_attend": (None, [P, P, c.c_int, c.c_int, P, P]),
+            "oracle_layer_attend_threads": (None, [P, P, c.c_int, c.c_int, P, P, c.c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -243,8 +244,11 @@ class OracleLayer:
             lib().oracle_layer_dequant(self._h, b, h, _ptr(K), _ptr(V))
         return K, V
 
-    def attend(self, Q: np.ndarray, batch: int | None = None, seqs=None) -> np.ndarray:
-        """Q: [batch, Hq, D] (bf16 values). Returns fp64 [batch, Hq, D]."""
+    def attend(self, Q: np.ndarray, batch: int | None = None, seqs=None, threads: int = 1) -> np.ndarray:
+        """Q: [batch, Hq, D] (bf16 values). Returns fp64 [batch, Hq, D].
+
+        threads > 1 shares the (sequence, KV head) units out over that many host
+        threads; the result is the same."""
         Q = np.ascontiguousarray(Q, dtype=np.float32)
         batch = Q.shape[0] if batch is None else batch
         hq = Q.shape[1]
@@ -256,5 +260,8 @@ class OracleLayer:
             mask = np.zeros(batch, dtype=np.uint8)
             mask[list(seqs)] = 1
             mptr = _ptr(mask)
-        lib().oracle_layer_attend(self._h, _ptr(Q), hq, batch, mptr, _ptr(out))
+        if threads > 1:
+            lib().oracle_layer_attend_threads(self._h, _ptr(Q), hq, batch, mptr, _ptr(out), int(threads))
+        else:
+            lib().oracle_layer_attend(self._h, _ptr(Q), hq, batch, mptr, _ptr(out))
         return out

@@ -5,7 +5,7 @@
 // benchmark's CPU-baseline leg may load it; the product library never does, and
 // the two share no source, header, table or helper.
 //
-// Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -shared -fPIC.
+// Build: g++ -O2 -std=c++17 -ffp-contract=off -fno-fast-math -shared -fPIC -pthread.
 // -ffp-contract=off keeps every fp32 multiply and add a separate IEEE
 // operation, which is what makes the packed codes reproducible bit for bit.
 //
@@ -65,6 +65,9 @@
 #include <cstdlib>
 #include <vector>
 #include <algorithm>
+#include <atomic>
+#include <thread>
+#include <utility>
 
 namespace {
 
@@ -648,44 +651,78 @@ void oracle_layer_dequant(void* p, int b, int h, double* Kh, double* Vh) {
   }
 }
 
+}  // extern "C"
+
+namespace {
+
+// Decode attention of the G query heads of KV head h of sequence b (fp64).
+void attend_one(void* p, const float* Q, int n_q_heads, int b, int h, double* out) {
+  Layer* L = static_cast<Layer*>(p);
+  const int D = L->D, H = L->hkv, G = n_q_heads / H;
+  const double inv_sqrt_d = 1.0 / std::sqrt((double)D);
+  const int64_t T = L->seqs[b].len;
+  std::vector<double> Kh(T * D), Vh(T * D), sc(T);
+  if (T > 0) oracle_layer_dequant(p, b, h, Kh.data(), Vh.data());
+  for (int gq = 0; gq < G; ++gq) {
+    int hq = h * G + gq;
+    double* o = out + ((int64_t)b * n_q_heads + hq) * D;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (T == 0) continue;
+    std::vector<double> q(D);
+    for (int d = 0; d < D; ++d)
+      q[d] = bf16_to_f32(f32_to_bf16_rne(Q[((int64_t)b * n_q_heads + hq) * D + d]));
+    double m = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) {
+      double acc = 0;
+      for (int d = 0; d < D; ++d) acc += q[d] * Kh[t * D + d];
+      sc[t] = acc * inv_sqrt_d;
+      m = std::max(m, sc[t]);
+    }
+    double l = 0;
+    for (int64_t t = 0; t < T; ++t) { sc[t] = std::exp(sc[t] - m); l += sc[t]; }
+    for (int64_t t = 0; t < T; ++t) {
+      double w = sc[t] / l;
+      for (int d = 0; d < D; ++d) o[d] += w * Vh[t * D + d];
+    }
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
 // Decode attention for every (b < batch, q head): Q [batch][Hq][D] fp32 holding
 // bf16 values (rounded on entry), out [batch][Hq][D] fp64. Only the sequences
 // listed in `seq_mask` (nonzero) are computed when seq_mask is not null.
 void oracle_layer_attend(void* p, const float* Q, int n_q_heads, int batch, const uint8_t* seq_mask,
                          double* out) {
   Layer* L = static_cast<Layer*>(p);
-  const int D = L->D, H = L->hkv, G = n_q_heads / H;
-  const double inv_sqrt_d = 1.0 / std::sqrt((double)D);
   for (int b = 0; b < batch; ++b) {
     if (seq_mask && !seq_mask[b]) continue;
-    const int64_t T = L->seqs[b].len;
-    std::vector<double> Kh(T * D), Vh(T * D), sc(T);
-    for (int h = 0; h < H; ++h) {
-      if (T > 0) oracle_layer_dequant(p, b, h, Kh.data(), Vh.data());
-      for (int gq = 0; gq < G; ++gq) {
-        int hq = h * G + gq;
-        double* o = out + ((int64_t)b * n_q_heads + hq) * D;
-        for (int d = 0; d < D; ++d) o[d] = 0.0;
-        if (T == 0) continue;
-        std::vector<double> q(D);
-        for (int d = 0; d < D; ++d)
-          q[d] = bf16_to_f32(f32_to_bf16_rne(Q[((int64_t)b * n_q_heads + hq) * D + d]));
-        double m = -INFINITY;
-        for (int64_t t = 0; t < T; ++t) {
-          double acc = 0;
-          for (int d = 0; d < D; ++d) acc += q[d] * Kh[t * D + d];
-          sc[t] = acc * inv_sqrt_d;
-          m = std::max(m, sc[t]);
-        }
-        double l = 0;
-        for (int64_t t = 0; t < T; ++t) { sc[t] = std::exp(sc[t] - m); l += sc[t]; }
-        for (int64_t t = 0; t < T; ++t) {
-          double w = sc[t] / l;
-          for (int d = 0; d < D; ++d) o[d] += w * Vh[t * D + d];
-        }
-      }
-    }
+    for (int h = 0; h < L->hkv; ++h) attend_one(p, Q, n_q_heads, b, h, out);
   }
+}
+
+// The same attention with the (sequence, KV head) units shared out over
+// n_threads host threads (each unit writes its own output rows, so the result
+// is identical to oracle_layer_attend's). Used to time the oracle on every core.
+void oracle_layer_attend_threads(void* p, const float* Q, int n_q_heads, int batch, const uint8_t* seq_mask,
+                                 double* out, int n_threads) {
+  Layer* L = static_cast<Layer*>(p);
+  std::vector<std::pair<int, int>> units;
+  for (int b = 0; b < batch; ++b)
+    if (!seq_mask || seq_mask[b])
+      for (int h = 0; h < L->hkv; ++h) units.emplace_back(b, h);
+  std::atomic<size_t> next{0};
+  auto worker = [&]() {
+    for (size_t i = next++; i < units.size(); i = next++)
+      attend_one(p, Q, n_q_heads, units[i].first, units[i].second, out);
+  };
+  const int n = std::max(1, std::min<int>(n_threads, (int)units.size()));
+  std::vector<std::thread> pool;
+  for (int t = 1; t < n; ++t) pool.emplace_back(worker);
+  worker();
+  for (auto& th : pool) th.join();
 }
 
 }  // extern "C"

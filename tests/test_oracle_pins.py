@@ -434,3 +434,20 @@ def test_gqa_head_mapping(oracle):
     out = L.attend(np.ones((1, H * G, D), dtype=np.float32))
     for hq in range(H * G):
         np.testing.assert_allclose(out[0, hq], float(hq // G + 1), rtol=0, atol=1e-12)
+
+
+def test_threaded_attention_equals_single_thread(oracle):
+    """The oracle's multi-threaded driver (used to time it on every host core)
+    shares out (sequence, KV head) units only: its output is the single-thread
+    output bit for bit, including empty and window-only sequences."""
+    rng = np.random.default_rng(21)
+    lens = [0, 5, 32, 70, 129]
+    L = oracle.OracleLayer(4, 2, len(lens), 3, 64)
+    K = rng.standard_normal((sum(lens), 3, 64)).astype(np.float32)
+    V = rng.standard_normal((sum(lens), 3, 64)).astype(np.float32)
+    L.append(K, V, lens)
+    Q = rng.standard_normal((len(lens), 6, 64)).astype(np.float32)
+    one = L.attend(Q)
+    for n in (2, 3, 64):
+        assert np.array_equal(L.attend(Q, threads=n), one)
+    assert np.array_equal(L.attend(Q, seqs=[1, 4], threads=4)[[1, 4]], one[[1, 4]])
