@@ -184,6 +184,15 @@ kvq_status kvq_append(kvq_cache* cache, int layer, const void* K, const void* V,
  * persistent grid share each (sequence, KV head) segment's pages and the last
  * CTA of a split segment merges the partial softmax states, or, for short
  * sequences (see kvq_set_decode_mode), one warp attends each segment whole.
+ * Launched on a stream that is not being captured, the call passes the
+ * sequence lengths to the kernel (no device-side scan), and, unless the last
+ * launch this cache made on `stream` wrote `layer` (kvq_append,
+ * kvq_decode_step, kvq_cache_reset), the kernel may start copying pages below
+ * those lengths before the preceding kernel on the stream has finished
+ * (programmatic dependent launch). So a kernel of the caller's own that writes
+ * this cache's pages (a caller-owned pool) must not be the one launched right
+ * before this call on the same stream; record an event or launch anything else
+ * in between.
  * Errors: KVQ_EINVAL. */
 kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch, float* out,
                            void* stream);
@@ -195,16 +204,17 @@ kvq_status kvq_decode_attn(kvq_cache* cache, int layer, const void* Q, int batch
  *   K, V: device bf16 [batch, n_kv_heads, head_dim], the new token of each
  *         sequence, 16-byte aligned.
  *   Q, out: as for kvq_decode_attn.
- * Where kvq_decode_attn would take the one-warp-per-segment split (short
- * sequences, at most 4 query heads per KV head; see kvq_set_decode_mode) this is
- * ONE kernel launch: the warp that attends segment (b, h) first writes its new
- * token into the window or, when the token completes a 32-token group,
- * quantizes and packs that group into the next page and attends it from there.
- * Otherwise it runs the two kernels. The KVTuner pages warn that per-layer
- * dispatch overhead can erase the savings of a small KV cache; at short
- * sequences the append kernel costs about as much as the attention itself.
- * A CUDA graph keeps the form it was captured with; inside a graph the one-
- * token capacity guard of kvq_append applies (see kvq_refresh_lengths).
+ * ONE kernel launch, in either work split of kvq_decode_attn: the warp that
+ * owns segment (b, h)'s tail unit first writes its new token into the window
+ * or, when the token completes a 32-token group, quantizes and packs that group
+ * into the next page (the append kernel's quantizer and packing, bit for bit)
+ * and attends it from there; the other warps stream the older pages meanwhile.
+ * The KVTuner pages warn that per-layer dispatch overhead can erase the savings
+ * of a small KV cache. With KVQ_DECODE_KERNEL=simt (the CUDA-core check kernel)
+ * it runs kvq_append and kvq_decode_attn. The same early page copies as
+ * kvq_decode_attn apply. Inside a captured CUDA graph the kernel reads and
+ * advances the device lengths, and a sequence already at max_tokens is left
+ * unchanged with the cache's error flag raised (see kvq_refresh_lengths).
  * Errors: KVQ_EINVAL, KVQ_ECAPACITY (some sequence is full; nothing changes). */
 kvq_status kvq_decode_step(kvq_cache* cache, int layer, const void* K, const void* V, const void* Q, int batch,
                            float* out, void* stream);
@@ -233,12 +243,22 @@ kvq_status kvq_decode_step(kvq_cache* cache, int layer, const void* K, const voi
  * serialise them. The scratch holds one 4-byte merge counter per
  * (sequence, KV head) and split-K records of (n_q_heads / n_kv_heads) *
  * (head_dim + 2) * 4 bytes; KVQ_ECAPACITY when the counters leave no room for
- * two records in 16 MiB; KVQ_EINVAL for bad arguments. Nothing is launched on
- * error. */
+ * two records in 16 MiB; KVQ_EINVAL for bad arguments (including more than
+ * 2^31 units of work: batch * n_kv_heads * (max_seq_len/32 + 17)). Nothing is
+ * launched on error. A call whose kernel gave up waiting for a page copy (its
+ * output is then wrong) raises an error word in the same array; read it with
+ * kvq_noalloc_check. */
 kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n_q_heads, int n_kv_heads,
                                    const void* pages, int64_t max_pages, const void* window,
                                    const int32_t* seq_len, int64_t max_seq_len, const void* Q,
                                    int batch, float* out, void* stream);
+
+/* Status of the kvq_decode_attn_noalloc calls made on the current device since
+ * the last check: waits for the device, then returns KVQ_ECUDA (and clears the
+ * word) if one of them gave up waiting for a page copy, KVQ_OK otherwise.
+ * Allocates nothing. Like kvq_decode_attn_noalloc, it has no counterpart on the
+ * KVTuner pages. */
+kvq_status kvq_noalloc_check(void);
 
 /* Per-layer quantization error report ([rebut] Table 3 and the layer-wise
  * error figures: quantization error is tracked layer by layer). Sums over every

@@ -45,7 +45,8 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Geometry {
   int64_t max_pages = 0;
   std::vector<size_t> page_region, window_region;
-  size_t len_region = 0, partial_region = 0, merge_region = 0, append_region = 0, plan_region = 0, err_region = 0;
+  size_t len_region = 0, partial_region = 0, merge_region = 0, append_region = 0, plan_region = 0, err_region = 0,
+         grid_region = 0;
   int64_t partial_slots = 0;
   size_t total = 0;
 };
@@ -83,7 +84,8 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
     size_t wr = round_up((size_t)max_batch * n_kv_heads * 2 * kvq::kPageTokens * head_dim * 2);
     g.page_region.push_back(pr);
     g.window_region.push_back(wr);
-    total += pr + wr + round_up((size_t)max_batch * 4) + round_up((size_t)n_kv_heads * 2 * 4) + round_up(5 * 8);
+    total += pr + wr + round_up((size_t)max_batch * 4) + round_up((size_t)n_kv_heads * 2 * 4) +
+             round_up((size_t)kvq::kErrBins * kvq::kErrStride * 8);
   }
   g.len_region = round_up((size_t)max_batch * 4);
   g.partial_slots = partial_slots_for(max_batch, n_kv_heads);
@@ -93,7 +95,8 @@ bool make_geometry(const kvq_pair* map, int n_layers, int n_q_heads, int n_kv_he
   g.append_region = round_up((size_t)max_batch * 4);
   g.plan_region = round_up((size_t)max_batch * 4 * 4);
   g.err_region = round_up(4);
-  total += g.partial_region + g.merge_region + g.append_region + g.plan_region + g.err_region;
+  g.grid_region = round_up(4);
+  total += g.partial_region + g.merge_region + g.append_region + g.plan_region + g.err_region + g.grid_region;
   g.total = total;
   return true;
 }
@@ -102,6 +105,36 @@ kvq_status check_cache(const kvq_cache* c, int layer) {
   if (!c) return fail(KVQ_EINVAL, "cache is null");
   if (layer < 0 || layer >= c->n_layers) return fail(KVQ_EINVAL, "layer index out of range");
   return KVQ_OK;
+}
+
+// The layer the latest launch of this cache on `stream` wrote (-1: none; -2:
+// every layer, or unknown because the table of streams overflowed).
+int stream_written_layer(const kvq_cache* c, void* stream) {
+  for (const auto& w : c->stream_writes)
+    if (w.stream == stream) return w.layer;
+  return c->stream_table_full ? -2 : -1;
+}
+
+void note_stream_write(kvq_cache* c, void* stream, int layer) {
+  for (auto& w : c->stream_writes)
+    if (w.stream == stream) {
+      w.layer = layer;
+      return;
+    }
+  if (c->stream_writes.size() >= 64) {
+    c->stream_writes.clear();
+    c->stream_table_full = true;
+  }
+  c->stream_writes.push_back({stream, layer});
+}
+
+bool capturing(void* stream) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &st) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return st != cudaStreamCaptureStatusNone;
 }
 
 }  // namespace
@@ -237,7 +270,7 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     L.fp8_scales = reinterpret_cast<float*>(p);
     p += round_up((size_t)n_kv_heads * 2 * 4);
     L.err_stats = reinterpret_cast<double*>(p);
-    p += round_up(5 * 8);
+    p += round_up((size_t)kvq::kErrBins * kvq::kErrStride * 8);
     L.host_len.assign(max_batch, 0);
   }
   c->partials = reinterpret_cast<float*>(p);
@@ -250,6 +283,8 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
   p += g.plan_region;
   c->err = reinterpret_cast<int32_t*>(p);
   p += g.err_region;
+  c->grid_ctr = reinterpret_cast<int32_t*>(p);
+  p += g.grid_region;
 
   e = cudaMallocHost(&c->plan_host, (size_t)max_batch * 4 * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->plan_done, cudaEventDisableTiming);
@@ -259,11 +294,12 @@ kvq_status kvq_cache_create(const kvq_pair* map, int n_layers, int n_q_heads, in
     e = cudaMemset(c->layers[l].len, 0, (size_t)max_batch * 4);
     if (e == cudaSuccess)
       e = cudaMemcpy(c->layers[l].fp8_scales, ones.data(), ones.size() * 4, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemset(c->layers[l].err_stats, 0, 5 * 8);
+    if (e == cudaSuccess) e = cudaMemset(c->layers[l].err_stats, 0, (size_t)kvq::kErrBins * kvq::kErrStride * 8);
   }
   if (e == cudaSuccess) e = cudaMemset(c->merge_ctr, 0, (size_t)max_batch * n_kv_heads * 4);
   if (e == cudaSuccess) e = cudaMemset(c->append_ctr, 0, (size_t)max_batch * 4);
   if (e == cudaSuccess) e = cudaMemset(c->err, 0, 4);
+  if (e == cudaSuccess) e = cudaMemset(c->grid_ctr, 0, 4);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     kvq_status st = cuda_fail(e, "cache initialisation");
@@ -288,10 +324,11 @@ kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (auto& L : c->layers) {
     cudaError_t e = cudaMemsetAsync(L.len, 0, (size_t)c->max_batch * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(L.err_stats, 0, 5 * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.err_stats, 0, (size_t)kvq::kErrBins * kvq::kErrStride * 8, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     std::fill(L.host_len.begin(), L.host_len.end(), 0);
   }
+  note_stream_write(c, stream, -2);
   return KVQ_OK;
 }
 
@@ -299,10 +336,14 @@ kvq_status kvq_layer_error(const kvq_cache* c, int layer, kvq_error_stats* out) 
   kvq_status st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
   if (!out) return fail(KVQ_EINVAL, "out is null");
-  double h[5];
+  std::vector<double> bins((size_t)kvq::kErrBins * kvq::kErrStride);
   cudaError_t e = cudaDeviceSynchronize();
-  if (e == cudaSuccess) e = cudaMemcpy(h, c->layers[layer].err_stats, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(bins.data(), c->layers[layer].err_stats, bins.size() * 8, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error report)");
+  double h[5] = {0.0, 0.0, 0.0, 0.0, 0.0};
+  for (int b = 0; b < kvq::kErrBins; ++b)
+    for (int i = 0; i < 5; ++i) h[i] += bins[(size_t)b * kvq::kErrStride + i];
   out->k_sq_err = h[0];
   out->k_sq = h[1];
   out->v_sq_err = h[2];
@@ -415,6 +456,8 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
   cudaError_t e = kvq::launch_append(L.kb, L.vb, c->head_dim, dtype, p, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
   c->launches += 1;
+  note_stream_write(c, stream, layer);
+  if (capturing(stream)) c->graph_captured = true;
   for (int b = 0; b < batch; ++b) L.host_len[b] += n_new[b];
   return KVQ_OK;
 }
@@ -433,19 +476,18 @@ static bool choose_warp_split(const kvq_cache* c, int gqa, int batch, int64_t ma
   return t_warp < t_shared;
 }
 
-kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, float* out, void* stream) {
-  kvq_status st = check_cache(c, layer);
-  if (st != KVQ_OK) return st;
-  if (batch <= 0 || batch > c->max_batch) return fail(KVQ_EINVAL, "batch must be in [1, max_batch]");
-  if (!Q || !out) return fail(KVQ_EINVAL, "Q or out is null");
-  if (!aligned16(Q) || !aligned16(out)) return fail(KVQ_EINVAL, "Q and out must be 16-byte aligned");
+// Parameters of one decode launch of `layer` over sequences b < batch at the
+// host's lengths `lens` (before a fused step's append). Fails with a message
+// when the units exceed 32-bit indexing.
+static kvq_status decode_params(kvq_cache* c, int layer, const void* Q, int batch, float* out, void* stream,
+                                bool append, const std::vector<int64_t>& lens, kvq::DecodeParams& p) {
   const kvq::LayerState& L = c->layers[layer];
   int64_t total_pages = 0, max_p = 0, n_units = 0;
   for (int b = 0; b < batch; ++b) {
-    int64_t T = L.host_len[b], P = T / kvq::kPageTokens;
+    const int64_t P = lens[b] / kvq::kPageTokens;
     total_pages += P;
     max_p = std::max(max_p, P);
-    n_units += std::max<int64_t>(1, P + (T % kvq::kPageTokens ? 1 : 0)) + kvq::seg_overhead_units();
+    n_units += P + 1 + kvq::seg_overhead_units();
   }
   total_pages *= c->n_kv_heads;
   n_units *= c->n_kv_heads;
@@ -455,9 +497,8 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   int chunk = c->split_pages > 0 ? c->split_pages : kvq::choose_chunk(c->sm_count, total_pages, max_p, stride);
   // never more splits than the partial buffer holds
   chunk = (int)std::max<int64_t>(chunk, (max_p + stride - 1) / stride);
-  int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
 
-  kvq::DecodeParams p{};
+  p = kvq::DecodeParams{};
   p.pages = L.pages;
   p.window = L.window;
   p.len = L.len;
@@ -485,11 +526,50 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   p.key_mode = L.km;
   p.fmt = L.fmt;
   p.fp8_scales = L.fp8_scales;
-  p.warp_split = choose_warp_split(c, p.gqa, batch, max_p, total_pages) ? 1 : 0;
+  p.warp_split = choose_warp_split(c, p.gqa, batch, max_p + (append ? 1 : 0), total_pages) ? 1 : 0;
+  // The lengths travel in the parameters unless a captured graph may replay this
+  // launch (frozen parameters) or replays have moved the device lengths past the
+  // host's view. Then the page copies may start under the preceding kernel's
+  // tail, unless that kernel is one of ours that wrote this layer.
+  const bool capture = capturing(stream);
+  if (capture) c->graph_captured = true;
+  p.host_units = (!capture && !c->graph_captured && batch <= kvq::kHostLens) ? 1 : 0;
+  if (p.host_units) {
+    for (int b = 0; b < batch; ++b) p.hlen[b] = (int32_t)lens[b];
+    const int w = stream_written_layer(c, stream);
+    p.early = (w != layer && w != -2) ? 1 : 0;
+  }
+  if (append) {
+    p.append = 1;
+    p.step_pages = L.pages;
+    p.step_window = L.window;
+    p.step_len = L.len;
+    p.append_ctr = c->append_ctr;
+    p.grid_ctr = c->grid_ctr;
+    p.err_stats = L.err_stats;
+    p.max_tokens = (int)std::min<int64_t>(c->max_tokens, INT32_MAX);
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, float* out, void* stream) {
+  kvq_status st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (batch <= 0 || batch > c->max_batch) return fail(KVQ_EINVAL, "batch must be in [1, max_batch]");
+  if (!Q || !out) return fail(KVQ_EINVAL, "Q or out is null");
+  if (!aligned16(Q) || !aligned16(out)) return fail(KVQ_EINVAL, "Q and out must be 16-byte aligned");
+  const kvq::LayerState& L = c->layers[layer];
+  kvq::DecodeParams p;
+  st = decode_params(c, layer, Q, batch, out, stream, false, L.host_len, p);
+  if (st != KVQ_OK) return st;
+  int splits = 1;
+  for (int b = 0; b < batch; ++b)
+    splits = std::max<int>(splits, (int)((L.host_len[b] / kvq::kPageTokens + p.chunk - 1) / p.chunk));
   dim3 grid(splits, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_decode(L.kb, L.vb, c->head_dim, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   c->launches += 1;
+  note_stream_write(c, stream, -1);
   return KVQ_OK;
 }
 
@@ -502,57 +582,25 @@ kvq_status kvq_decode_step(kvq_cache* c, int layer, const void* K, const void* V
   if (!aligned16(K) || !aligned16(V) || !aligned16(Q) || !aligned16(out))
     return fail(KVQ_EINVAL, "K, V, Q and out must be 16-byte aligned");
   kvq::LayerState& L = c->layers[layer];
-  int64_t total_pages = 0, max_p = 0;
-  for (int b = 0; b < batch; ++b) {
+  for (int b = 0; b < batch; ++b)
     if (L.host_len[b] + 1 > c->max_tokens)
       return fail(KVQ_ECAPACITY, "append would exceed max_tokens for sequence " + std::to_string(b));
-    const int64_t P = (L.host_len[b] + 1) / kvq::kPageTokens;
-    total_pages += P;
-    max_p = std::max(max_p, P);
-  }
-  total_pages *= c->n_kv_heads;
-  const int gqa = c->n_q_heads / c->n_kv_heads;
-  auto two_launches = [&]() -> kvq_status {
+  if (kvq::decode_uses_simt()) {
+    // the CUDA-core decode kernel has no fused form: append, then attend
     std::vector<int32_t> ones((size_t)batch, 1);
-    kvq_status r = kvq_append(c, layer, K, V, KVQ_BF16, ones.data(), batch, stream);
-    return r != KVQ_OK ? r : kvq_decode_attn(c, layer, Q, batch, out, stream);
-  };
-  if (kvq::decode_uses_simt() || !choose_warp_split(c, gqa, batch, max_p, total_pages)) return two_launches();
-
-  kvq::DecodeParams p{};
-  p.pages = L.pages;
-  p.window = L.window;
-  p.len = L.len;
-  p.Q = static_cast<const __nv_bfloat16*>(Q);
-  p.out = out;
-  p.page_bytes = L.page_bytes;
-  p.max_pages = (int)c->max_pages;
-  p.n_kv_heads = c->n_kv_heads;
-  p.gqa = gqa;
-  p.batch = batch;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->head_dim));
-  p.err = c->err;
-  p.sm_count = c->sm_count;
-  p.key_mode = L.km;
-  p.fmt = L.fmt;
-  p.fp8_scales = L.fp8_scales;
-  p.warp_split = 1;
-  p.step_pages = L.pages;
-  p.step_window = L.window;
-  p.step_len = L.len;
-  p.append_ctr = c->append_ctr;
+    st = kvq_append(c, layer, K, V, KVQ_BF16, ones.data(), batch, stream);
+    return st != KVQ_OK ? st : kvq_decode_attn(c, layer, Q, batch, out, stream);
+  }
+  kvq::DecodeParams p;
+  st = decode_params(c, layer, Q, batch, out, stream, true, L.host_len, p);
+  if (st != KVQ_OK) return st;
   p.k_new = static_cast<const __nv_bfloat16*>(K);
   p.v_new = static_cast<const __nv_bfloat16*>(V);
-  p.err_stats = L.err_stats;
-  p.max_tokens = (int)std::min<int64_t>(c->max_tokens, INT32_MAX);
-  cudaError_t e = kvq::launch_decode_step(L.kb, L.vb, c->head_dim, p, static_cast<cudaStream_t>(stream));
-  if (e == cudaErrorNotSupported) {
-    cudaGetLastError();
-    return two_launches();
-  }
+  cudaError_t e = kvq::launch_decode_mma(L.kb, L.vb, c->head_dim, p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode step kernel launch");
   for (int b = 0; b < batch; ++b) L.host_len[b] += 1;
   c->launches += 1;
+  note_stream_write(c, stream, layer);
   return KVQ_OK;
 }
 
@@ -648,6 +696,7 @@ kvq_status kvq_refresh_lengths(kvq_cache* c) {
     for (int b = 0; b < c->max_batch; ++b) L.host_len[b] = tmp[b];
   }
   if (e != cudaSuccess) return cuda_fail(e, "kvq_refresh_lengths");
+  c->graph_captured = false;
   return KVQ_OK;
 }
 

@@ -13,7 +13,11 @@
 // Grid (items, n_kv_heads, batch), 128 threads. Work item i of (b, h) quantizes
 // group floor(T0/32) + i when that group completes during this call; item 0
 // also rewrites the window afterwards (it is the only item reading old window
-// tokens). With no completed group, item 0 only writes the window.
+// tokens). With no completed group, item 0 only writes the window. A flush
+// stages the group's 32 key and value rows in shared memory as bf16 (16-byte
+// vector loads), takes the quantizer parameters (a thread per key channel, a
+// warp per token), then quantizes every element as it is packed into the
+// fragment-ordered page.
 //
 // Quantizer (bit-exact contract with the CPU oracle; every fp32 step is a
 // single IEEE operation, the __f*_rn intrinsics are never contracted):
@@ -59,12 +63,34 @@ __device__ __forceinline__ __nv_bfloat16 load_in(const void* base, int64_t idx) 
   else return reinterpret_cast<const __nv_bfloat16*>(base)[idx];
 }
 
+// Eight consecutive input values as bf16 (a 16-byte vector; fp32 inputs are
+// rounded to nearest even). idx is a multiple of 8.
+template <bool F32IN>
+__device__ __forceinline__ uint4 load8(const void* base, int64_t idx) {
+  if constexpr (F32IN) {
+    const float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    const float4 y = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx + 4);
+    auto pack = [](float lo, float hi) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+      return *reinterpret_cast<const uint32_t*>(&b);
+    };
+    return make_uint4(pack(x.x, x.y), pack(x.z, x.w), pack(y.x, y.y), pack(y.z, y.w));
+  } else {
+    return *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+  }
+}
+
 template <int KB, int VB, int D, bool F32IN>
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
   pdl_enter();
   constexpr bool kBf16Layer = (KB == 16);
+  constexpr int RS = D + 8;          // bf16 row stride of the staged rows (16-byte rows, staggered banks)
+  constexpr int NP = D > 32 ? D : 32;
   const int b = blockIdx.z, h = blockIdx.y, item = blockIdx.x;
   const int H = a.n_kv_heads;
+  __shared__ __align__(16) __nv_bfloat16 xs[2][kPageTokens][RS];  // keys, values of the group
+  __shared__ float pz[2][NP], pr[2][NP], ps[2][NP];  // quantizer zero, reciprocal, scale: keys, values
+  __shared__ double red[kThreads / 32][4];
   __shared__ int s_T0;
   __nv_bfloat16 k_new, v_new;  // one-token mode: this thread's channel of the new row
 
@@ -117,46 +143,27 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
   if (ng > 0) {
     const int g = g0 + item;
     uint8_t* page = a.pages + ((int64_t)(b * H + h) * a.max_pages + g) * a.page_bytes;
+    // the group's 32 key and value rows, old window slots first, as 16-byte vectors
+    constexpr int VPR = D / 8;
+    for (int v = threadIdx.x; v < 2 * kPageTokens * VPR; v += kThreads) {
+      const int r = v / (kPageTokens * VPR), rem = v % (kPageTokens * VPR);
+      const int tk = rem / VPR, c8 = (rem % VPR) * 8;
+      const int tau = g * kPageTokens + tk;
+      uint4 x;
+      if (tau < T0) {
+        x = *reinterpret_cast<const uint4*>(win + (r * kPageTokens + (tau % kPageTokens)) * D + c8);
+      } else {
+        const int64_t row = off + (tau - T0);
+        x = load8<F32IN>(r ? a.V : a.K, (row * H + h) * D + c8);
+      }
+      *reinterpret_cast<uint4*>(&xs[r][tk][c8]) = x;
+    }
+    __syncthreads();
     if constexpr (kBf16Layer) {
-      __shared__ uint16_t sv[2][kPageTokens][D];
-      for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
-        int t = idx / D, d = idx % D;
-        int tau = g * kPageTokens + t;
-        __nv_bfloat16 kx, vx;
-        if (tau < T0) {
-          kx = win[(0 * kPageTokens + (tau % kPageTokens)) * D + d];
-          vx = win[(1 * kPageTokens + (tau % kPageTokens)) * D + d];
-        } else {
-          int64_t row = off + (tau - T0);
-          kx = load_in<F32IN>(a.K, (row * H + h) * D + d);
-          vx = load_in<F32IN>(a.V, (row * H + h) * D + d);
-        }
-        sv[0][t][d] = __bfloat16_as_ushort(kx);
-        sv[1][t][d] = __bfloat16_as_ushort(vx);
-      }
-      __syncthreads();
-      store_block<16, D>(page, false, [&](int tok, int dim) { return (uint32_t)sv[0][tok][dim]; });
+      store_block<16, D>(page, false, [&](int tok, int dim) { return (uint32_t)__bfloat16_as_ushort(xs[0][tok][dim]); });
       store_block<16, D>(page + code_block_bytes(16, D), true,
-                         [&](int tok, int dim) { return (uint32_t)sv[1][tok][dim]; });
+                         [&](int tok, int dim) { return (uint32_t)__bfloat16_as_ushort(xs[1][tok][dim]); });
     } else {
-      __shared__ float xs[2][kPageTokens][D + 1];
-      __shared__ uint8_t cs[2][kPageTokens][D];
-      for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
-        int t = idx / D, d = idx % D;
-        int tau = g * kPageTokens + t;
-        __nv_bfloat16 kx, vx;
-        if (tau < T0) {
-          kx = win[(0 * kPageTokens + (tau % kPageTokens)) * D + d];
-          vx = win[(1 * kPageTokens + (tau % kPageTokens)) * D + d];
-        } else {
-          int64_t row = off + (tau - T0);
-          kx = load_in<F32IN>(a.K, (row * H + h) * D + d);
-          vx = load_in<F32IN>(a.V, (row * H + h) * D + d);
-        }
-        xs[0][t][d] = __bfloat162float(kx);
-        xs[1][t][d] = __bfloat162float(vx);
-      }
-      __syncthreads();
       double err[4] = {0.0, 0.0, 0.0, 0.0};  // this thread's share of the error report
       auto add_err = [&](int r, float x, double xh) {
         const double dx = (double)x - xh;
@@ -165,19 +172,15 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
       };
       if (a.fmt != 0) {
         if constexpr (KB == 8 && VB == 8) {
-          const float ksc = a.fp8_scales[h], vsc = a.fp8_scales[H + h];
-          for (int idx = threadIdx.x; idx < kPageTokens * D; idx += kThreads) {
-            const int t = idx / D, d = idx % D;
-            const __nv_fp8_storage_t ck = __nv_cvt_float_to_fp8(__fdiv_rn(xs[0][t][d], ksc), __NV_SATFINITE, __NV_E4M3);
-            const __nv_fp8_storage_t cv = __nv_cvt_float_to_fp8(__fdiv_rn(xs[1][t][d], vsc), __NV_SATFINITE, __NV_E4M3);
-            cs[0][t][d] = (uint8_t)ck;
-            cs[1][t][d] = (uint8_t)cv;
-            add_err(0, xs[0][t][d], (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(ck, __NV_E4M3))) * ksc);
-            add_err(1, xs[1][t][d], (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(cv, __NV_E4M3))) * vsc);
-          }
-          __syncthreads();
-          store_block<8, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
-          store_block<8, D>(page + code_block_bytes(8, D), true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
+          const float sc[2] = {a.fp8_scales[h], a.fp8_scales[H + h]};
+          auto code = [&](int r, int tok, int dim) -> uint32_t {
+            const float x = __bfloat162float(xs[r][tok][dim]);
+            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(__fdiv_rn(x, sc[r]), __NV_SATFINITE, __NV_E4M3);
+            add_err(r, x, (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3))) * sc[r]);
+            return (uint32_t)c;
+          };
+          store_block<8, D>(page, false, [&](int tok, int dim) { return code(0, tok, dim); });
+          store_block<8, D>(page + code_block_bytes(8, D), true, [&](int tok, int dim) { return code(1, tok, dim); });
         }
       } else {
         const bool per_token_keys = a.key_mode != 0;
@@ -187,68 +190,72 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         __half* kzero = kscale + nk;
         __half* vscale = kzero + nk;
         __half* vzero = vscale + kPageTokens;
+        auto keep = [&](int r, int i, const QParams& q) {
+          pz[r][i] = q.z;
+          pr[r][i] = q.r;  // 0 for a constant set
+          ps[r][i] = __half2float(q.s_h);
+        };
         // one warp per token over the head dimension: row r of xs (0 keys, 1 values)
         auto quantize_tokens = [&](int r, int qmax, __half* sdst, __half* zdst) {
           const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
           for (int t = warp; t < kPageTokens; t += kThreads / 32) {
-            float mn = xs[r][t][lane], mx = mn;
-  #pragma unroll
+            float mn = __bfloat162float(xs[r][t][lane]), mx = mn;
+#pragma unroll
             for (int k = 1; k < D / 32; ++k) {
-              float x = xs[r][t][lane + 32 * k];
+              const float x = __bfloat162float(xs[r][t][lane + 32 * k]);
               mn = fminf(mn, x);
               mx = fmaxf(mx, x);
             }
-  #pragma unroll
+#pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
               mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
               mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             }
-            QParams q = make_qparams(mn, mx, qmax);
-            const double s = (double)__half2float(q.s_h), z = (double)q.z;
-  #pragma unroll
-            for (int k = 0; k < D / 32; ++k) {
-              const float x = xs[r][t][lane + 32 * k];
-              const uint32_t c = quant_code(x, q, qmax);
-              cs[r][t][lane + 32 * k] = (uint8_t)c;
-              add_err(r, x, (double)c * s + z);
-            }
             if (lane == 0) {
+              const QParams q = make_qparams(mn, mx, qmax);
               sdst[t] = q.s_h;
               zdst[t] = q.z_h;
+              keep(r, t, q);
             }
           }
         };
         if (per_token_keys) quantize_tokens(0, (1 << KB) - 1, kscale, kzero);
         // keys (per-channel mode): one thread per channel, over the group's 32 tokens
         for (int d = threadIdx.x; d < (per_token_keys ? 0 : D); d += kThreads) {
-          constexpr int qmax = (1 << KB) - 1;
-          float mn = xs[0][0][d], mx = mn;
-  #pragma unroll 8
+          float mn = __bfloat162float(xs[0][0][d]), mx = mn;
+#pragma unroll 8
           for (int t = 1; t < kPageTokens; ++t) {
-            float x = xs[0][t][d];
+            const float x = __bfloat162float(xs[0][t][d]);
             mn = fminf(mn, x);
             mx = fmaxf(mx, x);
           }
-          QParams q = make_qparams(mn, mx, qmax);
-          const double s = (double)__half2float(q.s_h), z = (double)q.z;
-  #pragma unroll 8
-          for (int t = 0; t < kPageTokens; ++t) {
-            const uint32_t c = quant_code(xs[0][t][d], q, qmax);
-            cs[0][t][d] = (uint8_t)c;
-            add_err(0, xs[0][t][d], (double)c * s + z);
-          }
-          int slot = kmeta_slot<D>(d);
+          const QParams q = make_qparams(mn, mx, (1 << KB) - 1);
+          const int slot = kmeta_slot<D>(d);
           kscale[slot] = q.s_h;
           kzero[slot] = q.z_h;
+          keep(0, d, q);
         }
-        // values: one warp per token, over the head dimension
         quantize_tokens(1, (1 << VB) - 1, vscale, vzero);
         __syncthreads();
-        store_block<KB, D>(page, false, [&](int tok, int dim) { return (uint32_t)cs[0][tok][dim]; });
-        store_block<VB, D>(vblk, true, [&](int tok, int dim) { return (uint32_t)cs[1][tok][dim]; });
+        // codes, each element quantized as it is packed, and its error report terms
+        auto code = [&](int r, int i, float x, int qmax) -> uint32_t {
+          QParams q;
+          q.z = pz[r][i];
+          q.r = pr[r][i];
+          q.zero_scale = (q.r == 0.0f);
+          const uint32_t c = quant_code(x, q, qmax);
+          add_err(r, x, (double)c * (double)ps[r][i] + (double)q.z);
+          return c;
+        };
+        store_block<KB, D>(page, false, [&](int tok, int dim) {
+          return code(0, per_token_keys ? tok : dim, __bfloat162float(xs[0][tok][dim]), (1 << KB) - 1);
+        });
+        store_block<VB, D>(vblk, true, [&](int tok, int dim) {
+          return code(1, tok, __bfloat162float(xs[1][tok][dim]), (1 << VB) - 1);
+        });
       }
-      // this flush's error sums: warp shuffles, then one fp64 atomic per sum
-      __shared__ double red[kThreads / 32][4];
+      // this flush's error sums: warp shuffles, then one fp64 atomic per sum into
+      // one of the layer's bins
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -258,13 +265,14 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         if (lane == 0) red[warp][i] = v;
       }
       __syncthreads();
-      if (a.err_stats && threadIdx.x < 4) {
+      double* bin = err_bin(a.err_stats, blockIdx.x + 131u * blockIdx.y + 8191u * blockIdx.z);
+      if (bin && threadIdx.x < 4) {
         double v = 0.0;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) v += red[w][threadIdx.x];
-        atomicAdd(&a.err_stats[threadIdx.x], v);
+        atomicAdd(&bin[threadIdx.x], v);
       }
-      if (a.err_stats && threadIdx.x == 4) atomicAdd(&a.err_stats[4], (double)(kPageTokens * D));
+      if (bin && threadIdx.x == 4) atomicAdd(&bin[4], (double)(kPageTokens * D));
     }
   }
 
@@ -280,13 +288,14 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         win[(1 * kPageTokens + slot) * D + threadIdx.x] = v_new;
       }
     } else {
-      for (int idx = threadIdx.x; idx < cnt * D; idx += kThreads) {
-        int i = idx / D, d = idx % D;
-        int tau = from + i;
-        int64_t row = off + (tau - T0);
-        int slot = tau % kPageTokens;
-        win[(0 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.K, (row * H + h) * D + d);
-        win[(1 * kPageTokens + slot) * D + d] = load_in<F32IN>(a.V, (row * H + h) * D + d);
+      constexpr int VPR = D / 8;
+      for (int v = threadIdx.x; v < cnt * VPR; v += kThreads) {
+        const int i = v / VPR, c8 = (v % VPR) * 8;
+        const int tau = from + i;
+        const int64_t row = off + (tau - T0);
+        const int slot = tau % kPageTokens;
+        *reinterpret_cast<uint4*>(win + (0 * kPageTokens + slot) * D + c8) = load8<F32IN>(a.K, (row * H + h) * D + c8);
+        *reinterpret_cast<uint4*>(win + (1 * kPageTokens + slot) * D + c8) = load8<F32IN>(a.V, (row * H + h) * D + c8);
       }
     }
   }

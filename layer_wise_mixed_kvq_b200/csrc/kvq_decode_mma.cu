@@ -5,34 +5,41 @@
 // FlashAttention-style kernels directly over the int8 / mixed-precision K and V
 // cache; "New GQA efficiency results": grouped-query attention. Keys are
 // dequantized per channel (x = code * s_c + z_c over each 32-token page) and
-// values per token (x = code * s_t + z_t).
+// values per token (x = code * s_t + z_t); "Computational cost": only the new
+// token is quantized online, which the fused decode step does in this kernel.
 //
 // Work splits, 4 warps per CTA, each warp streaming pages through a private
 // ring of shared-memory stages filled by bulk copies (cp.async.bulk, one copy
 // per page, mbarrier completion) with its own online-softmax state:
 //  * shared split (decode_mma_kernel): a persistent grid cuts all (sequence,
-//    KV head) segments' pages into balanced contiguous slices, one per CTA; the
-//    CTA's warps take a segment part's pages in turn, merge in shared memory,
+//    KV head) segments' units into balanced contiguous slices, one per CTA; the
+//    CTA's warps take a segment part's units in turn, merge in shared memory,
 //    and either write the output or leave a split record that the last CTA of
-//    the segment merges;
+//    the segment merges. A segment's units are: overhead units (no work), its
+//    tail unit (the bf16 window; in the fused step, the new token's append and
+//    then the window or the page that token completed), then its pages.
 //  * warp split (decode_warp_kernel, short sequences, G <= 4): each warp
-//    attends whole segments alone and writes their outputs; its fused form
-//    first appends the segment's new token (window slot, or a warp-level
-//    flush of the completed group into the next page).
+//    attends whole segments alone and writes their outputs.
 //
-// Per page (32 tokens), with MMA rows = query heads: row g holds the high f16
-// part of head g's operand and row g + 8 the low part (hi + lo carries ~22
-// bits), so any G <= 8 fits one 16-row tile and S = C[g] + C[g + 8].
-//   z-term : C_z = q_hi/lo x z (z broadcast over the 8 columns): sum_c q_c z_c.
-//   QK     : A = q' = q * s_c (hi/lo), B = key codes, accumulators seeded with C_z.
-//   softmax: online max / sum in the log2 domain (q carries log2(e)/sqrt(D)).
-//   PV     : A = p' = p * s_t (hi/lo, straight from the QK accumulators),
-//            B = value codes; sum_t p_t z_t is added per head at the end.
+// Per page (32 tokens), token rows (G <= 4): MMA rows are tokens (QK) and value
+// channels (PV); the 8 columns are (head c/2, part c%2), part 0 the high and
+// part 1 the low f16 half of the operand (hi + lo carries the operand exactly).
+//   QK : A = key codes, B = q'_c = q_c * s_c. q is a bf16 value scaled by a power
+//        of two into (-1, 1), so it is exact in f16, and s_c is the page's f16
+//        scale: hi = RN(q s) (HMUL2) and lo = q s - hi (HFMA2) are exact, i.e. the
+//        product is formed without rounding. The z term sum_c q_c z_c is one MMA
+//        per 16 channels (B = q on part-0 columns).
+//   softmax: online max / sum in the log2 domain, raised lazily (p <= 2^8).
+//   PV : A = value codes, B = p' = p * s_t * 2^E as (hi, lo) f16 pairs, moved from
+//        the score layout to the B layout by 8x8 transposes (movmatrix); E is a
+//        per-segment power of two that keeps p' in f16's normal range whatever
+//        the value scales are; sum_t p_t z_t is added per head at the end.
+// Head rows (G > 4) put (head, part) on the MMA rows and tokens on the columns.
 // Codes enter the tensor core as f16 *subnormals*: masking a packed word with
 // 0x000F000F (4-bit), 0x00030003 (2-bit) or byte-permuting with zero (8-bit)
 // yields the f16 pair (c_a * 2^-24, c_b * 2^-24) exactly, so unpacking costs one
 // logic op per two codes. Codes sitting higher in a word come out multiplied
-// by a power of two; those factors are folded, exactly, into q', p', the score
+// by a power of two; those factors are folded, exactly, into q, p', the score
 // scale and the output scale (see the sigma/tau constants below).
 // bf16 layers and the bf16 window use bf16 MMAs on the raw values.
 
@@ -52,7 +59,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr uint32_t kWaitLimit = 1u << 24;   // try_wait polls before a copy is declared lost
 constexpr float kTwo24 = 16777216.0f;         // codes are c * 2^-24 inside the MMA
 constexpr float kTau = 8.0f;                  // lazy rescale: p may grow to 2^kTau before a rescale
-constexpr float kScaleCapLazy = 255.0f;       // largest value scale for which p' = p * s <= 65504 at p <= 2^kTau
+constexpr int kNoExp = -1000;                 // value exponent not chosen yet (no nonzero value scale seen)
 
 // ------------------------------------------------------------ PTX helpers --
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -126,7 +133,6 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-
 __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -143,6 +149,29 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// f16x2 arithmetic, each half rounded to nearest (IEEE binary16).
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hneg2(uint32_t a) { return a ^ 0x80008000u; }
+
+// 8x8 transpose of 16-bit elements across the warp: lane l holds row l/4,
+// columns 2(l%4), 2(l%4)+1 before and after.
+__device__ __forceinline__ uint32_t movtrans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -162,6 +191,27 @@ __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uin
   hi = b2_bits(h);
   lo = b2_bits(__floats2bfloat162_rn(x0 - f.x, x1 - f.y));
 }
+
+// (hi, lo) of one value as one register: low half f16(x), high half f16(x - hi).
+__device__ __forceinline__ uint32_t pack_hl_f16(float x) {
+  const float h = __half2float(__float2half_rn(x));
+  return h2_bits(__floats2half2_rn(h, x - h));
+}
+
+__device__ __forceinline__ uint32_t pack_hl_bf16(float x) {
+  const float h = __bfloat162float(__float2bfloat16_rn(x));
+  return b2_bits(__floats2bfloat162_rn(h, x - h));
+}
+
+// hi (part 0) or lo (part 1) halves of (x0, x1) as one register.
+__device__ __forceinline__ uint32_t part_f16(float x0, float x1, float partf) {
+  __half2 h = __floats2half2_rn(x0, x1);
+  float2 f = __half22float2(h);
+  return h2_bits(__floats2half2_rn(fmaf(-partf, f.x, x0), fmaf(-partf, f.y, x1)));
+}
+
+// 2^k as a float, -126 <= k <= 127.
+__device__ __forceinline__ float exp2i(int k) { return __int_as_float((127 + k) << 23); }
 
 // 2^x on the MUFU unit (flushes results below 2^-126 to zero).
 __device__ __forceinline__ float ex2(float x) {
@@ -183,7 +233,7 @@ struct Cfg {
   static constexpr int MINB = 2;
   static constexpr int MINB_TOK = PB <= 5000 ? 3 : 2;
   // bytes of stages per warp: with 3 CTAs per SM, 3 x 4 warps x 14 KB; with 2, 2 x 4 x 20 KB, leaving
-  // room for the rest of a CTA's shared memory (about 20-30 KB) inside half an SM
+  // room for the rest of a CTA's shared memory inside its share of the SM
   static constexpr int RING_BUDGET = MINB_TOK == 3 ? 14336 : 20480;
   static constexpr int R = (RING_BUDGET / PB) < 2 ? 2 : ((RING_BUDGET / PB) > 4 ? 4 : (RING_BUDGET / PB));
   static constexpr int STAGE = (PB + 127) / 128 * 128;
@@ -196,37 +246,79 @@ struct Cfg {
   static constexpr float tauK = KB == 2 ? 16.f : 1.f;
   static constexpr float sigmaV = VB == 4 ? 16.f : (VB == 2 ? 4.f : 1.f);
   static constexpr float tauV = VB == 2 ? 16.f : 1.f;
-  // per-warp key-scale table: row t holds this lane's D/4 scales, rows padded by
-  // 4 floats so the four rows fall on different banks
-  static constexpr int KSROW = D / 4 + 4;
   // shared memory layout
   static constexpr int RING = kWarps * R * STAGE;
   static constexpr int MBAR_OFF = RING;
   static constexpr int MBAR_BYTES = ((kWarps * R + 2) * 8 + 127) / 128 * 128;  // + 2 query-row barriers
-  static constexpr int WSCR_FLOATS = 4 * KSROW + 64 + 160;  // key scales, value scales/zeros, p' transpose tile
+  // per-warp scratch: value scales and zeros, per-token key scales and zeros
+  // (4 x 32 floats), or a flush's quantizer parameters (2 D + 64 floats)
+  static constexpr int WSCR_FLOATS = 2 * D + 64 > 128 ? 2 * D + 64 : 128;
   static constexpr int WSCR_OFF = MBAR_OFF + MBAR_BYTES;
   static constexpr int WSCR_STRIDE = (WSCR_FLOATS * 4 + 127) / 128 * 128;
   static constexpr int QZ_OFF = WSCR_OFF + kWarps * WSCR_STRIDE;
-  static constexpr int QZ_BYTES = KS * 32 * 16;            // head rows: z-term q fragments
-  static constexpr int QBUF_BYTES = 2 * kMaxGqa * D * 2;   // 2 x [8][D] bf16 query rows (= QZ_BYTES)
-  // token rows have no z-term fragments in shared memory: their query rows take that place
+  static constexpr int QZ_BYTES = KS * 32 * 16;            // head rows: query operand table
+  static constexpr int QBUF_BYTES = 2 * kMaxGqa * D * 2;   // 2 x [8][D] bf16 query rows
   static constexpr int qbuf_off(bool tok) { return tok ? QZ_OFF : QZ_OFF + QZ_BYTES; }
   static constexpr int merge_off(bool tok) { return qbuf_off(tok) + QBUF_BYTES; }
-  // then: merge area [kWarps][G][D] + m, l [kWarps][8] floats, unit starts [batch + 1] ints
+  // then: merge area [kWarps][G][D] + m, l [kWarps][8] floats, unit starts [batch + 1] and
+  // lengths [batch] ints
   static int smem_bytes(bool tok, int G, int batch) {
-    return merge_off(tok) + (kWarps * G * D + 2 * kWarps * kMaxGqa) * 4 + (batch + 1) * 4;
+    return merge_off(tok) + (kWarps * G * D + 2 * kWarps * kMaxGqa) * 4 + (2 * batch + 1) * 4;
   }
   static_assert(PB % 16 == 0, "bulk copies need 16-byte multiples");
 };
 
-// Per-warp running state for the G heads (lane (g, t) owns head g).
-template <int D>
-struct WarpState {
-  float o[D / 8][4];   // PV accumulators: [n-tile][c0..c3], rows g (hi) and g+8 (lo)
-  float m;             // reference max (log2 domain), identical across the quad
+// Running state of one warp. Head rows: lane (g, t) owns head g, o[n-tile] with
+// rows g (hi) and g + 8 (lo). Token rows: lane (g, t) owns head t's scores and
+// o[channel tile] (c0/c1: channel g, parts; c2/c3: channel g + 8).
+template <int NT>
+struct State {
+  float o[NT][4];
+  float m;             // reference max (log2 domain)
   float l;             // partial sum over this lane's tokens
   float vz;            // partial sum_t p_t z_t over this lane's tokens
+  int E;               // integer pages: o is kept in units of 2^-E (p' = p * s * 2^E), kNoExp before
 };
+template <int D> using WarpState = State<D / 8>;
+template <int D> using TokState = State<D / 16>;
+
+template <int NT>
+__device__ __forceinline__ void state_init(State<NT>& st) {
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) st.o[j][k] = 0.f;
+  st.m = -INFINITY;
+  st.l = 0.f;
+  st.vz = 0.f;
+  st.E = kNoExp;
+}
+
+// Value-operand exponent for one integer page whose value scales (lane = token)
+// are vs: p' = p * s_t * 2^E stays below 2^15 (p <= 2^kTau) and, for the page's
+// largest scale, above 2^6, so the (hi, lo) f16 pair keeps p' to ~22 bits even
+// when every scale is far below f16's normal range. E changes (and o is rescaled
+// exactly by the power of two) only when the page needs a smaller E or could
+// use one larger by more than 8. Warp-uniform. Returns 2^E.
+template <int NT>
+__device__ __forceinline__ float value_exponent(State<NT>& st, float vs) {
+  const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(vs));  // vs >= 0: bit order = value order
+  if (mb != 0u) {
+    const int e = (int)(mb >> 23) - 127;   // largest scale in [2^e, 2^(e+1)); fp16 scales: -24 <= e <= 15
+    const int want = 6 - e;                // 2^8 * 2^(e+1) * 2^want = 2^15
+    if (st.E == kNoExp) {
+      st.E = want;
+    } else if (want < st.E || want > st.E + 8) {
+      const float f = exp2i(want - st.E);
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st.o[j][k] *= f;
+      st.E = want;
+    }
+  }
+  return exp2i(st.E == kNoExp ? 0 : st.E);
+}
 
 // ------------------------------------------------------ B fragments of codes --
 // Words of one 16-channel tile row dt of a code block for this lane: tiles
@@ -289,6 +381,36 @@ __device__ __forceinline__ void tile_frags(const uint32_t (&w)[TileWords<BITS>::
   }
 }
 
+// A fragment of tile (dt, tt) from this lane's words (rows: tokens for keys,
+// channels for values; columns: channels for keys, tokens for values).
+template <int BITS>
+__device__ __forceinline__ void tile_afrag(const uint32_t (&w)[TileWords<BITS>::N], int tt, uint32_t (&a)[4]) {
+  if constexpr (BITS == 4) {
+    uint32_t x = w[tt], y = x >> 8;
+    a[0] = x & 0x000F000Fu;   // rows g,   cols 2t..     x1
+    a[1] = x & 0x00F000F0u;   // rows g+8, cols 2t..     x16
+    a[2] = y & 0x000F000Fu;   // rows g,   cols 2t+8..   x1
+    a[3] = y & 0x00F000F0u;   // rows g+8, cols 2t+8..   x16
+  } else if constexpr (BITS == 2) {
+    uint32_t x = tt ? (w[0] >> 8) : w[0];
+    a[0] = x & 0x00030003u;   // x1
+    a[1] = x & 0x000C000Cu;   // x4
+    a[2] = x & 0x00300030u;   // x16
+    a[3] = x & 0x00C000C0u;   // x64
+  } else if constexpr (BITS == 8) {
+    uint32_t x = w[2 * tt], y = w[2 * tt + 1];
+    a[0] = __byte_perm(x, 0u, 0x4140);
+    a[1] = __byte_perm(x, 0u, 0x4342);
+    a[2] = __byte_perm(y, 0u, 0x4140);
+    a[3] = __byte_perm(y, 0u, 0x4342);
+  } else {
+    a[0] = w[4 * tt + 0];
+    a[1] = w[4 * tt + 1];
+    a[2] = w[4 * tt + 2];
+    a[3] = w[4 * tt + 3];
+  }
+}
+
 // Two e4m3 bytes of x (bytes 0, 1 for kSelLo; 2, 3 for kSelHi) -> f16x2 whose
 // values are the e4m3 values times 2^-8, exactly. prmt puts each byte in the
 // low half of a 16-bit lane with its sign replicated into the high byte; a
@@ -324,16 +446,16 @@ __device__ __forceinline__ void tile_frags_f8(const uint32_t (&w)[TileWords<8>::
   b[3] = e4m3x2_f16x2(y, kSelHi);
 }
 
-// Online-softmax update with this page's scores sc[8] (log2 domain; tokens
-// 8j + 2t + {0,1} for n-tile j = i/2; masked tokens are -inf). The reference
-// max is raised only when a score exceeds it by more than tau, so p <= 2^tau.
-// Returns p in sc.
+// ---------------------------------------------------------- online softmax --
+// Head rows: scores sc[8] (log2 domain; tokens 8j + 2t + {0,1} for n-tile
+// j = i/2; masked tokens are -inf). The reference max is raised only when a
+// score exceeds it by more than kTau, so p <= 2^kTau. Returns p in sc.
 template <int D>
-__device__ __forceinline__ void softmax_update(WarpState<D>& st, float (&sc)[8], float tau) {
+__device__ __forceinline__ void softmax_update(WarpState<D>& st, float (&sc)[8]) {
   float mx = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])), fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  if (mx > st.m + tau) {
+  if (mx > st.m + kTau) {
     const float alpha = ex2(st.m - mx);  // 0 when st.m = -inf
 #pragma unroll
     for (int j = 0; j < D / 8; ++j)
@@ -353,11 +475,194 @@ __device__ __forceinline__ void softmax_update(WarpState<D>& st, float (&sc)[8],
   st.l += sum;
 }
 
-// ------------------------------------------------------------ page kernels --
-// One full quantized page in shared memory -> state.
+// Token rows: scores sc[4] of head t for tokens g + 8i.
+template <int D>
+__device__ __forceinline__ void tok_softmax_update(TokState<D>& st, float (&sc)[4]) {
+  float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+  if (mx > st.m + kTau) {
+    const float alpha = ex2(st.m - mx);
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st.o[j][k] *= alpha;
+    st.l *= alpha;
+    st.vz *= alpha;
+    st.m = mx;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sc[i] = ex2(sc[i] - st.m);
+    st.l += sc[i];
+  }
+}
+
+// ----------------------------------------------------------- query operands --
+// Power of two k with max |q| * 2^-k < 1 over the warp's query values (bits:
+// this lane's largest |q| as float bits); q * 2^-k then fits f16 exactly and
+// q * 2^-k * s (s <= 65504) cannot overflow it.
+__device__ __forceinline__ int query_shift(float amax) {
+  const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+  if (mb == 0u) return 0;
+  const int k = (int)(mb >> 23) - 126;
+  return k < -100 ? -100 : (k > 100 ? 100 : k);
+}
+
+// Token rows: query operands of one segment for lane (g, t), column g = (head
+// g/2, part g%2).
+template <int D>
+struct TokOps {
+  // integer per-channel keys: q * 2^-k as f16 pairs of head g/2, channels
+  // 16dt + 2t (+1) and 16dt + 2t + 8 (+9), the second pair / tauK;
+  // integer per-token keys: the QK B fragments (that q on part-0 columns, 0 on
+  // part 1); fp8: the QK B fragments (q * key scale * log2(e)/sqrt(D), parts)
+  uint32_t q2[D / 8];
+  uint32_t qz[D / 8];   // integer per-channel keys: z-term B fragments (q * 2^-k on part-0 columns)
+  uint32_t npart;       // f16x2 0 (part 0) or -1 (part 1)
+  float fs0, fs1;       // QK accumulator -> score (log2 units) for n-tiles of parity 0 / 1
+  float lsc;            // log2(e)/sqrt(D) * 2^k
+  float qsum;           // per-token keys: sum_c q_c * 2^-k of the head this lane scores
+};
+
+template <int KB, int D, bool PT, bool F8>
+__device__ __forceinline__ void prep_tok_ops(TokOps<D>& ops, const __nv_bfloat16* qrow, bool qvalid, int lane,
+                                             float L, float ksc) {
+  using C = Cfg<KB, 4, D>;
+  constexpr int KS = D / 16;
+  const int g = lane >> 2, t = lane & 3;
+  const bool part0 = (g & 1) == 0;
+  float2 lo[KS], hi[KS];
+  float amax = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t a = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
+    uint32_t b = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
+    if (!qvalid) a = b = 0u;
+    lo[dt] = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&a));
+    hi[dt] = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&b));
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(lo[dt].x), fabsf(lo[dt].y)), fmaxf(fabsf(hi[dt].x), fabsf(hi[dt].y))));
+  }
+  if constexpr (F8) {
+    const float f = L * ksc, partf = part0 ? 0.f : 1.f;
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      ops.q2[2 * dt] = part_f16(lo[dt].x * f, lo[dt].y * f, partf);
+      ops.q2[2 * dt + 1] = part_f16(hi[dt].x * f, hi[dt].y * f, partf);
+    }
+    ops.fs0 = ops.fs1 = kF8Unit;
+    return;
+  } else {
+    const int k = query_shift(amax);
+    const float down = exp2i(-k), lp = L * exp2i(k);
+    const float fold = down / C::tauK;
+    float qs = 0.f;
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const uint32_t ql = h2_bits(__floats2half2_rn(lo[dt].x * down, lo[dt].y * down));
+      const uint32_t qh = h2_bits(__floats2half2_rn(hi[dt].x * down, hi[dt].y * down));
+      const uint32_t qf = C::tauK != 1.f ? h2_bits(__floats2half2_rn(hi[dt].x * fold, hi[dt].y * fold)) : qh;
+      qs += (lo[dt].x + lo[dt].y) + (hi[dt].x + hi[dt].y);
+      if constexpr (PT) {
+        ops.q2[2 * dt] = part0 ? ql : 0u;
+        ops.q2[2 * dt + 1] = part0 ? qf : 0u;
+      } else {
+        ops.q2[2 * dt] = ql;
+        ops.q2[2 * dt + 1] = qf;
+        ops.qz[2 * dt] = part0 ? ql : 0u;
+        ops.qz[2 * dt + 1] = part0 ? qh : 0u;
+      }
+    }
+    ops.npart = part0 ? 0u : 0xBC00BC00u;
+    ops.lsc = lp;
+    ops.fs0 = kTwo24 * lp;
+    ops.fs1 = kTwo24 / C::sigmaK * lp;
+    if constexpr (PT) {
+      // head g/2's sum over its D channels (the quad holds them), then head t's
+      qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+      ops.qsum = __shfl_sync(0xffffffffu, qs, 8 * t) * down;
+    }
+  }
+}
+
+// Raw bf16 pairs of q for the bf16 pages and the window (token rows: q on
+// part-0 columns, 0 on part 1; head rows: row g).
+template <int D>
+__device__ __forceinline__ void load_qb(const __nv_bfloat16* qrow, bool keep, int t, uint32_t (&qb)[D / 8]) {
+#pragma unroll
+  for (int dt = 0; dt < D / 16; ++dt) {
+    qb[2 * dt] = keep ? *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t) : 0u;
+    qb[2 * dt + 1] = keep ? *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8) : 0u;
+  }
+}
+
+// ------------------------------------------------------- token-row pages --
+// p' of this lane (head t, tokens g + 8i) -> the PV B fragments. r[i] packs
+// (hi, lo) of token g + 8i: block i of the [token][(head, part)] matrix in the
+// C-fragment layout; an 8x8 transpose turns blocks 2ks, 2ks+1 into the B
+// fragment of k-step ks (tokens 16ks + 2t, +1 and 16ks + 8 + 2t, +1; column g).
+template <bool BF16>
+__device__ __forceinline__ void tok_pv_frags(const float (&pv)[4], uint32_t (&b)[2][2]) {
+  uint32_t r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r[i] = BF16 ? pack_hl_bf16(pv[i]) : pack_hl_f16(pv[i]);
+  b[0][0] = movtrans(r[0]);
+  b[0][1] = movtrans(r[1]);
+  b[1][0] = movtrans(r[2]);
+  b[1][1] = movtrans(r[3]);
+}
+
+// PV of one integer / fp8 / bf16 value block with the B fragments above.
+template <int VB, int D, bool F8>
+__device__ __forceinline__ void tok_pv(const uint8_t* vblk, TokState<D>& st, const uint32_t (&b)[2][2], int lane) {
+#pragma unroll
+  for (int dt = 0; dt < D / 16; ++dt) {
+    uint32_t w[TileWords<VB>::N];
+    load_tile_words<VB>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a[4];
+      if constexpr (F8) tile_afrag_f8(w, ks, a);
+      else tile_afrag<VB>(w, ks, a);
+      if constexpr (VB == 16) mma_bf16(st.o[dt], a[0], a[1], a[2], a[3], b[ks][0], b[ks][1]);
+      else mma_f16(st.o[dt], a[0], a[1], a[2], a[3], b[ks][0], b[ks][1]);
+    }
+  }
+}
+
+// Value scales (x 2^E, tauV folded) and zeros of an integer page into the warp's tables.
+template <int VB, int NT>
+__device__ __forceinline__ void value_tables(const __half* vscale, const __half* vzero, State<NT>& st, float* svf,
+                                             float* zvf, int lane) {
+  constexpr float tauV = VB == 2 ? 16.f : 1.f;
+  const float vs = __half2float(vscale[lane]);
+  const float f = value_exponent(st, vs);
+  svf[lane] = vs * ((tauV != 1.f && (lane & 8)) ? f * (1.f / tauV) : f);
+  zvf[lane] = __half2float(vzero[lane]);
+}
+
+// p' = p * s_t * 2^E and the value zero term, then PV.
+template <int VB, int D>
+__device__ __forceinline__ void tok_int_pv(const uint8_t* vblk, TokState<D>& st, float (&sc)[4], const float* svf,
+                                           const float* zvf, int lane) {
+  const int g = lane >> 2;
+  float pv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pv[i] = sc[i] * svf[g + 8 * i];
+    st.vz = fmaf(sc[i], zvf[g + 8 * i], st.vz);
+  }
+  uint32_t b[2][2];
+  tok_pv_frags<false>(pv, b);
+  tok_pv<VB, D, false>(vblk, st, b, lane);
+}
+
+// Integer page, per-channel keys.
 template <int KB, int VB, int D>
-__device__ __forceinline__ void attend_qpage(const uint8_t* page, WarpState<D>& st, const float (&qf)[D / 4],
-                                             const uint32_t* qz, float* wscr, int lane) {
+__device__ __forceinline__ void attend_qpage_tok(const uint8_t* page, TokState<D>& st, const TokOps<D>& ops,
+                                                 float* wscr, int lane) {
   using C = Cfg<KB, VB, D>;
   const int t = lane & 3;
   const uint8_t* vblk = page + code_block_bytes(KB, D);
@@ -365,73 +670,299 @@ __device__ __forceinline__ void attend_qpage(const uint8_t* page, WarpState<D>& 
   const __half* kzero = kscale + D;
   const __half* vscale = kzero + D;
   const __half* vzero = vscale + kPageTokens;
-  float* ksf = wscr;                   // [4][KSROW] key scales by lane row t, tauK folded
-  float* svf = wscr + 4 * C::KSROW;    // [32] value scales, tauV folded
-  float* zvf = svf + kPageTokens;      // [32] value zeros
-
-  // --- scale tables in fp32, converted cooperatively by the warp
-  {
-    constexpr int NE = D / 32;         // entries per lane, all in one row
-    const int i0 = lane * NE;
-    float* dst = ksf + (i0 / (D / 4)) * C::KSROW + (i0 % (D / 4));
-    if constexpr (NE == 4) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(kscale + i0);
-      float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      if (C::tauK != 1.f) { c.x *= 1.f / C::tauK; c.y *= 1.f / C::tauK; }  // entries j = 2, 3
-      *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, c.x, c.y);
-    } else {
-      const uint32_t raw = *reinterpret_cast<const uint32_t*>(kscale + i0);
-      float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw));
-      if (C::tauK != 1.f && (i0 & 2)) { a.x *= 1.f / C::tauK; a.y *= 1.f / C::tauK; }
-      *reinterpret_cast<float2*>(dst) = a;
-    }
-  }
-  const float vs = __half2float(vscale[lane]);
-  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
-  zvf[lane] = __half2float(vzero[lane]);
-  // lazy rescaling keeps p <= 2^kTau; p' = p * s must stay inside f16
-  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
+  float* svf = wscr;
+  float* zvf = wscr + kPageTokens;
+  value_tables<VB>(vscale, vzero, st, svf, zvf, lane);
   __syncwarp();
 
-  // --- QK (A = q' hi/lo, B = key codes) and the z-term (A = q hi/lo, B = z)
-  float s4[4][4], cz[4] = {0.f, 0.f, 0.f, 0.f};
+  // QK: two token m-tiles, B = exact (hi, lo) of q * s_c; z term: A = z rows, B = q
+  float s2[2][4], cz[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) s4[j][k] = 0.f;
-  const float* ksl = ksf + t * C::KSROW;
-  const uint32_t* zrow = reinterpret_cast<const uint32_t*>(kzero + t * (D / 4));
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+  const uint2* srow = reinterpret_cast<const uint2*>(kscale + t * (D / 4));   // channels 2t, 2t+1, 2t+8, 2t+9 per tile
+  const uint2* zrow = reinterpret_cast<const uint2*>(kzero + t * (D / 4));
 #pragma unroll
   for (int dt = 0; dt < C::KS; ++dt) {
     uint32_t w[TileWords<KB>::N];
     load_tile_words<KB>(page, lane, dt, w);
-    const float4 sc4 = *reinterpret_cast<const float4*>(ksl + dt * 4);
-    uint32_t ah0, al0, ah1, al1;
-    split_f16(qf[dt * 4 + 0] * sc4.x, qf[dt * 4 + 1] * sc4.y, ah0, al0);
-    split_f16(qf[dt * 4 + 2] * sc4.z, qf[dt * 4 + 3] * sc4.w, ah1, al1);
+    const uint2 s = srow[dt];
+    const uint32_t h0 = hmul2(ops.q2[2 * dt], s.x), h1 = hmul2(ops.q2[2 * dt + 1], s.y);
+    const uint32_t b0 = hfma2(ops.q2[2 * dt], s.x, hmul2(h0, ops.npart));
+    const uint32_t b1 = hfma2(ops.q2[2 * dt + 1], s.y, hmul2(h1, ops.npart));
 #pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-      uint32_t b[4];
-      tile_frags<KB>(w, tt, b);
-      mma_f16(s4[2 * tt], ah0, al0, ah1, al1, b[0], b[1]);
-      mma_f16(s4[2 * tt + 1], ah0, al0, ah1, al1, b[2], b[3]);
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag<KB>(w, mt, a);
+      mma_f16(s2[mt], a[0], a[1], a[2], a[3], b0, b1);
     }
-    const uint4 a = *reinterpret_cast<const uint4*>(qz + (dt * 32 + lane) * 4);
-    const uint2 z = *reinterpret_cast<const uint2*>(zrow + dt * 2);
-    mma_f16(cz, a.x, a.y, a.z, a.w, z.x, z.y);
+    const uint2 z = zrow[dt];
+    mma_f16(cz, z.x, z.x, z.y, z.y, ops.qz[2 * dt], ops.qz[2 * dt + 1]);
   }
-  const float czv = cz[0] + cz[2];  // every column holds the same sum
-  float sc[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float f = (j & 1) ? kTwo24 / C::sigmaK : kTwo24;
-    sc[2 * j] = fmaf(s4[j][0] + s4[j][2], f, czv);
-    sc[2 * j + 1] = fmaf(s4[j][1] + s4[j][3], f, czv);
-  }
-  softmax_update<D>(st, sc, tau);
+  const float czv = (cz[0] + cz[1]) * ops.lsc;  // head t: sum_c q_c z_c
+  float sc[4];
+  sc[0] = fmaf(s2[0][0] + s2[0][1], ops.fs0, czv);
+  sc[1] = fmaf(s2[0][2] + s2[0][3], ops.fs1, czv);
+  sc[2] = fmaf(s2[1][0] + s2[1][1], ops.fs0, czv);
+  sc[3] = fmaf(s2[1][2] + s2[1][3], ops.fs1, czv);
+  tok_softmax_update<D>(st, sc);
+  tok_int_pv<VB, D>(vblk, st, sc, svf, zvf, lane);
+}
 
-  // --- PV: A = p' (hi/lo) per 16-token k-step, B = value codes
+// Integer page, per-token keys: B = the segment's q (fixed); score of token
+// g + 8i for head t = (s_tok * acc + z_tok * sum_c q_c) * log2(e)/sqrt(D) * 2^k.
+template <int KB, int VB, int D>
+__device__ __forceinline__ void attend_qpage_tok_pt(const uint8_t* page, TokState<D>& st, const TokOps<D>& ops,
+                                                    float* wscr, int lane) {
+  using C = Cfg<KB, VB, D, true>;
+  const int g = lane >> 2;
+  const uint8_t* vblk = page + code_block_bytes(KB, D);
+  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
+  const __half* kzero = kscale + kPageTokens;
+  const __half* vscale = kzero + kPageTokens;
+  const __half* vzero = vscale + kPageTokens;
+  float* svf = wscr;
+  float* zvf = wscr + kPageTokens;
+  float* kst = wscr + 2 * kPageTokens;
+  float* kzt = wscr + 3 * kPageTokens;
+  kst[lane] = __half2float(kscale[lane]) * ((lane & 8) ? ops.fs1 : ops.fs0);
+  kzt[lane] = __half2float(kzero[lane]) * ops.lsc;
+  value_tables<VB>(vscale, vzero, st, svf, zvf, lane);
+  __syncwarp();
+
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<KB>::N];
+    load_tile_words<KB>(page, lane, dt, w);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag<KB>(w, mt, a);
+      mma_f16(s2[mt], a[0], a[1], a[2], a[3], ops.q2[2 * dt], ops.q2[2 * dt + 1]);
+    }
+  }
+  float sc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int tok = g + 8 * i;
+    const float acc = s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1];
+    sc[i] = fmaf(acc, kst[tok], kzt[tok] * ops.qsum);
+  }
+  tok_softmax_update<D>(st, sc);
+  tok_int_pv<VB, D>(vblk, st, sc, svf, zvf, lane);
+}
+
+// fp8 page: A = e4m3 keys/values as f16, B = the segment's q' parts (key scale
+// folded in) or p parts.
+template <int D>
+__device__ __forceinline__ void attend_f8page_tok(const uint8_t* page, TokState<D>& st, const TokOps<D>& ops,
+                                                  int lane) {
+  constexpr int KS = D / 16;
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<8>::N];
+    load_tile_words<8>(page, lane, dt, w);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag_f8(w, mt, a);
+      mma_f16(s2[mt], a[0], a[1], a[2], a[3], ops.q2[2 * dt], ops.q2[2 * dt + 1]);
+    }
+  }
+  float sc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sc[i] = (s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1]) * kF8Unit;
+  tok_softmax_update<D>(st, sc);
+  uint32_t b[2][2];
+  tok_pv_frags<false>(sc, b);
+  tok_pv<8, D, true>(page + code_block_bytes(8, D), st, b, lane);
+}
+
+template <int D>
+__device__ __forceinline__ void attend_bpage_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qbp)[D / 8],
+                                                 float scale_log2, int lane) {
+  constexpr int KS = D / 16;
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t w[TileWords<16>::N];
+    load_tile_words<16>(page, lane, dt, w);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      uint32_t a[4];
+      tile_afrag<16>(w, mt, a);
+      mma_bf16(s2[mt], a[0], a[1], a[2], a[3], qbp[2 * dt], qbp[2 * dt + 1]);
+    }
+  }
+  float sc[4] = {(s2[0][0] + s2[0][1]) * scale_log2, (s2[0][2] + s2[0][3]) * scale_log2,
+                 (s2[1][0] + s2[1][1]) * scale_log2, (s2[1][2] + s2[1][3]) * scale_log2};
+  tok_softmax_update<D>(st, sc);
+  uint32_t b[2][2];
+  tok_pv_frags<true>(sc, b);
+  tok_pv<16, D, false>(page + code_block_bytes(16, D), st, b, lane);
+}
+
+// bf16 window (natural [32][D] rows in global memory), W < 32 valid tokens.
+template <int D>
+__device__ __forceinline__ void attend_window_tok(const __nv_bfloat16* win, int W, TokState<D>& st,
+                                                  const uint32_t (&qbp)[D / 8], float scale_log2, int lane) {
+  constexpr int KS = D / 16;
+  const int g = lane >> 2, t = lane & 3;
+  const uint16_t* kw = reinterpret_cast<const uint16_t*>(win);
+  const uint16_t* vw = kw + kPageTokens * D;
+  auto kpair = [&](int tok, int dim) -> uint32_t {
+    return tok < W ? *reinterpret_cast<const uint32_t*>(kw + tok * D + dim) : 0u;
+  };
+  auto vpair = [&](int tok, int dim) -> uint32_t {
+    const uint32_t lo = tok < W ? vw[tok * D + dim] : 0u;
+    const uint32_t hi = tok + 1 < W ? vw[(tok + 1) * D + dim] : 0u;
+    return lo | (hi << 16);
+  };
+  float s2[2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    if (16 * mt >= W) continue;  // warp-uniform
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int r0 = 16 * mt + g, c0 = 16 * dt + 2 * t;
+      mma_bf16(s2[mt], kpair(r0, c0), kpair(r0 + 8, c0), kpair(r0, c0 + 8), kpair(r0 + 8, c0 + 8), qbp[2 * dt],
+               qbp[2 * dt + 1]);
+    }
+  }
+  float sc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float v = (i & 1) ? (s2[i >> 1][2] + s2[i >> 1][3]) : (s2[i >> 1][0] + s2[i >> 1][1]);
+    sc[i] = (g + 8 * i) < W ? v * scale_log2 : -INFINITY;
+  }
+  tok_softmax_update<D>(st, sc);
+  uint32_t b[2][2];
+  tok_pv_frags<true>(sc, b);
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    if (16 * ks >= W) continue;  // warp-uniform
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int tk = 16 * ks + 2 * t, ch = 16 * dt + g;
+      mma_bf16(st.o[dt], vpair(tk, ch), vpair(tk, ch + 8), vpair(tk + 8, ch), vpair(tk + 8, ch + 8), b[ks][0],
+               b[ks][1]);
+    }
+  }
+}
+
+// -------------------------------------------------------- head-row pages --
+// Query operand table of a segment in shared memory, built by one warp: entry
+// (dt, lane) for head g, channels 16dt + 2t (+1) and + 8 (+9):
+//   integer per-channel keys: {q01, q89 / tauK, q01, q89} (q * 2^-k as f16 pairs;
+//     the first two are the QK A operand, the last two the z-term A operand);
+//   integer per-token keys: {q01, q89 / tauK, -, -};
+//   fp8: {hi01, lo01, hi89, lo89} of q * key scale * log2(e)/sqrt(D).
+struct HeadOps {
+  float fs0, fs1, lsc, qsum;
+};
+
+template <int KB, int D, bool PT, bool F8>
+__device__ __forceinline__ void prep_head_ops(HeadOps& ops, uint32_t* qtab, bool write_tab, const __nv_bfloat16* qrow,
+                                              bool qvalid, int lane, float L, float ksc) {
+  using C = Cfg<KB, 4, D>;
+  constexpr int KS = D / 16;
+  const int t = lane & 3;
+  float2 lo[KS], hi[KS];
+  float amax = 0.f;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t a = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
+    uint32_t b = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
+    if (!qvalid) a = b = 0u;
+    lo[dt] = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&a));
+    hi[dt] = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&b));
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(lo[dt].x), fabsf(lo[dt].y)), fmaxf(fabsf(hi[dt].x), fabsf(hi[dt].y))));
+  }
+  if constexpr (F8) {
+    const float f = L * ksc;
+    if (write_tab) {
+#pragma unroll
+      for (int dt = 0; dt < KS; ++dt) {
+        uint4 q4;
+        split_f16(lo[dt].x * f, lo[dt].y * f, q4.x, q4.y);
+        split_f16(hi[dt].x * f, hi[dt].y * f, q4.z, q4.w);
+        *reinterpret_cast<uint4*>(qtab + (dt * 32 + lane) * 4) = q4;
+      }
+    }
+    ops.fs0 = ops.fs1 = kF8Unit;
+  } else {
+    const int k = query_shift(amax);
+    const float down = exp2i(-k), lp = L * exp2i(k);
+    const float fold = down / C::tauK;
+    float qs = 0.f;
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      qs += (lo[dt].x + lo[dt].y) + (hi[dt].x + hi[dt].y);
+      if (write_tab) {
+        uint4 q4;
+        q4.x = h2_bits(__floats2half2_rn(lo[dt].x * down, lo[dt].y * down));
+        q4.w = h2_bits(__floats2half2_rn(hi[dt].x * down, hi[dt].y * down));
+        q4.y = C::tauK != 1.f ? h2_bits(__floats2half2_rn(hi[dt].x * fold, hi[dt].y * fold)) : q4.w;
+        q4.z = q4.x;
+        *reinterpret_cast<uint4*>(qtab + (dt * 32 + lane) * 4) = q4;
+      }
+    }
+    ops.lsc = lp;
+    ops.fs0 = kTwo24 * lp;
+    ops.fs1 = kTwo24 / C::sigmaK * lp;
+    qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+    qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+    ops.qsum = qs * down;  // head g
+  }
+}
+
+// PV of head rows: A = p' (hi/lo) per 16-token k-step, B = value codes.
+template <int VB, int D, bool F8>
+__device__ __forceinline__ void head_pv(const uint8_t* vblk, WarpState<D>& st, const uint32_t (&pa)[2][4], int lane) {
+#pragma unroll
+  for (int dt = 0; dt < D / 16; ++dt) {
+    uint32_t w[TileWords<VB>::N];
+    load_tile_words<VB>(vblk, lane, dt, w);
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t b[4];
+      if constexpr (F8) tile_frags_f8(w, ks, b);
+      else tile_frags<VB>(w, ks, b);
+      if constexpr (VB == 16) {
+        mma_bf16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
+        mma_bf16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
+      } else {
+        mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
+        mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
+      }
+    }
+  }
+}
+
+// p' = p * s_t * 2^E (hi/lo) and the value zero term, then PV.
+template <int VB, int D>
+__device__ __forceinline__ void head_int_pv(const uint8_t* vblk, WarpState<D>& st, const float (&sc)[8],
+                                            const float* svf, const float* zvf, int lane) {
+  const int t = lane & 3;
   uint32_t pa[2][4];
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
@@ -445,26 +976,67 @@ __device__ __forceinline__ void attend_qpage(const uint8_t* page, WarpState<D>& 
     split_f16(p2 * s1.x, p3 * s1.y, pa[ks][2], pa[ks][3]);
     st.vz = fmaf(p0, z0.x, fmaf(p1, z0.y, fmaf(p2, z1.x, fmaf(p3, z1.y, st.vz))));
   }
-#pragma unroll
-  for (int dt = 0; dt < C::KS; ++dt) {
-    uint32_t w[TileWords<VB>::N];
-    load_tile_words<VB>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t b[4];
-      tile_frags<VB>(w, ks, b);
-      mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
-      mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
-    }
-  }
+  head_pv<VB, D, false>(vblk, st, pa, lane);
 }
 
-// Per-token keys, head rows: score of head g, token t = s_t * sum_c q'_c code_tc
-// + z_t * sum_c q'_c. The A operand is the segment's q' hi/lo fragments in
-// shared memory (2-bit tauK already folded in); no key-scale table, no z-term MMA.
+// Integer page, per-channel keys: A = exact (hi, lo) of q * s_c, B = key codes.
 template <int KB, int VB, int D>
-__device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D>& st, const uint32_t* qz,
-                                                float qsum, float* wscr, int lane) {
+__device__ __forceinline__ void attend_qpage(const uint8_t* page, WarpState<D>& st, const uint32_t* qtab,
+                                             const HeadOps& ops, float* wscr, int lane) {
+  using C = Cfg<KB, VB, D>;
+  const int t = lane & 3;
+  const uint8_t* vblk = page + code_block_bytes(KB, D);
+  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
+  const __half* kzero = kscale + D;
+  const __half* vscale = kzero + D;
+  const __half* vzero = vscale + kPageTokens;
+  float* svf = wscr;
+  float* zvf = wscr + kPageTokens;
+  value_tables<VB>(vscale, vzero, st, svf, zvf, lane);
+  __syncwarp();
+
+  float s4[4][4], cz[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s4[j][k] = 0.f;
+  const uint2* srow = reinterpret_cast<const uint2*>(kscale + t * (D / 4));
+  const uint2* zrow = reinterpret_cast<const uint2*>(kzero + t * (D / 4));
+#pragma unroll
+  for (int dt = 0; dt < C::KS; ++dt) {
+    uint32_t w[TileWords<KB>::N];
+    load_tile_words<KB>(page, lane, dt, w);
+    const uint4 q = *reinterpret_cast<const uint4*>(qtab + (dt * 32 + lane) * 4);
+    const uint2 s = srow[dt];
+    const uint32_t h01 = hmul2(q.x, s.x), h89 = hmul2(q.y, s.y);
+    const uint32_t l01 = hfma2(q.x, s.x, hneg2(h01)), l89 = hfma2(q.y, s.y, hneg2(h89));
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      uint32_t b[4];
+      tile_frags<KB>(w, tt, b);
+      mma_f16(s4[2 * tt], h01, l01, h89, l89, b[0], b[1]);
+      mma_f16(s4[2 * tt + 1], h01, l01, h89, l89, b[2], b[3]);
+    }
+    const uint2 z = zrow[dt];
+    mma_f16(cz, q.z, 0u, q.w, 0u, z.x, z.y);
+  }
+  const float czv = (cz[0] + cz[2]) * ops.lsc;  // every column holds the same sum
+  float sc[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float f = (j & 1) ? ops.fs1 : ops.fs0;
+    sc[2 * j] = fmaf(s4[j][0] + s4[j][2], f, czv);
+    sc[2 * j + 1] = fmaf(s4[j][1] + s4[j][3], f, czv);
+  }
+  softmax_update<D>(st, sc);
+  head_int_pv<VB, D>(vblk, st, sc, svf, zvf, lane);
+}
+
+// Integer page, per-token keys: score of head g, token t = (s_t * sum_c q_c
+// code_tc + z_t * sum_c q_c) * log2(e)/sqrt(D) * 2^k.
+template <int KB, int VB, int D>
+__device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D>& st, const uint32_t* qtab,
+                                                const HeadOps& ops, float* wscr, int lane) {
   using C = Cfg<KB, VB, D, true>;
   const int t = lane & 3;
   const uint8_t* vblk = page + code_block_bytes(KB, D);
@@ -472,16 +1044,13 @@ __device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D
   const __half* kzero = kscale + kPageTokens;
   const __half* vscale = kzero + kPageTokens;
   const __half* vzero = vscale + kPageTokens;
-  float* kst = wscr;                   // [32] key scales x 2^24 (/ sigmaK on tokens with bit 3 set)
-  float* kzt = wscr + kPageTokens;     // [32] key zeros
-  float* svf = wscr + 4 * C::KSROW;    // [32] value scales, tauV folded
-  float* zvf = svf + kPageTokens;      // [32] value zeros
-  kst[lane] = __half2float(kscale[lane]) * ((lane & 8) ? kTwo24 / C::sigmaK : kTwo24);
-  kzt[lane] = __half2float(kzero[lane]);
-  const float vs = __half2float(vscale[lane]);
-  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
-  zvf[lane] = __half2float(vzero[lane]);
-  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
+  float* svf = wscr;
+  float* zvf = wscr + kPageTokens;
+  float* kst = wscr + 2 * kPageTokens;
+  float* kzt = wscr + 3 * kPageTokens;
+  kst[lane] = __half2float(kscale[lane]) * ((lane & 8) ? ops.fs1 : ops.fs0);
+  kzt[lane] = __half2float(kzero[lane]) * ops.lsc;
+  value_tables<VB>(vscale, vzero, st, svf, zvf, lane);
   __syncwarp();
 
   float s4[4][4];
@@ -493,13 +1062,13 @@ __device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D
   for (int dt = 0; dt < C::KS; ++dt) {
     uint32_t w[TileWords<KB>::N];
     load_tile_words<KB>(page, lane, dt, w);
-    const uint4 a = *reinterpret_cast<const uint4*>(qz + (dt * 32 + lane) * 4);
+    const uint2 q = *reinterpret_cast<const uint2*>(qtab + (dt * 32 + lane) * 4);
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
       uint32_t b[4];
       tile_frags<KB>(w, tt, b);
-      mma_f16(s4[2 * tt], a.x, a.y, a.z, a.w, b[0], b[1]);
-      mma_f16(s4[2 * tt + 1], a.x, a.y, a.z, a.w, b[2], b[3]);
+      mma_f16(s4[2 * tt], q.x, 0u, q.y, 0u, b[0], b[1]);
+      mma_f16(s4[2 * tt + 1], q.x, 0u, q.y, 0u, b[2], b[3]);
     }
   }
   float sc[8];
@@ -508,43 +1077,17 @@ __device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D
 #pragma unroll
     for (int jj = 0; jj < 2; ++jj) {
       const int tok = 8 * j + 2 * t + jj;
-      sc[2 * j + jj] = fmaf(s4[j][jj] + s4[j][jj + 2], kst[tok], kzt[tok] * qsum);
+      sc[2 * j + jj] = fmaf(s4[j][jj] + s4[j][jj + 2], kst[tok], kzt[tok] * ops.qsum);
     }
-  softmax_update<D>(st, sc, tau);
-
-  uint32_t pa[2][4];
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    const int t0 = 16 * ks + 2 * t, t1 = t0 + 8;
-    const float2 s0 = *reinterpret_cast<const float2*>(svf + t0);
-    const float2 s1 = *reinterpret_cast<const float2*>(svf + t1);
-    const float2 z0 = *reinterpret_cast<const float2*>(zvf + t0);
-    const float2 z1 = *reinterpret_cast<const float2*>(zvf + t1);
-    const float p0 = sc[4 * ks + 0], p1 = sc[4 * ks + 1], p2 = sc[4 * ks + 2], p3 = sc[4 * ks + 3];
-    split_f16(p0 * s0.x, p1 * s0.y, pa[ks][0], pa[ks][1]);
-    split_f16(p2 * s1.x, p3 * s1.y, pa[ks][2], pa[ks][3]);
-    st.vz = fmaf(p0, z0.x, fmaf(p1, z0.y, fmaf(p2, z1.x, fmaf(p3, z1.y, st.vz))));
-  }
-#pragma unroll
-  for (int dt = 0; dt < C::KS; ++dt) {
-    uint32_t w[TileWords<VB>::N];
-    load_tile_words<VB>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t b[4];
-      tile_frags<VB>(w, ks, b);
-      mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
-      mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
-    }
-  }
+  softmax_update<D>(st, sc);
+  head_int_pv<VB, D>(vblk, st, sc, svf, zvf, lane);
 }
 
-// fp8 page, head rows: A = the segment's q' hi/lo fragments with the KV head's
-// key scale folded in, B = e4m3 keys as f16 (times 2^-8, undone on the scores);
-// p hi/lo against e4m3 values (the value scale and 2^8 are applied once, to
-// the accumulators).
+// fp8 page: A = the segment's q' hi/lo fragments with the KV head's key scale
+// folded in, B = e4m3 keys as f16 (times 2^-8, undone on the scores); p hi/lo
+// against e4m3 values (the value scale and 2^8 are applied once, at the end).
 template <int D>
-__device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>& st, const uint32_t* qz, int lane) {
+__device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>& st, const uint32_t* qtab, int lane) {
   constexpr int KS = D / 16;
   float s4[4][4];
 #pragma unroll
@@ -555,7 +1098,7 @@ __device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>&
   for (int dt = 0; dt < KS; ++dt) {
     uint32_t w[TileWords<8>::N];
     load_tile_words<8>(page, lane, dt, w);
-    const uint4 a = *reinterpret_cast<const uint4*>(qz + (dt * 32 + lane) * 4);
+    const uint4 a = *reinterpret_cast<const uint4*>(qtab + (dt * 32 + lane) * 4);
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
       uint32_t b[4];
@@ -570,32 +1113,20 @@ __device__ __forceinline__ void attend_f8page(const uint8_t* page, WarpState<D>&
     sc[2 * j] = (s4[j][0] + s4[j][2]) * kF8Unit;
     sc[2 * j + 1] = (s4[j][1] + s4[j][3]) * kF8Unit;
   }
-  softmax_update<D>(st, sc, kTau);
+  softmax_update<D>(st, sc);
   uint32_t pa[2][4];
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
     split_f16(sc[4 * ks + 0], sc[4 * ks + 1], pa[ks][0], pa[ks][1]);
     split_f16(sc[4 * ks + 2], sc[4 * ks + 3], pa[ks][2], pa[ks][3]);
   }
-  const uint8_t* vblk = page + code_block_bytes(8, D);
-#pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t w[TileWords<8>::N];
-    load_tile_words<8>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t b[4];
-      tile_frags_f8(w, ks, b);
-      mma_f16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
-      mma_f16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
-    }
-  }
+  head_pv<8, D, true>(page + code_block_bytes(8, D), st, pa, lane);
 }
 
 // One full bf16 page: raw bf16 values, q unscaled (exact in bf16), p hi/lo.
 template <int D>
-__device__ __forceinline__ void attend_bpage(const uint8_t* page, WarpState<D>& st,
-                                             const uint32_t (&qb)[D / 8], float scale_log2, int lane) {
+__device__ __forceinline__ void attend_bpage(const uint8_t* page, WarpState<D>& st, const uint32_t (&qb)[D / 8],
+                                             float scale_log2, int lane) {
   constexpr int KS = D / 16;
   float s4[4][4];
 #pragma unroll
@@ -620,26 +1151,14 @@ __device__ __forceinline__ void attend_bpage(const uint8_t* page, WarpState<D>& 
     sc[2 * j] = s4[j][0] * scale_log2;
     sc[2 * j + 1] = s4[j][1] * scale_log2;
   }
-  softmax_update<D>(st, sc, kTau);
+  softmax_update<D>(st, sc);
   uint32_t pa[2][4];
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
     split_bf16(sc[4 * ks + 0], sc[4 * ks + 1], pa[ks][0], pa[ks][1]);
     split_bf16(sc[4 * ks + 2], sc[4 * ks + 3], pa[ks][2], pa[ks][3]);
   }
-  const uint8_t* vblk = page + code_block_bytes(16, D);
-#pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t w[TileWords<16>::N];
-    load_tile_words<16>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t b[4];
-      tile_frags<16>(w, ks, b);
-      mma_bf16(st.o[2 * dt], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[0], b[1]);
-      mma_bf16(st.o[2 * dt + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b[2], b[3]);
-    }
-  }
+  head_pv<16, D, false>(page + code_block_bytes(16, D), st, pa, lane);
 }
 
 // The bf16 window (natural [32][D] rows in global memory), W < 32 valid tokens.
@@ -676,7 +1195,7 @@ __device__ __forceinline__ void attend_window(const __nv_bfloat16* win, int W, W
     sc[2 * j] = tok < W ? s4[j][0] * scale_log2 : -INFINITY;
     sc[2 * j + 1] = tok + 1 < W ? s4[j][1] * scale_log2 : -INFINITY;
   }
-  softmax_update<D>(st, sc, kTau);
+  softmax_update<D>(st, sc);
   uint32_t pa[2][4];
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
@@ -700,428 +1219,222 @@ __device__ __forceinline__ void attend_window(const __nv_bfloat16* win, int W, W
   }
 }
 
-// Raw bf16 pairs of q for lane (g, t): channels 16dt + 2t (+1) and 16dt + 2t + 8 (+9).
-template <int D>
-__device__ __forceinline__ void load_qb(const __nv_bfloat16* qrow, bool valid, int t, uint32_t (&qb)[D / 8]) {
+// ---------------------------------------------------- output scaling --
+// Integer / fp8 accumulators to true units: acc * 2^24 * 2^-E (/ sigmaV on value
+// channels with bit 3 set); fp8: acc * the KV head's value scale * 2^8.
+template <int VB, bool TOK, bool F8, int NT>
+__device__ __forceinline__ void to_true_units(State<NT>& st, float f8_vscale) {
+  if constexpr (F8) {
+    const float f = f8_vscale * kF8Unit;
 #pragma unroll
-  for (int dt = 0; dt < D / 16; ++dt) {
-    qb[2 * dt] = valid ? *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t) : 0u;
-    qb[2 * dt + 1] = valid ? *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8) : 0u;
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st.o[j][k] *= f;
+  } else if constexpr (VB != 16) {
+    constexpr float sigmaV = VB == 4 ? 16.f : (VB == 2 ? 4.f : 1.f);
+    const float f = kTwo24 * exp2i(st.E == kNoExp ? 0 : -st.E);
+    const float fh = f * (1.f / sigmaV);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if constexpr (TOK) {
+        st.o[j][0] *= f;
+        st.o[j][1] *= f;
+        st.o[j][2] *= fh;
+        st.o[j][3] *= fh;
+      } else {
+        const float x = (j & 1) ? fh : f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st.o[j][k] *= x;
+      }
+    }
   }
 }
 
-// ============================================================================
-// Token-row formulation (G <= 4): MMA rows are tokens (QK) and channels (PV);
-// the 8 columns are (head c/2, part c%2) with part 0 = high f16 half and part 1
-// = low half of q' (QK) or p' (PV). Lane (g, t) keeps head t's scores for
-// tokens g, g+8, g+16, g+24 and head t's output for channels g, g+8 of every
-// 16-channel tile. 16 QK + 16 PV + 8 z-term MMAs per page.
-template <int D>
-struct TokState {
-  float o[D / 16][4];  // [channel tile]: c0/c1 = head t parts at channel g, c2/c3 at channel g+8
-  float m, l, vz;      // head t: reference max, partial sum over this lane's tokens, sum p*z
-};
-
-template <int D>
-__device__ __forceinline__ void tok_rescale_update(TokState<D>& st, float (&sc)[4], float tau) {
-  float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-  if (mx > st.m + tau) {
-    const float alpha = ex2(st.m - mx);
-#pragma unroll
-    for (int j = 0; j < D / 16; ++j)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) st.o[j][k] *= alpha;
-    st.l *= alpha;
-    st.vz *= alpha;
-    st.m = mx;
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    sc[i] = ex2(sc[i] - st.m);
-    st.l += sc[i];
+// ------------------------------------------------------------ fused append --
+// Warp-level flush of one completed 32-token group (the window's 31 tokens and
+// the new token) into `page`, bit-identical to the append kernel's CTA-wide
+// flush: the same quantizer and packing (kvq_quant.cuh), only the work split
+// differs. It needs no staging buffer: a first pass takes each set's min and
+// max and keeps the quantizer parameters in `prm` (this warp's scratch, 2D + 64
+// floats); the second pass quantizes each element as it is packed.
+template <int BITS, int D, typename Get>
+__device__ __forceinline__ void pack_block_warp(uint8_t* blk, bool is_value, int lane, Get vals) {
+  constexpr int kPerLane = (int)(code_block_bytes(BITS, D) / 16) / 32;  // 16-byte vectors per lane
+#pragma unroll 1
+  for (int vi = 0; vi < kPerLane; ++vi) {
+    uint4 q;
+    q.x = lane_word<BITS>(lane, 4 * vi + 0, is_value, vals);
+    q.y = lane_word<BITS>(lane, 4 * vi + 1, is_value, vals);
+    q.z = lane_word<BITS>(lane, 4 * vi + 2, is_value, vals);
+    q.w = lane_word<BITS>(lane, 4 * vi + 3, is_value, vals);
+    reinterpret_cast<uint4*>(blk)[vi * 32 + lane] = q;
   }
 }
 
-// A fragment of tile (dt, tt) from this lane's words (rows: tokens for keys,
-// channels for values; columns: channels for keys, tokens for values).
-template <int BITS>
-__device__ __forceinline__ void tile_afrag(const uint32_t (&w)[TileWords<BITS>::N], int tt, uint32_t (&a)[4]) {
-  if constexpr (BITS == 4) {
-    uint32_t x = w[tt], y = x >> 8;
-    a[0] = x & 0x000F000Fu;   // rows g,   cols 2t..     x1
-    a[1] = x & 0x00F000F0u;   // rows g+8, cols 2t..     x16
-    a[2] = y & 0x000F000Fu;   // rows g,   cols 2t+8..   x1
-    a[3] = y & 0x00F000F0u;   // rows g+8, cols 2t+8..   x16
-  } else if constexpr (BITS == 2) {
-    uint32_t x = tt ? (w[0] >> 8) : w[0];
-    a[0] = x & 0x00030003u;   // x1
-    a[1] = x & 0x000C000Cu;   // x4
-    a[2] = x & 0x00300030u;   // x16
-    a[3] = x & 0x00C000C0u;   // x64
-  } else if constexpr (BITS == 8) {
-    uint32_t x = w[2 * tt], y = w[2 * tt + 1];
-    a[0] = __byte_perm(x, 0u, 0x4140);
-    a[1] = __byte_perm(x, 0u, 0x4342);
-    a[2] = __byte_perm(y, 0u, 0x4140);
-    a[3] = __byte_perm(y, 0u, 0x4342);
+template <int KB, int VB, int D, bool PT, bool F8>
+__device__ __noinline__ void warp_flush(uint8_t* page, const __nv_bfloat16* win, const __nv_bfloat16* kn,
+                                        const __nv_bfloat16* vn, float* prm, float ksc, float vsc,
+                                        double* err_stats, int lane) {
+  // row of token tok (0..31) of keys (r = 0) or values (r = 1)
+  auto row = [&](int r, int tok) -> const __nv_bfloat16* {
+    return tok < kPageTokens - 1 ? win + (r * kPageTokens + tok) * D : (r ? vn : kn);
+  };
+  if constexpr (KB == 16) {
+    pack_block_warp<16, D>(page, false, lane,
+                           [&](int tok, int dim) { return (uint32_t)__bfloat16_as_ushort(row(0, tok)[dim]); });
+    pack_block_warp<16, D>(page + code_block_bytes(16, D), true, lane,
+                           [&](int tok, int dim) { return (uint32_t)__bfloat16_as_ushort(row(1, tok)[dim]); });
+    return;
   } else {
-    a[0] = w[4 * tt + 0];
-    a[1] = w[4 * tt + 1];
-    a[2] = w[4 * tt + 2];
-    a[3] = w[4 * tt + 3];
-  }
-}
-
-// hi (part 0) or lo (part 1) f16 halves of (x0, x1) as one register.
-__device__ __forceinline__ uint32_t part_f16(float x0, float x1, float partf) {
-  __half2 h = __floats2half2_rn(x0, x1);
-  float2 f = __half22float2(h);
-  return h2_bits(__floats2half2_rn(fmaf(-partf, f.x, x0), fmaf(-partf, f.y, x1)));
-}
-
-__device__ __forceinline__ uint32_t part_bf16(float x0, float x1, float partf) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  float2 f = __bfloat1622float2(h);
-  return b2_bits(__floats2bfloat162_rn(fmaf(-partf, f.x, x0), fmaf(-partf, f.y, x1)));
-}
-
-// Transpose p' (this lane: head t, tokens g + 8i) into the PV B fragments
-// (this lane: column g = (head g/2, part g%2), tokens 2t, 2t+1, 2t+8, 2t+9 of
-// each 16-token k-step). `ptr` is a per-warp [4][40] float tile.
-template <bool BF16>
-__device__ __forceinline__ void tok_pfrags(float* ptr, const float (&pv)[4], int lane, float partf,
-                                           uint32_t (&b)[2][2]) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) ptr[t * 40 + g + 8 * i] = pv[i];
-  __syncwarp();
-  const float* row = ptr + (g >> 1) * 40 + 2 * t;
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    const float2 lo = *reinterpret_cast<const float2*>(row + 16 * ks);
-    const float2 hi = *reinterpret_cast<const float2*>(row + 16 * ks + 8);
-    if constexpr (BF16) {
-      b[ks][0] = part_bf16(lo.x, lo.y, partf);
-      b[ks][1] = part_bf16(hi.x, hi.y, partf);
+    double err[4] = {0.0, 0.0, 0.0, 0.0};
+    auto add_err = [&](int r, float x, double xh) {
+      const double dx = (double)x - xh;
+      err[2 * r] += dx * dx;
+      err[2 * r + 1] += (double)x * (double)x;
+    };
+    if constexpr (F8) {
+      // every element is e4m3(x / s_h) of its KV head's scale
+      auto code = [&](int r, int tok, int dim) -> uint32_t {
+        const float x = __bfloat162float(row(r, tok)[dim]);
+        const float sc = r ? vsc : ksc;
+        const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(__fdiv_rn(x, sc), __NV_SATFINITE, __NV_E4M3);
+        add_err(r, x, (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3))) * sc);
+        return (uint32_t)c;
+      };
+      pack_block_warp<8, D>(page, false, lane, [&](int tok, int dim) { return code(0, tok, dim); });
+      pack_block_warp<8, D>(page + code_block_bytes(8, D), true, lane,
+                            [&](int tok, int dim) { return code(1, tok, dim); });
     } else {
-      b[ks][0] = part_f16(lo.x, lo.y, partf);
-      b[ks][1] = part_f16(hi.x, hi.y, partf);
+      constexpr int nk = PT ? kPageTokens : D;  // key scale/zero pairs
+      uint8_t* vblk = page + code_block_bytes(KB, D);
+      __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
+      __half* kzero = kscale + nk;
+      __half* vscale = kzero + nk;
+      __half* vzero = vscale + kPageTokens;
+      // quantizer parameters (zero point z and reciprocal r = 1/s, r = 0 for a
+      // constant set) of the keys (by channel, or by token) and of the values
+      float* kz = prm;
+      float* kr = prm + nk;
+      float* vz = prm + 2 * nk;
+      float* vr = vz + kPageTokens;
+      // per token over head_dim (values; keys in per-token mode): lane = token
+      auto per_token = [&](int r, int qmax, __half* sdst, __half* zdst, float* zp, float* rp) {
+        const __nv_bfloat16* src = row(r, lane);
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll 1
+        for (int c8 = 0; c8 < D; c8 += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
+          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float x = __bfloat162float(xv[j]);
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+        }
+        const QParams q = make_qparams(mn, mx, qmax);
+        sdst[lane] = q.s_h;
+        zdst[lane] = q.z_h;
+        zp[lane] = q.z;
+        rp[lane] = q.r;  // 0 for a constant set
+      };
+      if constexpr (PT) {
+        per_token(0, (1 << KB) - 1, kscale, kzero, kz, kr);
+      } else {
+        // keys per channel over the 32 tokens: lane owns channels lane * NC .. + NC - 1
+        constexpr int NC = D / 32;
+        const int c0 = lane * NC;
+        float mn[NC], mx[NC];
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+          mn[j] = INFINITY;
+          mx[j] = -INFINITY;
+        }
+#pragma unroll 1
+        for (int tok = 0; tok < kPageTokens; ++tok) {
+          const __nv_bfloat16* src = row(0, tok) + c0;
+#pragma unroll
+          for (int j = 0; j < NC; ++j) {
+            const float x = __bfloat162float(src[j]);
+            mn[j] = fminf(mn[j], x);
+            mx[j] = fmaxf(mx[j], x);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+          const QParams q = make_qparams(mn[j], mx[j], (1 << KB) - 1);
+          const int slot = kmeta_slot<D>(c0 + j);
+          kscale[slot] = q.s_h;
+          kzero[slot] = q.z_h;
+          kz[c0 + j] = q.z;
+          kr[c0 + j] = q.r;
+        }
+      }
+      per_token(1, (1 << VB) - 1, vscale, vzero, vz, vr);
+      __syncwarp();  // parameters and page metadata visible to the warp
+      // element (tok, dim) of keys (r = 0) or values (r = 1): its code, counted once in the report
+      auto code = [&](int r, int tok, int dim) -> uint32_t {
+        const float x = __bfloat162float(row(r, tok)[dim]);
+        const int i = (r == 0 && !PT) ? dim : tok;
+        QParams q;
+        q.z = r ? vz[i] : kz[i];
+        q.r = r ? vr[i] : kr[i];
+        q.zero_scale = (q.r == 0.0f);
+        const int qmax = (1 << (r ? VB : KB)) - 1;
+        const uint32_t c = quant_code(x, q, qmax);
+        const __half sh = r ? vscale[i] : kscale[(PT ? i : kmeta_slot<D>(i))];
+        add_err(r, x, (double)c * (double)__half2float(sh) + (double)q.z);
+        return c;
+      };
+      pack_block_warp<KB, D>(page, false, lane, [&](int tok, int dim) { return code(0, tok, dim); });
+      pack_block_warp<VB, D>(vblk, true, lane, [&](int tok, int dim) { return code(1, tok, dim); });
     }
-  }
-  __syncwarp();
-}
-
-template <int KB, int VB, int D>
-__device__ __forceinline__ void attend_qpage_tok(const uint8_t* page, TokState<D>& st, const float (&qf)[D / 4],
-                                                 const uint32_t (&qzb)[D / 8], float* wscr, float partf,
-                                                 int lane) {
-  using C = Cfg<KB, VB, D>;
-  const int g = lane >> 2, t = lane & 3;
-  const uint8_t* vblk = page + code_block_bytes(KB, D);
-  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
-  const __half* kzero = kscale + D;
-  const __half* vscale = kzero + D;
-  const __half* vzero = vscale + kPageTokens;
-  float* ksf = wscr;
-  float* svf = wscr + 4 * C::KSROW;
-  float* zvf = svf + kPageTokens;
-  float* ptr = zvf + kPageTokens;  // [4][40]
-  {
-    constexpr int NE = D / 32;
-    const int i0 = lane * NE;
-    float* dst = ksf + (i0 / (D / 4)) * C::KSROW + (i0 % (D / 4));
-    if constexpr (NE == 4) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(kscale + i0);
-      float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      if (C::tauK != 1.f) { c.x *= 1.f / C::tauK; c.y *= 1.f / C::tauK; }
-      *reinterpret_cast<float4*>(dst) = make_float4(a.x, a.y, c.x, c.y);
-    } else {
-      const uint32_t raw = *reinterpret_cast<const uint32_t*>(kscale + i0);
-      float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw));
-      if (C::tauK != 1.f && (i0 & 2)) { a.x *= 1.f / C::tauK; a.y *= 1.f / C::tauK; }
-      *reinterpret_cast<float2*>(dst) = a;
+    // this flush's error sums: warp shuffles, then one fp64 atomic per sum
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      double v = err[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      err[i] = v;
     }
-  }
-  const float vs = __half2float(vscale[lane]);
-  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
-  zvf[lane] = __half2float(vzero[lane]);
-  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
-  __syncwarp();
-
-  // --- QK: two token m-tiles, B = q' parts; z-term: A = z rows, B = q parts
-  float s2[2][4], cz[4] = {0.f, 0.f, 0.f, 0.f};
+    if (err_stats && lane == 0) {
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
-  const float* ksl = ksf + t * C::KSROW;
-  const uint32_t* zrow = reinterpret_cast<const uint32_t*>(kzero + t * (D / 4));
-#pragma unroll
-  for (int dt = 0; dt < C::KS; ++dt) {
-    uint32_t w[TileWords<KB>::N];
-    load_tile_words<KB>(page, lane, dt, w);
-    const float4 sc4 = *reinterpret_cast<const float4*>(ksl + dt * 4);
-    const uint32_t b0 = part_f16(qf[dt * 4 + 0] * sc4.x, qf[dt * 4 + 1] * sc4.y, partf);
-    const uint32_t b1 = part_f16(qf[dt * 4 + 2] * sc4.z, qf[dt * 4 + 3] * sc4.w, partf);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t a[4];
-      tile_afrag<KB>(w, mt, a);
-      mma_f16(s2[mt], a[0], a[1], a[2], a[3], b0, b1);
-    }
-    const uint2 z = *reinterpret_cast<const uint2*>(zrow + dt * 2);
-    mma_f16(cz, z.x, z.x, z.y, z.y, qzb[2 * dt], qzb[2 * dt + 1]);
-  }
-  const float czv = cz[0] + cz[1];  // head t: both parts of sum_c q_c z_c
-  float sc[4];
-  sc[0] = fmaf(s2[0][0] + s2[0][1], kTwo24, czv);
-  sc[1] = fmaf(s2[0][2] + s2[0][3], kTwo24 / C::sigmaK, czv);
-  sc[2] = fmaf(s2[1][0] + s2[1][1], kTwo24, czv);
-  sc[3] = fmaf(s2[1][2] + s2[1][3], kTwo24 / C::sigmaK, czv);
-  tok_rescale_update<D>(st, sc, tau);
-
-  // --- p' = p * s_t for tokens g + 8i; value zero term; transpose to B fragments
-  float pv[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    pv[i] = sc[i] * svf[g + 8 * i];
-    st.vz = fmaf(sc[i], zvf[g + 8 * i], st.vz);
-  }
-  uint32_t pb[2][2];
-  tok_pfrags<false>(ptr, pv, lane, partf, pb);
-
-  // --- PV: A = value codes (rows = channels), B = p' parts
-#pragma unroll
-  for (int dt = 0; dt < C::KS; ++dt) {
-    uint32_t w[TileWords<VB>::N];
-    load_tile_words<VB>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t a[4];
-      tile_afrag<VB>(w, ks, a);
-      mma_f16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
-    }
-  }
-}
-
-// Per-token keys, token rows: B = the segment's q' parts (tauK folded, fixed per
-// segment); score of token g + 8i for head t = s * acc + z * sum_c q'_c.
-template <int KB, int VB, int D>
-__device__ __forceinline__ void attend_qpage_tok_pt(const uint8_t* page, TokState<D>& st,
-                                                    const uint32_t (&qkb)[D / 8], float qsum, float* wscr,
-                                                    float partf, int lane) {
-  using C = Cfg<KB, VB, D, true>;
-  const int g = lane >> 2;
-  const uint8_t* vblk = page + code_block_bytes(KB, D);
-  const __half* kscale = reinterpret_cast<const __half*>(vblk + code_block_bytes(VB, D));
-  const __half* kzero = kscale + kPageTokens;
-  const __half* vscale = kzero + kPageTokens;
-  const __half* vzero = vscale + kPageTokens;
-  float* kst = wscr;
-  float* kzt = wscr + kPageTokens;
-  float* svf = wscr + 4 * C::KSROW;
-  float* zvf = svf + kPageTokens;
-  float* ptr = zvf + kPageTokens;  // [4][40]
-  kst[lane] = __half2float(kscale[lane]) * ((lane & 8) ? kTwo24 / C::sigmaK : kTwo24);
-  kzt[lane] = __half2float(kzero[lane]);
-  const float vs = __half2float(vscale[lane]);
-  svf[lane] = (C::tauV != 1.f && (lane & 8)) ? vs * (1.f / C::tauV) : vs;
-  zvf[lane] = __half2float(vzero[lane]);
-  const float tau = __any_sync(0xffffffffu, vs > kScaleCapLazy) ? 0.f : kTau;
-  __syncwarp();
-
-  float s2[2][4];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
-#pragma unroll
-  for (int dt = 0; dt < C::KS; ++dt) {
-    uint32_t w[TileWords<KB>::N];
-    load_tile_words<KB>(page, lane, dt, w);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t a[4];
-      tile_afrag<KB>(w, mt, a);
-      mma_f16(s2[mt], a[0], a[1], a[2], a[3], qkb[2 * dt], qkb[2 * dt + 1]);
-    }
-  }
-  float sc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int tok = g + 8 * i;
-    const float acc = s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1];
-    sc[i] = fmaf(acc, kst[tok], kzt[tok] * qsum);
-  }
-  tok_rescale_update<D>(st, sc, tau);
-
-  float pv[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    pv[i] = sc[i] * svf[g + 8 * i];
-    st.vz = fmaf(sc[i], zvf[g + 8 * i], st.vz);
-  }
-  uint32_t pb[2][2];
-  tok_pfrags<false>(ptr, pv, lane, partf, pb);
-#pragma unroll
-  for (int dt = 0; dt < C::KS; ++dt) {
-    uint32_t w[TileWords<VB>::N];
-    load_tile_words<VB>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t a[4];
-      tile_afrag<VB>(w, ks, a);
-      mma_f16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
+      for (int i = 0; i < 4; ++i) atomicAdd(&err_stats[i], err[i]);
+      atomicAdd(&err_stats[4], (double)(kPageTokens * D));
     }
   }
 }
 
-// fp8 page, token rows: A = e4m3 keys/values as f16, B = the segment's q' parts
-// (key scale folded in) or p parts.
-template <int D>
-__device__ __forceinline__ void attend_f8page_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qkb)[D / 8],
-                                                  float* wscr, float partf, int lane) {
-  constexpr int KS = D / 16;
-  float* ptr = wscr + 4 * (D / 4 + 4) + 2 * kPageTokens;
-  float s2[2][4];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
-#pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t w[TileWords<8>::N];
-    load_tile_words<8>(page, lane, dt, w);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t a[4];
-      tile_afrag_f8(w, mt, a);
-      mma_f16(s2[mt], a[0], a[1], a[2], a[3], qkb[2 * dt], qkb[2 * dt + 1]);
+// Append segment s's new token: into window slot t0 mod 32, or, when it
+// completes a group, quantized with the window's 31 tokens into page t0 / 32.
+// Returns true when a page was written.
+template <int KB, int VB, int D, bool PT, bool F8>
+__device__ __forceinline__ bool append_token(const DecodeParams& p, int s, int h, int t0, float* prm, int lane) {
+  __nv_bfloat16* wwin = p.step_window + ((int64_t)s * 2) * kPageTokens * D;
+  const __nv_bfloat16* kn = p.k_new + (int64_t)s * D;
+  const __nv_bfloat16* vn = p.v_new + (int64_t)s * D;
+  bool flushed = false;
+  if ((t0 + 1) % kPageTokens != 0) {
+    const int slot = t0 % kPageTokens;
+    for (int d = 2 * lane; d < D; d += 64) {
+      *reinterpret_cast<uint32_t*>(wwin + slot * D + d) = *reinterpret_cast<const uint32_t*>(kn + d);
+      *reinterpret_cast<uint32_t*>(wwin + (kPageTokens + slot) * D + d) = *reinterpret_cast<const uint32_t*>(vn + d);
     }
+  } else {
+    flushed = true;
+    warp_flush<KB, VB, D, PT, F8>(p.step_pages + ((int64_t)s * p.max_pages + t0 / kPageTokens) * p.page_bytes, wwin,
+                                  kn, vn, prm, F8 ? p.fp8_scales[h] : 1.f, F8 ? p.fp8_scales[p.n_kv_heads + h] : 1.f,
+                                  err_bin(p.err_stats, (unsigned)s), lane);
   }
-  float sc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) sc[i] = (s2[i >> 1][2 * (i & 1)] + s2[i >> 1][2 * (i & 1) + 1]) * kF8Unit;
-  tok_rescale_update<D>(st, sc, kTau);
-  uint32_t pb[2][2];
-  tok_pfrags<false>(ptr, sc, lane, partf, pb);
-  const uint8_t* vblk = page + code_block_bytes(8, D);
-#pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t w[TileWords<8>::N];
-    load_tile_words<8>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t a[4];
-      tile_afrag_f8(w, ks, a);
-      mma_f16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
-    }
-  }
-}
-
-template <int D>
-__device__ __forceinline__ void attend_bpage_tok(const uint8_t* page, TokState<D>& st, const uint32_t (&qbp)[D / 8],
-                                                 float* wscr, float partf, float scale_log2, int lane) {
-  constexpr int KS = D / 16;
-  float* ptr = wscr + 4 * (D / 4 + 4) + 2 * kPageTokens;
-  float s2[2][4];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
-#pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t w[TileWords<16>::N];
-    load_tile_words<16>(page, lane, dt, w);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t a[4];
-      tile_afrag<16>(w, mt, a);
-      mma_bf16(s2[mt], a[0], a[1], a[2], a[3], qbp[2 * dt], qbp[2 * dt + 1]);
-    }
-  }
-  float sc[4] = {(s2[0][0] + s2[0][1]) * scale_log2, (s2[0][2] + s2[0][3]) * scale_log2,
-                 (s2[1][0] + s2[1][1]) * scale_log2, (s2[1][2] + s2[1][3]) * scale_log2};
-  tok_rescale_update<D>(st, sc, kTau);
-  uint32_t pb[2][2];
-  tok_pfrags<true>(ptr, sc, lane, partf, pb);
-  const uint8_t* vblk = page + code_block_bytes(16, D);
-#pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t w[TileWords<16>::N];
-    load_tile_words<16>(vblk, lane, dt, w);
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t a[4];
-      tile_afrag<16>(w, ks, a);
-      mma_bf16(st.o[dt], a[0], a[1], a[2], a[3], pb[ks][0], pb[ks][1]);
-    }
-  }
-}
-
-// bf16 window (natural [32][D] rows in global memory), W < 32 valid tokens.
-template <int D>
-__device__ __forceinline__ void attend_window_tok(const __nv_bfloat16* win, int W, TokState<D>& st,
-                                                  const uint32_t (&qbp)[D / 8], float* wscr, float partf,
-                                                  float scale_log2, int lane) {
-  constexpr int KS = D / 16;
-  const int g = lane >> 2, t = lane & 3;
-  float* ptr = wscr + 4 * (D / 4 + 4) + 2 * kPageTokens;
-  const uint16_t* kw = reinterpret_cast<const uint16_t*>(win);
-  const uint16_t* vw = kw + kPageTokens * D;
-  auto kpair = [&](int tok, int dim) -> uint32_t {
-    return tok < W ? *reinterpret_cast<const uint32_t*>(kw + tok * D + dim) : 0u;
-  };
-  auto vpair = [&](int tok, int dim) -> uint32_t {
-    const uint32_t lo = tok < W ? vw[tok * D + dim] : 0u;
-    const uint32_t hi = tok + 1 < W ? vw[(tok + 1) * D + dim] : 0u;
-    return lo | (hi << 16);
-  };
-  float s2[2][4];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-    if (16 * mt >= W) continue;  // warp-uniform
-#pragma unroll
-    for (int dt = 0; dt < KS; ++dt) {
-      const int r0 = 16 * mt + g, c0 = 16 * dt + 2 * t;
-      mma_bf16(s2[mt], kpair(r0, c0), kpair(r0 + 8, c0), kpair(r0, c0 + 8), kpair(r0 + 8, c0 + 8), qbp[2 * dt],
-               qbp[2 * dt + 1]);
-    }
-  }
-  float sc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float v = (i & 1) ? (s2[i >> 1][2] + s2[i >> 1][3]) : (s2[i >> 1][0] + s2[i >> 1][1]);
-    sc[i] = (g + 8 * i) < W ? v * scale_log2 : -INFINITY;
-  }
-  tok_rescale_update<D>(st, sc, kTau);
-  uint32_t pb[2][2];
-  tok_pfrags<true>(ptr, sc, lane, partf, pb);
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    if (16 * ks >= W) continue;  // warp-uniform
-#pragma unroll
-    for (int dt = 0; dt < KS; ++dt) {
-      const int tk = 16 * ks + 2 * t, ch = 16 * dt + g;
-      mma_bf16(st.o[dt], vpair(tk, ch), vpair(tk, ch + 8), vpair(tk + 8, ch), vpair(tk + 8, ch + 8), pb[ks][0],
-               pb[ks][1]);
-    }
-  }
+  __syncwarp();  // the window row or the page is complete for every lane
+  return flushed;
 }
 
 // ------------------------------------------------------------------ kernel --
 // Units: per (sequence b, KV head h) segment, V "overhead" units (no work:
 // they stand for the fixed cost of starting and merging a segment part, so a
-// CTA that spans several segments gets fewer pages), then the pages in order,
-// then one window unit when T mod 32 > 0 (or one empty unit when T = 0).
+// CTA that spans several segments gets fewer pages), then one tail unit (the
+// bf16 window, and in the fused step the new token's append), then the pages.
 // Segment (b, h) occupies units [ustart[b] + h * n_b, ... + n_b). The N units
 // are cut into gridDim.x balanced contiguous slices, one per CTA. A slice that
 // ends inside a segment's overhead units takes no part in that segment: the
@@ -1169,33 +1482,31 @@ struct PageCursor {
   const uint8_t* base;  // pages of the current (b, h)
 };
 
-template <int D>
-__device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p, const int* ustart, int B, int u1,
-                                            int warp) {
+__device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p, const int* ustart, const int* slen,
+                                            int B, int u1, int warp) {
   for (;;) {
     if (c.u < c.e) {
       const int k = c.u - c.first;
       if (k >= 0 && k < c.P) return true;
-      c.u += kWarps;  // overhead units lead a segment, the window / empty unit ends it
+      c.u += kWarps;  // overhead units and the tail unit lead a segment
       continue;
     }
     if (c.e >= u1) return false;
     const int a = c.e;
     const Seg sg = seg_of(ustart, B, p.n_kv_heads, a);
-    c.first = sg.start + p.seg_overhead;
+    c.first = sg.start + p.seg_overhead + 1;
     c.e = min(sg.start + sg.n, u1);
-    c.P = p.len[sg.b] / kPageTokens;
+    c.P = slen[sg.b] / kPageTokens;
     c.base = p.pages + ((int64_t)(sg.b * p.n_kv_heads + sg.h) * p.max_pages) * p.page_bytes;
     c.u = a + warp;
   }
 }
 
-template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
+template <int KB, int VB, int D, bool TOK, bool PT, bool F8, bool AP>
 __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_TOK : Cfg<KB, VB, D, PT, F8>::MINB)
-    decode_mma_kernel(DecodeParams p) {
-  pdl_enter();
+    decode_mma_kernel(const __grid_constant__ DecodeParams p) {
   using C = Cfg<KB, VB, D, PT, F8>;
-  using State = typename std::conditional<TOK, TokState<D>, WarpState<D>>::type;
+  using St = typename std::conditional<TOK, TokState<D>, WarpState<D>>::type;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_last;
   const int H = p.n_kv_heads, G = p.gqa, B = p.batch;
@@ -1203,41 +1514,43 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
   const int g = lane >> 2, t = lane & 3;
   // this lane's query head: row g (head rows) or column head g/2 (token rows)
   const int qh = TOK ? (g >> 1) : g;
-  const float partf = (float)(g & 1);
 
   uint8_t* ring = smem + warp * C::R * C::STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + warp * C::R;
   float* wscr = reinterpret_cast<float*>(smem + C::WSCR_OFF + warp * C::WSCR_STRIDE);
-  uint32_t* qz = reinterpret_cast<uint32_t*>(smem + C::QZ_OFF);
+  uint32_t* qtab = reinterpret_cast<uint32_t*>(smem + C::QZ_OFF);
   float* mo = reinterpret_cast<float*>(smem + C::merge_off(TOK));   // [kWarps][G][D]
   float* mm = mo + kWarps * G * D;                                   // [kWarps][8]
   float* ml = mm + kWarps * kMaxGqa;                                 // [kWarps][8]
   int* ustart = reinterpret_cast<int*>(ml + kWarps * kMaxGqa);       // [B + 1]
+  int* slen = ustart + B + 1;                                        // [B]: lengths before this call's append
   __nv_bfloat16* qbuf = reinterpret_cast<__nv_bfloat16*>(smem + C::qbuf_off(TOK));  // [2][8][D]
   uint64_t* qbars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + kWarps * C::R;
 
-  // ---- units per sequence: exclusive scan (warp 0), n_b = H * max(1, P + (W > 0))
-  if (warp == 0) {
-    int carry = 0;
-    for (int b0 = 0; b0 < B; b0 += 32) {
-      const int bb = b0 + lane;
-      int n = 0;
-      if (bb < B) {
-        const int T = p.len[bb];
-        n = T / kPageTokens + (T % kPageTokens > 0 ? 1 : 0);
-        n = ((n > 0 ? n : 1) + p.seg_overhead) * H;
-      }
-      int x = n;
+  // ---- units per sequence: exclusive scan (warp 0), n_b = H * (V + 1 + P_b)
+  auto scan_units = [&](bool host) {
+    if (warp == 0) {
+      int carry = 0;
+      for (int b0 = 0; b0 < B; b0 += 32) {
+        const int bb = b0 + lane;
+        int n = 0;
+        if (bb < B) {
+          const int T = host ? p.hlen[bb] : p.len[bb];
+          slen[bb] = T;
+          n = (T / kPageTokens + 1 + p.seg_overhead) * H;
+        }
+        int x = n;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (bb < B) ustart[bb] = carry + x - n;
+        carry += __shfl_sync(0xffffffffu, x, 31);
       }
-      if (bb < B) ustart[bb] = carry + x - n;
-      carry += __shfl_sync(0xffffffffu, x, 31);
+      if (lane == 0) ustart[B] = carry;
     }
-    if (lane == 0) ustart[B] = carry;
-  }
+  };
   if (lane == 0) {
     for (int r = 0; r < C::R; ++r) mbar_init(&bars[r], 1);
     if (warp == 0) {
@@ -1246,16 +1559,61 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     }
     mbar_init_fence();
   }
+  // with the lengths in the parameters the slices are known before the wait for
+  // the preceding kernel; otherwise the device lengths are read after it
+  if (p.host_units) scan_units(true);
+  else pdl_enter();
+  if (!p.host_units) scan_units(false);
   __syncthreads();
+  if constexpr (AP) {
+    // device lengths: the last CTA to have read them publishes the new ones
+    // (acquire-release: every CTA's reads are ordered before that write); a full
+    // sequence is left unchanged and the cache's error flag raised
+    if (!p.host_units && threadIdx.x == 0) {
+      if (atomic_add_acq_rel(p.grid_ctr, 1) == (int)gridDim.x - 1) {
+        *p.grid_ctr = 0;
+        for (int b = 0; b < B; ++b)
+          if (slen[b] < p.max_tokens) p.step_len[b] = slen[b] + 1;
+      }
+    }
+  }
   const int N = ustart[B];
   const Slicer sl{N / (int)gridDim.x, N % (int)gridDim.x};
   const int u0 = sl.lo(blockIdx.x), u1 = sl.lo(blockIdx.x + 1);
-  if (u0 >= u1) return;
-  {
+  bool work = u0 < u1;
+  if (work) {
     // nothing to do when the whole slice lies in one segment's overhead units
     const Seg s0 = seg_of(ustart, B, H, u0);
-    if (u1 <= s0.start + p.seg_overhead) return;
+    work = u1 > s0.start + p.seg_overhead;
   }
+
+  // ---- producer: the first R page units of this warp (pages below the lengths
+  // the slices were cut from are never written by the preceding kernel when
+  // `early` is set, so they may stream in under its tail)
+  PageCursor cur;
+  cur.u = u0;  // >= e: the first call looks up the segment of u0
+  cur.e = u0;
+  cur.first = 0;
+  cur.P = 0;
+  cur.base = nullptr;
+  int issued = 0;
+  const uint64_t pol = l2_evict_first_policy();
+  auto issue_first = [&]() {
+    if (lane == 0 && work) {
+      for (int r = 0; r < C::R; ++r) {
+        if (!cursor_next(cur, p, ustart, slen, B, u1, warp)) break;
+        mbar_expect_tx(&bars[r], C::PB);
+        bulk_load_once(ring + r * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes, C::PB, &bars[r],
+                       pol);
+        cur.u += kWarps;
+        ++issued;
+      }
+    }
+  };
+  if (p.host_units && p.early) issue_first();
+  if (p.host_units) pdl_enter();
+  if (!(p.host_units && p.early)) issue_first();
+  if (!work) return;  // no copy was issued
 
   // ---- query rows arrive by bulk copy (the first one ahead of the page stream)
   const uint32_t qbytes = (uint32_t)(G * D * 2);
@@ -1266,26 +1624,6 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
   };
   if (threadIdx.x == 0) issue_q(u0, 0);
 
-  // ---- producer: the first R page units of this warp
-  PageCursor cur;
-  cur.u = u0;  // >= e: the first call looks up the segment of u0
-  cur.e = u0;
-  cur.first = 0;
-  cur.P = 0;
-  cur.base = nullptr;
-  int issued = 0;
-  const uint64_t pol = l2_evict_first_policy();
-  if (lane == 0) {
-    for (int r = 0; r < C::R; ++r) {
-      if (!cursor_next<D>(cur, p, ustart, B, u1, warp)) break;
-      mbar_expect_tx(&bars[r], C::PB);
-      bulk_load_once(ring + r * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes, C::PB, &bars[r],
-                     pol);
-      cur.u += kWarps;
-      ++issued;
-    }
-  }
-
   bool ok = true;
   int consumed = 0;
   int segi = 0;
@@ -1293,13 +1631,32 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     const Seg sg = seg_of(ustart, B, H, a);
     const int e = min(sg.start + sg.n, u1);
     if (e <= sg.start + p.seg_overhead) break;  // overhead units only (the slice's last part)
-    const int T = p.len[sg.b];
-    const int P = T / kPageTokens, W = T % kPageTokens;
-    if (threadIdx.x == 0 && W > 0 && e == sg.start + sg.n) {
-      // this part ends with the bf16 window: bring its W key and W value rows into L2
-      const __nv_bfloat16* w0 = p.window + ((int64_t)(sg.b * H + sg.h) * 2) * kPageTokens * D;
-      prefetch_l2(w0, (uint32_t)(W * D * 2));
-      prefetch_l2(w0 + kPageTokens * D, (uint32_t)(W * D * 2));
+    const int seg = sg.b * H + sg.h;
+    const int T = slen[sg.b];
+    const int P = T / kPageTokens;
+    const int tu = sg.start + p.seg_overhead;  // the tail unit
+    const __nv_bfloat16* win = p.window + ((int64_t)seg * 2) * kPageTokens * D;
+    if (threadIdx.x == 0 && a <= tu && T % kPageTokens > 0) {
+      // this part holds the tail: bring the window's key and value rows into L2
+      prefetch_l2(win, (uint32_t)((T % kPageTokens) * D * 2));
+      prefetch_l2(win + kPageTokens * D, (uint32_t)((T % kPageTokens) * D * 2));
+    }
+    // ---- the tail unit (its warp: the one whose turn it is at unit tu): the
+    // fused step's append happens here, before the query operands are live; its
+    // window, or the page it completed, is attended after the warp's pages
+    int tail_w = 0;          // tokens of the window this warp attends after its pages
+    bool tail_page = false;  // the page the new token completed, attended after the pages
+    if (a <= tu && tu < e && (tu - a) % kWarps == warp) {
+      tail_w = T % kPageTokens;
+      if constexpr (AP) {
+        if (!p.host_units && T >= p.max_tokens) {
+          if (lane == 0 && p.err) atomicExch(p.err, 2);
+        } else {
+          tail_page = append_token<KB, VB, D, PT, F8>(p, seg, sg.h, T, wscr, lane);
+          tail_w = (T + 1) % kPageTokens;
+          if (p.host_units && sg.h == 0 && lane == 0) p.step_len[sg.b] = T + 1;
+        }
+      }
     }
     const bool qvalid = qh < G;
     {
@@ -1311,153 +1668,71 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     const __nv_bfloat16* qrow = qbuf + (segi & 1) * kMaxGqa * D + (qvalid ? qh : 0) * D;
 
     // ---- query operands
-    float qf[D / 4];
-    uint32_t qb[D / 8];   // bf16 pairs (head rows) or bf16 parts (token rows)
-    uint32_t qzb[D / 8];  // token rows: z-term B fragments (q parts); QK B fragments with per-token keys
-    float qsum = 0.f;     // per-token keys: sum_c q'_c of the head this lane scores
-    auto load_qbp = [&]() {
-#pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
-        uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
-        const bool keep = qvalid && (!TOK || (g & 1) == 0);  // q is exact in bf16: low part is zero
-        qb[2 * dt] = keep ? lo : 0u;
-        qb[2 * dt + 1] = keep ? hi : 0u;
-      }
-    };
-    if constexpr (C::kBf16) {
-      load_qbp();
-    } else {
-#pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
-        uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
-        if (!qvalid) lo = hi = 0u;
-        const float2 l2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&lo));
-        const float2 h2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&hi));
-        qf[dt * 4 + 0] = l2.x * p.scale_log2;
-        qf[dt * 4 + 1] = l2.y * p.scale_log2;
-        qf[dt * 4 + 2] = h2.x * p.scale_log2;
-        qf[dt * 4 + 3] = h2.y * p.scale_log2;
-      }
-      // q parts: the z-term B/A operands (per-channel keys) or the QK operands
-      // themselves (per-token keys: the 2-bit tauK channel factor is folded
-      // here; fp8: the KV head's key scale is)
-      const float qlo = F8 ? p.fp8_scales[sg.h] : 1.f;
-      const float qhi = PT ? 1.f / C::tauK : qlo;  // channels 2t+8, 2t+9 of each tile
+    const float ksc = F8 ? p.fp8_scales[sg.h] : 1.f;
+    TokOps<D> tops;
+    HeadOps hops;
+    if constexpr (!C::kBf16) {
       if constexpr (TOK) {
-#pragma unroll
-        for (int dt = 0; dt < C::KS; ++dt) {
-          qzb[2 * dt] = part_f16(qf[dt * 4 + 0] * qlo, qf[dt * 4 + 1] * qlo, partf);
-          qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, partf);
-        }
+        prep_tok_ops<KB, D, PT, F8>(tops, qrow, qvalid, lane, p.scale_log2, ksc);
       } else {
-        if (warp == 0) {
-#pragma unroll
-          for (int dt = 0; dt < C::KS; ++dt) {
-            uint4 q4;
-            split_f16(qf[dt * 4 + 0] * qlo, qf[dt * 4 + 1] * qlo, q4.x, q4.y);
-            split_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, q4.z, q4.w);
-            *reinterpret_cast<uint4*>(qz + (dt * 32 + lane) * 4) = q4;
-          }
-        }
+        prep_head_ops<KB, D, PT, F8>(hops, qtab, warp == 0, qrow, qvalid, lane, p.scale_log2, ksc);
         __syncthreads();
       }
-      if constexpr (PT) {
-        // sum_c q'_c of this lane's query head (its D/4 channels, then the quad)
-        float qs = 0.f;
-#pragma unroll
-        for (int i = 0; i < D / 4; ++i) qs += qf[i];
-        qs += __shfl_xor_sync(0xffffffffu, qs, 1);
-        qs += __shfl_xor_sync(0xffffffffu, qs, 2);
-        // token rows score head t (held by lanes with g = 2t); head rows score head g
-        qsum = TOK ? __shfl_sync(0xffffffffu, qs, 8 * t) : qs;
-      }
     }
+    uint32_t qb[D / 8];   // bf16 q for bf16 pages and the window (loaded when needed)
+    auto load_qbp = [&]() { load_qb<D>(qrow, qvalid && (!TOK || (g & 1) == 0), t, qb); };
+    if constexpr (C::kBf16) load_qbp();
 
-    State st;
-#pragma unroll
-    for (int j = 0; j < (TOK ? D / 16 : D / 8); ++j)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) st.o[j][k] = 0.f;
-    st.m = -INFINITY;
-    st.l = 0.f;
-    st.vz = 0.f;
-    bool converted = C::kBf16;
-    // quantized accumulators to true units: acc * 2^24 (/ sigmaV on channels with
-    // bit 3 set); fp8: acc * the KV head's value scale
-    auto to_true_units = [&]() {
-      if constexpr (F8) {
-        const float vsc = p.fp8_scales[H + sg.h] * kF8Unit;
-#pragma unroll
-        for (int j = 0; j < (TOK ? D / 16 : D / 8); ++j)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) st.o[j][k] *= vsc;
-      } else if constexpr (TOK) {
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          st.o[j][0] *= kTwo24;
-          st.o[j][1] *= kTwo24;
-          st.o[j][2] *= kTwo24 / C::sigmaV;
-          st.o[j][3] *= kTwo24 / C::sigmaV;
-        }
+    St st;
+    state_init(st);
+    auto attend_page = [&](const uint8_t* page) {
+      if constexpr (TOK) {
+        if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, p.scale_log2, lane);
+        else if constexpr (F8) attend_f8page_tok<D>(page, st, tops, lane);
+        else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, tops, wscr, lane);
+        else attend_qpage_tok<KB, VB, D>(page, st, tops, wscr, lane);
       } else {
-#pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-          const float f = (j & 1) ? kTwo24 / C::sigmaV : kTwo24;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) st.o[j][k] *= f;
-        }
+        if constexpr (C::kBf16) attend_bpage<D>(page, st, qb, p.scale_log2, lane);
+        else if constexpr (F8) attend_f8page<D>(page, st, qtab, lane);
+        else if constexpr (PT) attend_qpage_pt<KB, VB, D>(page, st, qtab, hops, wscr, lane);
+        else attend_qpage<KB, VB, D>(page, st, qtab, hops, wscr, lane);
       }
-      converted = true;
     };
 
-    // ---- this warp's units of the segment part [a, e)
+    // ---- this warp's page units of the segment part [a, e)
     for (int u = a + warp; u < e; u += kWarps) {
-      const int k = u - sg.start - p.seg_overhead;
-      if (k < 0) continue;  // overhead unit: no work
-      if (k < P) {
-        if (ok) {
-          const int stage = consumed % C::R;
-          const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
-          if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
-            ok = false;
-          } else {
-            const uint8_t* page = ring + stage * C::STAGE;
-            if constexpr (TOK) {
-              if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
-              else if constexpr (F8) attend_f8page_tok<D>(page, st, qzb, wscr, partf, lane);
-              else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
-              else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
-            } else {
-              if constexpr (C::kBf16) attend_bpage<D>(page, st, qb, p.scale_log2, lane);
-              else if constexpr (F8) attend_f8page<D>(page, st, qz, lane);
-              else if constexpr (PT) attend_qpage_pt<KB, VB, D>(page, st, qz, qsum, wscr, lane);
-              else attend_qpage<KB, VB, D>(page, st, qf, qz, wscr, lane);
-            }
-            ++consumed;
-            __syncwarp();
-            if (lane == 0 && cursor_next<D>(cur, p, ustart, B, u1, warp)) {
-              fence_proxy_async();
-              mbar_expect_tx(&bars[stage], C::PB);
-              bulk_load_once(ring + stage * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes,
-                             C::PB, &bars[stage], pol);
-              cur.u += kWarps;
-              ++issued;
-            }
+      const int k = u - tu - 1;
+      if (k < 0) continue;  // overhead units and the tail unit
+      if (k < P && ok) {
+        const int stage = consumed % C::R;
+        const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
+        if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
+          ok = false;
+        } else {
+          attend_page(ring + stage * C::STAGE);
+          ++consumed;
+          __syncwarp();
+          if (lane == 0 && cursor_next(cur, p, ustart, slen, B, u1, warp)) {
+            fence_proxy_async();
+            mbar_expect_tx(&bars[stage], C::PB);
+            bulk_load_once(ring + stage * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes, C::PB,
+                           &bars[stage], pol);
+            cur.u += kWarps;
+            ++issued;
           }
         }
-      } else if (W > 0) {
-        if constexpr (!C::kBf16) {
-          to_true_units();
-          load_qbp();
-        }
-        const __nv_bfloat16* win = p.window + ((int64_t)(sg.b * H + sg.h) * 2) * kPageTokens * D;
-        if constexpr (TOK) attend_window_tok<D>(win, W, st, qb, wscr, partf, p.scale_log2, lane);
-        else attend_window<D>(win, W, st, qb, p.scale_log2, lane);
       }
     }
-    if (!converted) to_true_units();
+    if (tail_page) {
+      // the page this warp has just written (generic loads: it never went through the async proxy)
+      attend_page(p.pages + ((int64_t)seg * p.max_pages + P) * p.page_bytes);
+    }
+    to_true_units<VB, TOK, F8>(st, F8 ? p.fp8_scales[H + sg.h] : 1.f);
+    if (tail_w > 0) {
+      if constexpr (!C::kBf16) load_qbp();
+      if constexpr (TOK) attend_window_tok<D>(win, tail_w, st, qb, p.scale_log2, lane);
+      else attend_window<D>(win, tail_w, st, qb, p.scale_log2, lane);
+    }
 
     // ---- warps -> shared memory, CTA merge
     if constexpr (TOK) {
@@ -1498,8 +1773,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
       }
     }
     __syncthreads();
-    const int seg = sg.b * H + sg.h;
-    const bool whole = (a <= sg.start + p.seg_overhead) && (e == sg.start + sg.n);
+    const bool whole = (a <= tu) && (e == sg.start + sg.n);
     float* outp = p.out + (int64_t)seg * G * D;
     float* part = p.partials + ((int64_t)blockIdx.x * 2 + (a == u0 ? 0 : 1)) * split_record_floats(G, D);
     for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
@@ -1529,7 +1803,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     if (!whole) {
       // The last CTA of a split segment merges the slices' partials in slice
       // order (empty slices, possible when CTAs outnumber units, hold nothing).
-      const int c_lo = sl.cta_of(sg.start + p.seg_overhead), c_hi = sl.cta_of(sg.start + sg.n - 1);
+      const int c_lo = sl.cta_of(tu), c_hi = sl.cta_of(sg.start + sg.n - 1);
       __syncthreads();  // this CTA's partial record is complete
       if (threadIdx.x == 0) {
         int parts = 0;
@@ -1567,7 +1841,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
         }
       }
     }
-    __syncthreads();  // merge area, qz and s_last are reused by the next segment
+    __syncthreads();  // merge area, query table and s_last are reused by the next segment
     a = e;
   }
 
@@ -1576,189 +1850,6 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     // (each wait bounded again) before this CTA's shared memory goes away
     if (lane == 0 && p.err) atomicExch(p.err, 1);
     for (int i = consumed; i < issued; ++i) mbar_wait(&bars[i % C::R], (uint32_t)((i / C::R) & 1));
-  }
-}
-
-// ------------------------------------------------------------ fused append --
-// Warp-level flush of one completed 32-token group (the window's 31 tokens and
-// the new token) into `page`, bit-identical to the append kernel's CTA-wide
-// flush: the same quantizer and packing (kvq_quant.cuh), only the work split
-// differs. `scr` is this warp's ring (free at a segment's start) and holds the
-// codes as bytes, [2][32][D] (bf16 layers: the rows themselves), before they
-// are packed in fragment order.
-template <int BITS, int D, typename Get>
-__device__ __forceinline__ void pack_block_warp(uint8_t* blk, bool is_value, int lane, Get vals) {
-  constexpr int kPerLane = (int)(code_block_bytes(BITS, D) / 16) / 32;  // 16-byte vectors per lane
-#pragma unroll 1
-  for (int vi = 0; vi < kPerLane; ++vi) {
-    uint4 q;
-    q.x = lane_word<BITS>(lane, 4 * vi + 0, is_value, vals);
-    q.y = lane_word<BITS>(lane, 4 * vi + 1, is_value, vals);
-    q.z = lane_word<BITS>(lane, 4 * vi + 2, is_value, vals);
-    q.w = lane_word<BITS>(lane, 4 * vi + 3, is_value, vals);
-    reinterpret_cast<uint4*>(blk)[vi * 32 + lane] = q;
-  }
-}
-
-template <int KB, int VB, int D, bool PT, bool F8>
-__device__ __noinline__ void warp_flush(uint8_t* page, const __nv_bfloat16* win, const __nv_bfloat16* kn,
-                                        const __nv_bfloat16* vn, uint8_t* scr, float ksc, float vsc,
-                                        double* err_stats, int lane) {
-  // row of token tok (0..31) of keys (r = 0) or values (r = 1)
-  auto row = [&](int r, int tok) -> const __nv_bfloat16* {
-    return tok < kPageTokens - 1 ? win + (r * kPageTokens + tok) * D : (r ? vn : kn);
-  };
-  if constexpr (KB == 16) {
-    // bf16 layer: stage the 32 rows of keys and values, then pack their bit patterns
-    uint16_t* sb = reinterpret_cast<uint16_t*>(scr);  // [2][32][D]
-#pragma unroll 1
-    for (int i = lane; i < 2 * kPageTokens * D / 8; i += 32) {
-      const int r = i / (kPageTokens * D / 8), rem = i % (kPageTokens * D / 8);
-      const int tok = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
-      *reinterpret_cast<uint4*>(sb + (r * kPageTokens + tok) * D + c8) =
-          *reinterpret_cast<const uint4*>(row(r, tok) + c8);
-    }
-    __syncwarp();
-    pack_block_warp<16, D>(page, false, lane, [&](int tok, int dim) { return (uint32_t)sb[tok * D + dim]; });
-    pack_block_warp<16, D>(page + code_block_bytes(16, D), true, lane,
-                           [&](int tok, int dim) { return (uint32_t)sb[(kPageTokens + tok) * D + dim]; });
-    return;
-  } else {
-    uint8_t* cs = scr;  // [2][32][D] codes
-    double err[4] = {0.0, 0.0, 0.0, 0.0};
-    auto add_err = [&](int r, float x, double xh) {
-      const double dx = (double)x - xh;
-      err[2 * r] += dx * dx;
-      err[2 * r + 1] += (double)x * (double)x;
-    };
-    if constexpr (F8) {
-      // lane = token: every element is e4m3(x / s_h) of its KV head's scale
-#pragma unroll 1
-      for (int r = 0; r < 2; ++r) {
-        const float sc = r ? vsc : ksc;
-        const __nv_bfloat16* src = row(r, lane);
-#pragma unroll 1
-        for (int c8 = 0; c8 < D; c8 += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
-          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-          uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float x = __bfloat162float(xv[j]);
-            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(__fdiv_rn(x, sc), __NV_SATFINITE, __NV_E4M3);
-            packed[j >> 2] |= (uint32_t)c << (8 * (j & 3));
-            add_err(r, x, (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3))) * sc);
-          }
-          *reinterpret_cast<uint2*>(cs + (r * kPageTokens + lane) * D + c8) = make_uint2(packed[0], packed[1]);
-        }
-      }
-      __syncwarp();
-      pack_block_warp<8, D>(page, false, lane, [&](int tok, int dim) { return (uint32_t)cs[tok * D + dim]; });
-      pack_block_warp<8, D>(page + code_block_bytes(8, D), true, lane,
-                            [&](int tok, int dim) { return (uint32_t)cs[(kPageTokens + tok) * D + dim]; });
-    } else {
-      constexpr int nk = PT ? kPageTokens : D;  // key scale/zero pairs
-      uint8_t* vblk = page + code_block_bytes(KB, D);
-      __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
-      __half* kzero = kscale + nk;
-      __half* vscale = kzero + nk;
-      __half* vzero = vscale + kPageTokens;
-      // per token over head_dim (values; keys in per-token mode): lane = token
-      auto per_token = [&](int r, int qmax, __half* sdst, __half* zdst) {
-        const __nv_bfloat16* src = row(r, lane);
-        float mn = INFINITY, mx = -INFINITY;
-#pragma unroll 1
-        for (int c8 = 0; c8 < D; c8 += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
-          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float x = __bfloat162float(xv[j]);
-            mn = fminf(mn, x);
-            mx = fmaxf(mx, x);
-          }
-        }
-        const QParams q = make_qparams(mn, mx, qmax);
-        const double s = (double)__half2float(q.s_h), z = (double)q.z;
-#pragma unroll 1
-        for (int c8 = 0; c8 < D; c8 += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + c8);
-          const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-          uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float x = __bfloat162float(xv[j]);
-            const uint32_t c = quant_code(x, q, qmax);
-            packed[j >> 2] |= c << (8 * (j & 3));
-            add_err(r, x, (double)c * s + z);
-          }
-          *reinterpret_cast<uint2*>(cs + (r * kPageTokens + lane) * D + c8) = make_uint2(packed[0], packed[1]);
-        }
-        sdst[lane] = q.s_h;
-        zdst[lane] = q.z_h;
-      };
-      if constexpr (PT) {
-        per_token(0, (1 << KB) - 1, kscale, kzero);
-      } else {
-        // keys per channel over the 32 tokens: lane owns channels lane * NC .. + NC - 1
-        constexpr int NC = D / 32;
-        constexpr int qmax = (1 << KB) - 1;
-        const int c0 = lane * NC;
-        float mn[NC], mx[NC];
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          mn[j] = INFINITY;
-          mx[j] = -INFINITY;
-        }
-#pragma unroll 1
-        for (int tok = 0; tok < kPageTokens; ++tok) {
-          const __nv_bfloat16* src = row(0, tok) + c0;
-#pragma unroll
-          for (int j = 0; j < NC; ++j) {
-            const float x = __bfloat162float(src[j]);
-            mn[j] = fminf(mn[j], x);
-            mx[j] = fmaxf(mx[j], x);
-          }
-        }
-        QParams q[NC];
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          q[j] = make_qparams(mn[j], mx[j], qmax);
-          const int slot = kmeta_slot<D>(c0 + j);
-          kscale[slot] = q[j].s_h;
-          kzero[slot] = q[j].z_h;
-        }
-#pragma unroll 1
-        for (int tok = 0; tok < kPageTokens; ++tok) {
-          const __nv_bfloat16* src = row(0, tok) + c0;
-#pragma unroll
-          for (int j = 0; j < NC; ++j) {
-            const float x = __bfloat162float(src[j]);
-            const uint32_t c = quant_code(x, q[j], qmax);
-            cs[tok * D + c0 + j] = (uint8_t)c;
-            add_err(0, x, (double)c * (double)__half2float(q[j].s_h) + (double)q[j].z);
-          }
-        }
-      }
-      per_token(1, (1 << VB) - 1, vscale, vzero);
-      __syncwarp();
-      pack_block_warp<KB, D>(page, false, lane, [&](int tok, int dim) { return (uint32_t)cs[tok * D + dim]; });
-      pack_block_warp<VB, D>(vblk, true, lane,
-                             [&](int tok, int dim) { return (uint32_t)cs[(kPageTokens + tok) * D + dim]; });
-    }
-    // this flush's error sums: warp shuffles, then one fp64 atomic per sum
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      double v = err[i];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      err[i] = v;
-    }
-    if (err_stats && lane == 0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) atomicAdd(&err_stats[i], err[i]);
-      atomicAdd(&err_stats[4], (double)(kPageTokens * D));
-    }
   }
 }
 
@@ -1787,17 +1878,15 @@ struct WarpCfg {
 // acquire-release increment orders every read before that write).
 template <int KB, int VB, int D, bool PT, bool F8, bool AP = false>
 __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
-    decode_warp_kernel(DecodeParams p) {
+    decode_warp_kernel(const __grid_constant__ DecodeParams p) {
   pdl_enter();
   using C = Cfg<KB, VB, D, PT, F8>;
   using WC = WarpCfg<KB, VB, D, PT, F8>;
-  static_assert(C::R * C::STAGE >= 2 * kPageTokens * D * (C::kBf16 ? 2 : 1), "flush scratch fits the warp's ring");
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = p.n_kv_heads, G = p.gqa;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int qh = g >> 1;  // column head of this lane
-  const float partf = (float)(g & 1);
   uint8_t* ring = smem + warp * C::R * C::STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WC::MBAR_OFF) + warp * (C::R + 1);
   uint64_t* qbar = bars + C::R;
@@ -1832,24 +1921,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
       P = t0 / kPageTokens;
       if (t0 < p.max_tokens) {
         T = t0 + 1;
-        __nv_bfloat16* wwin = p.step_window + ((int64_t)s * 2) * kPageTokens * D;
-        const __nv_bfloat16* kn = p.k_new + (int64_t)s * D;
-        const __nv_bfloat16* vn = p.v_new + (int64_t)s * D;
-        if (T % kPageTokens != 0) {
-          // the new token into window slot t0 mod 32
-          const int slot = t0 % kPageTokens;
-          for (int d = 2 * lane; d < D; d += 64) {
-            *reinterpret_cast<uint32_t*>(wwin + slot * D + d) = *reinterpret_cast<const uint32_t*>(kn + d);
-            *reinterpret_cast<uint32_t*>(wwin + (kPageTokens + slot) * D + d) =
-                *reinterpret_cast<const uint32_t*>(vn + d);
-          }
-        } else {
-          flushed = true;
-          warp_flush<KB, VB, D, PT, F8>(p.step_pages + ((int64_t)s * p.max_pages + P) * p.page_bytes, wwin, kn, vn,
-                                        ring, F8 ? p.fp8_scales[h] : 1.f, F8 ? p.fp8_scales[H + h] : 1.f,
-                                        p.err_stats, lane);
-        }
-        __syncwarp();  // the window row or page and the ring scratch are complete for every lane
+        flushed = append_token<KB, VB, D, PT, F8>(p, s, h, t0, wscr, lane);
       } else {
         T = t0;  // a full sequence is left unchanged and the cache's error flag raised
         if (lane == 0 && p.err) atomicExch(p.err, 2);
@@ -1887,80 +1959,20 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
     }
     const bool qvalid = qh < G;
     const __nv_bfloat16* qrow = qslot + (qvalid ? qh : 0) * D;
-    float qf[D / 4];
+    TokOps<D> tops;
+    if constexpr (!C::kBf16) prep_tok_ops<KB, D, PT, F8>(tops, qrow, qvalid, lane, p.scale_log2, F8 ? p.fp8_scales[h] : 1.f);
     uint32_t qb[D / 8];
-    uint32_t qzb[D / 8];
-    float qsum = 0.f;
-    auto load_qbp = [&]() {
-#pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        const uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
-        const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
-        const bool keep = qvalid && (g & 1) == 0;  // q is exact in bf16: its low part is zero
-        qb[2 * dt] = keep ? lo : 0u;
-        qb[2 * dt + 1] = keep ? hi : 0u;
-      }
-    };
-    if constexpr (C::kBf16) {
-      load_qbp();
-    } else {
-#pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t);
-        uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * dt + 2 * t + 8);
-        if (!qvalid) lo = hi = 0u;
-        const float2 l2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&lo));
-        const float2 h2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&hi));
-        qf[dt * 4 + 0] = l2.x * p.scale_log2;
-        qf[dt * 4 + 1] = l2.y * p.scale_log2;
-        qf[dt * 4 + 2] = h2.x * p.scale_log2;
-        qf[dt * 4 + 3] = h2.y * p.scale_log2;
-      }
-      const float qlo = F8 ? p.fp8_scales[h] : 1.f;
-      const float qhi = PT ? 1.f / C::tauK : qlo;
-#pragma unroll
-      for (int dt = 0; dt < C::KS; ++dt) {
-        qzb[2 * dt] = part_f16(qf[dt * 4 + 0] * qlo, qf[dt * 4 + 1] * qlo, partf);
-        qzb[2 * dt + 1] = part_f16(qf[dt * 4 + 2] * qhi, qf[dt * 4 + 3] * qhi, partf);
-      }
-      if constexpr (PT) {
-        float qs = 0.f;
-#pragma unroll
-        for (int i = 0; i < D / 4; ++i) qs += qf[i];
-        qs += __shfl_xor_sync(0xffffffffu, qs, 1);
-        qs += __shfl_xor_sync(0xffffffffu, qs, 2);
-        qsum = __shfl_sync(0xffffffffu, qs, 8 * t);
-      }
-    }
+    auto load_qbp = [&]() { load_qb<D>(qrow, qvalid && (g & 1) == 0, t, qb); };
+    if constexpr (C::kBf16) load_qbp();
 
     TokState<D> st;
-#pragma unroll
-    for (int j = 0; j < D / 16; ++j)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) st.o[j][k] = 0.f;
-    st.m = -INFINITY;
-    st.l = 0.f;
-    st.vz = 0.f;
-    bool converted = C::kBf16;
-    auto to_true_units = [&]() {
-      if constexpr (F8) {
-        const float vsc = p.fp8_scales[H + h] * kF8Unit;
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) st.o[j][k] *= vsc;
-      } else if constexpr (!C::kBf16) {
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          st.o[j][0] *= kTwo24;
-          st.o[j][1] *= kTwo24;
-          st.o[j][2] *= kTwo24 / C::sigmaV;
-          st.o[j][3] *= kTwo24 / C::sigmaV;
-        }
-      }
-      converted = true;
+    state_init(st);
+    auto attend_page = [&](const uint8_t* page) {
+      if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, p.scale_log2, lane);
+      else if constexpr (F8) attend_f8page_tok<D>(page, st, tops, lane);
+      else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, tops, wscr, lane);
+      else attend_qpage_tok<KB, VB, D>(page, st, tops, wscr, lane);
     };
-
     for (int k = 0; k < P; ++k) {
       const int stage = consumed % C::R;
       const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
@@ -1968,11 +1980,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
         ok = false;
         break;
       }
-      const uint8_t* page = ring + stage * C::STAGE;
-      if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
-      else if constexpr (F8) attend_f8page_tok<D>(page, st, qzb, wscr, partf, lane);
-      else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
-      else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
+      attend_page(ring + stage * C::STAGE);
       ++consumed;
       __syncwarp();
       if (next < P) {
@@ -1986,22 +1994,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
       }
     }
     if (!ok) break;
-    if (flushed) {
-      // the page this warp has just written (generic loads: it never went through the async proxy)
-      const uint8_t* page = base + (int64_t)P * p.page_bytes;
-      if constexpr (C::kBf16) attend_bpage_tok<D>(page, st, qb, wscr, partf, p.scale_log2, lane);
-      else if constexpr (F8) attend_f8page_tok<D>(page, st, qzb, wscr, partf, lane);
-      else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, qzb, qsum, wscr, partf, lane);
-      else attend_qpage_tok<KB, VB, D>(page, st, qf, qzb, wscr, partf, lane);
-    }
+    // the page this warp has just written (generic loads: it never went through the async proxy)
+    if (flushed) attend_page(base + (int64_t)P * p.page_bytes);
+    to_true_units<VB, true, F8>(st, F8 ? p.fp8_scales[H + h] : 1.f);
     if (W > 0) {
-      if constexpr (!C::kBf16) {
-        to_true_units();
-        load_qbp();
-      }
-      attend_window_tok<D>(win, W, st, qb, wscr, partf, p.scale_log2, lane);
+      if constexpr (!C::kBf16) load_qbp();
+      attend_window_tok<D>(win, W, st, qb, p.scale_log2, lane);
     }
-    if (!converted) to_true_units();
 
     // head t's sum over the warp's tokens, then the output rows of this segment
     float l = st.l, vz = st.vz;
@@ -2031,43 +2030,46 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
   }
 }
 
-template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
-cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
-  using C = Cfg<KB, VB, D, PT, F8>;
-  if constexpr (TOK) {
-    // short sequences: one warp per segment when every segment fits in one resident wave
-    if (p.warp_split) {
-      using WC = WarpCfg<KB, VB, D, PT, F8>;
-      static bool configured = false;
-      static int occ_w = 0;
-      if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM);
-        if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_w, decode_warp_kernel<KB, VB, D, PT, F8>, kThreads,
-                                                          WC::SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-      }
-      const int64_t segs = (int64_t)p.batch * p.n_kv_heads;
-      const int64_t ctas = (segs + kWarps - 1) / kWarps;
-      if (ctas >= 1 && ctas <= (int64_t)occ_w * p.sm_count)
-        return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8>, dim3((unsigned)ctas), dim3(kThreads),
-                          (size_t)WC::SMEM, s, p);
-    }
+// ---------------------------------------------------------------- launchers --
+// One warp per segment when every segment fits one resident wave of warps;
+// cudaErrorNotSupported (nothing launched) otherwise.
+template <int KB, int VB, int D, bool PT, bool F8, bool AP>
+cudaError_t launch_warp(const DecodeParams& p, cudaStream_t s) {
+  using WC = WarpCfg<KB, VB, D, PT, F8>;
+  static bool configured = false;
+  static int occ = 0;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8, AP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_warp_kernel<KB, VB, D, PT, F8, AP>, kThreads,
+                                                      WC::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
   }
+  const int64_t ctas = ((int64_t)p.batch * p.n_kv_heads + kWarps - 1) / kWarps;
+  if (ctas < 1 || ctas > (int64_t)occ * p.sm_count) return cudaErrorNotSupported;
+  return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8, AP>, dim3((unsigned)ctas), dim3(kThreads),
+                    (size_t)WC::SMEM, s, p);
+}
+
+// The shared split: resident CTAs per SM x SMs, capped by the units and the
+// split-record slots.
+template <int KB, int VB, int D, bool TOK, bool PT, bool F8, bool AP>
+cudaError_t launch_shared(const DecodeParams& p, cudaStream_t s) {
+  using C = Cfg<KB, VB, D, PT, F8>;
   static int configured_smem = 0;
   static int occ_smem = -1, occ_blocks = 0;
   const int smem = C::smem_bytes(TOK, p.gqa, p.batch);
   if (smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK, PT, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<KB, VB, D, TOK, PT, F8, AP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured_smem = smem;
   }
   if (smem != occ_smem) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_blocks, decode_mma_kernel<KB, VB, D, TOK, PT, F8>,
-                                                                  kThreads, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &occ_blocks, decode_mma_kernel<KB, VB, D, TOK, PT, F8, AP>, kThreads, smem);
     if (e != cudaSuccess) return e;
     occ_smem = smem;
   }
@@ -2075,8 +2077,21 @@ cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
   grid = std::min<int64_t>(grid, p.n_units);
   grid = std::min<int64_t>(grid, p.max_ctas);
   if (grid < 1) grid = 1;
-  return launch_pdl(decode_mma_kernel<KB, VB, D, TOK, PT, F8>, dim3((unsigned)grid), dim3(kThreads), (size_t)smem, s,
-                    p);
+  return launch_pdl(decode_mma_kernel<KB, VB, D, TOK, PT, F8, AP>, dim3((unsigned)grid), dim3(kThreads),
+                    (size_t)smem, s, p);
+}
+
+template <int KB, int VB, int D, bool TOK, bool PT, bool F8>
+cudaError_t launch4(const DecodeParams& p, cudaStream_t s) {
+  if constexpr (TOK) {
+    if (p.warp_split) {
+      const cudaError_t e =
+          p.append ? launch_warp<KB, VB, D, PT, F8, true>(p, s) : launch_warp<KB, VB, D, PT, F8, false>(p, s);
+      if (e != cudaErrorNotSupported) return e;
+    }
+  }
+  return p.append ? launch_shared<KB, VB, D, TOK, PT, F8, true>(p, s)
+                  : launch_shared<KB, VB, D, TOK, PT, F8, false>(p, s);
 }
 
 template <int KB, int VB, int D>
@@ -2105,63 +2120,11 @@ cudaError_t launch_d(int kb, int vb, const DecodeParams& p, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
-// fused append + decode (one warp per segment); not launched when the segments
-// do not fit one resident wave of warps
-template <int KB, int VB, int D, bool PT, bool F8>
-cudaError_t launch_step4(const DecodeParams& p, cudaStream_t s) {
-  using WC = WarpCfg<KB, VB, D, PT, F8>;
-  static bool configured = false;
-  static int occ = 0;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_warp_kernel<KB, VB, D, PT, F8, true>, kThreads,
-                                                      WC::SMEM);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  const int64_t ctas = ((int64_t)p.batch * p.n_kv_heads + kWarps - 1) / kWarps;
-  if (ctas < 1 || ctas > (int64_t)occ * p.sm_count) return cudaErrorNotSupported;
-  return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8, true>, dim3((unsigned)ctas), dim3(kThreads),
-                    (size_t)WC::SMEM, s, p);
-}
-
-template <int KB, int VB, int D>
-cudaError_t launch_step3(const DecodeParams& p, cudaStream_t s) {
-  if (p.gqa > 4) return cudaErrorNotSupported;
-  if constexpr (KB == 8 && VB == 8) {
-    if (p.fmt != 0) return launch_step4<KB, VB, D, false, true>(p, s);
-  }
-  if constexpr (KB != 16) {
-    if (p.key_mode != 0) return launch_step4<KB, VB, D, true, false>(p, s);
-  }
-  return launch_step4<KB, VB, D, false, false>(p, s);
-}
-
-template <int D>
-cudaError_t launch_step_d(int kb, int vb, const DecodeParams& p, cudaStream_t s) {
-#define KVQ_PAIR(K_, V_) \
-  if (kb == K_ && vb == V_) return launch_step3<K_, V_, D>(p, s);
-  KVQ_PAIR(2, 2) KVQ_PAIR(2, 4) KVQ_PAIR(2, 8)
-  KVQ_PAIR(4, 2) KVQ_PAIR(4, 4) KVQ_PAIR(4, 8)
-  KVQ_PAIR(8, 2) KVQ_PAIR(8, 4) KVQ_PAIR(8, 8)
-  KVQ_PAIR(16, 16)
-#undef KVQ_PAIR
-  return cudaErrorInvalidValue;
-}
-
 }  // namespace
 
 cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s) {
   if (D == 64) return launch_d<64>(kb, vb, p, s);
   if (D == 128) return launch_d<128>(kb, vb, p, s);
-  return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_decode_step(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s) {
-  if (D == 64) return launch_step_d<64>(kb, vb, p, s);
-  if (D == 128) return launch_step_d<128>(kb, vb, p, s);
   return cudaErrorInvalidValue;
 }
 

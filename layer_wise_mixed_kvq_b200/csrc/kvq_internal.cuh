@@ -28,6 +28,16 @@ namespace kvq {
 constexpr int kPageTokens = 32;   // key group size = tokens per page = window capacity
 constexpr int kMaxBatch = 1024;
 constexpr int kMaxGqa = 8;
+constexpr int kHostLens = 256;    // sequences whose lengths a decode launch can carry in its parameters
+// Per-layer quantization error report: kErrBins bins of kErrStride doubles (one
+// 128-byte line each), every flush adding into one bin, so concurrent flushes
+// seldom update the same address; the report is the sum over bins.
+constexpr int kErrBins = 64;
+constexpr int kErrStride = 16;
+
+__host__ __device__ inline double* err_bin(double* base, unsigned key) {
+  return base ? base + (key % kErrBins) * kErrStride : nullptr;
+}
 
 __host__ __device__ constexpr int64_t code_block_bytes(int bits, int D) { return 4LL * D * bits; }
 
@@ -45,7 +55,7 @@ __host__ __device__ constexpr int split_record_floats(int G, int D) { return G *
 struct LayerState {
   int kb = 0, vb = 0, km = 0, fmt = 0;
   float* fp8_scales = nullptr;   // fp8 layers: [2][n_kv_heads] key then value scales (device)
-  double* err_stats = nullptr;   // [4] sums (k-k^)^2, k^2, (v-v^)^2, v^2, then [1] element count (device)
+  double* err_stats = nullptr;   // [kErrBins][kErrStride]: sums (k-k^)^2, k^2, (v-v^)^2, v^2, element count
   int64_t page_bytes = 0;
   uint8_t* pages = nullptr;
   __nv_bfloat16* window = nullptr;
@@ -89,7 +99,7 @@ struct DecodeParams {
   int batch;             // sequences b < batch are attended
   int chunk;             // CUDA-core kernel: pages per split
   int splits_stride;     // CUDA-core kernel: partial slots per (b, h)
-  int n_units;           // tensor-core kernel: total units (pages + window/empty units), host view
+  int n_units;           // tensor-core kernel: total units (host view; an upper bound with device lengths)
   int max_ctas;          // tensor-core kernel: CTAs the partial buffer can serve (2 split records each)
   int sm_count;
   int seg_overhead;      // tensor-core kernel: overhead units leading each segment (>= 0)
@@ -100,16 +110,25 @@ struct DecodeParams {
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
   int warp_split;        // tensor-core kernel, G <= 4: one warp per segment (if the segments fit the
                          // resident warps) instead of CTAs sharing each segment's pages
-  // fused decode step (kvq_decode_step): the warp attending segment (b, h) first
-  // appends that segment's new token; the same buffers as above, writable
+  // fused decode step (kvq_decode_step): the warp that owns segment (b, h)'s tail
+  // unit first appends that segment's new token; the same buffers as above, writable
+  int append;
   uint8_t* step_pages;
   __nv_bfloat16* step_window;
   int32_t* step_len;
-  int32_t* append_ctr;           // [batch], zero between launches
+  int32_t* append_ctr;           // warp split: [batch], zero between launches
+  int32_t* grid_ctr;             // shared split with device lengths: one int, zero between launches
   const __nv_bfloat16* k_new;    // [batch][n_kv_heads][head_dim]
   const __nv_bfloat16* v_new;
   double* err_stats;
   int max_tokens;
+  // shared split: the lengths (before this call's append) come from hlen instead of
+  // a scan of `len` on the device; with `early` the first page copies are issued
+  // before the wait for the preceding kernel (pages below those lengths are not
+  // written by it)
+  int host_units;
+  int early;
+  int32_t hlen[kHostLens];
 };
 
 // Programmatic dependent launch. Every kernel of the library starts with
@@ -159,7 +178,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t launch_append(int kb, int vb, int D, kvq_dtype dtype, const AppendParams& p, dim3 grid,
                           cudaStream_t s);
 cudaError_t launch_decode_simt(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
-// Grid chosen inside: resident CTAs x SMs, capped by n_units and max_ctas.
+// Grid chosen inside: one warp per segment when p.warp_split and the segments fit
+// one resident wave, else resident CTAs x SMs capped by n_units and max_ctas.
 cudaError_t launch_decode_mma(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s);
 // Pages per split-K CTA for a layer-step: about 3 CTAs per SM, at least 8 pages
 // (2 per warp) per CTA, and no more than `stride` splits per (sequence, head).
@@ -172,12 +192,9 @@ void set_last_error(const std::string& msg);
 // KVQ_DECODE_KERNEL=simt: the CUDA-core decode kernel instead of the tensor-core one.
 bool decode_uses_simt();
 
-// Layer-map dispatcher: the kernel instance for a layer's pair.
+// Layer-map dispatcher: the kernel instance for a layer's pair (p.append = 1:
+// the fused one-token append + decode attention of kvq_decode_step).
 cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 grid, cudaStream_t s);
-// Fused one-token append + decode attention with one warp per segment (query
-// groups of at most 4 heads). cudaErrorNotSupported when the segments do not fit
-// the resident warps (nothing launched: the caller runs the two kernels).
-cudaError_t launch_decode_step(int kb, int vb, int D, const DecodeParams& p, cudaStream_t s);
 
 }  // namespace kvq
 
@@ -192,6 +209,7 @@ struct kvq_cache {
   int32_t* merge_ctr = nullptr;
   int32_t* append_ctr = nullptr;
   int32_t* err = nullptr;            // device flag raised by a decode wait that gave up
+  int32_t* grid_ctr = nullptr;       // fused step with device lengths: elects the CTA publishing lengths
   int32_t* plan_dev = nullptr;
   int32_t* plan_host = nullptr;      // pinned
   cudaEvent_t plan_done = nullptr;
@@ -202,4 +220,16 @@ struct kvq_cache {
   int split_pages = 0;
   int warp_pages = -1;               // kvq_set_decode_mode: -1 automatic, 0 never, n > 0 up to n pages
   int64_t launches = 0;
+  // Streams this cache launched on, each with the layer its latest launch wrote
+  // (-1: none, -2: every layer): a decode may stream pages in under the tail of
+  // the preceding kernel unless that kernel is one of ours writing the same layer.
+  struct StreamWrite {
+    void* stream;
+    int layer;
+  };
+  std::vector<StreamWrite> stream_writes;
+  bool stream_table_full = false;
+  // A CUDA graph was captured: its replays change the device lengths without the
+  // host, so launches read the device lengths until kvq_refresh_lengths.
+  bool graph_captured = false;
 };

@@ -29,8 +29,10 @@ namespace {
 constexpr size_t kScratchBytes = 16u << 20;  // 16 MiB per device
 constexpr int kMaxDevices = 64;
 
-// Split-K scratch: merge counters first, then (acc, m, l) partial records.
+// Split-K scratch: an error word (in its own 256-byte slot), the merge counters,
+// then (acc, m, l) partial records.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
+constexpr size_t kErrSlot = 256;
 
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
@@ -87,28 +89,30 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
 
   const int G = n_q_heads / n_kv_heads;
   const int64_t pairs = (int64_t)batch * n_kv_heads;
-  const size_t ctr_bytes = ((size_t)pairs * 4 + 255) / 256 * 256;
+  const size_t ctr_bytes = kErrSlot + ((size_t)pairs * 4 + 255) / 256 * 256;  // error word + merge counters
   const size_t rec_bytes = (size_t)G * (head_dim + 2) * 4;  // one split-K record (acc, m, l)
   if (ctr_bytes + 2 * rec_bytes > kScratchBytes)
     return fail(KVQ_ECAPACITY, "batch * n_kv_heads merge counters (4 bytes each) leave no room for split records "
                                "in the 16 MiB static scratch; use fewer sequences per call");
   const int64_t records = (int64_t)((kScratchBytes - ctr_bytes) / rec_bytes);
+  const int64_t max_p = max_seq_len / kvq::kPageTokens;
+  const int64_t n_units = pairs * (max_p + 1 + kvq::seg_overhead_units());
+  if (n_units > INT32_MAX) return fail(KVQ_EINVAL, "too many pages in one call");
 
   void* base = nullptr;
   kvq_status st = scratch_address(&base);
   if (st != KVQ_OK) return st;
-  int32_t* ctr = static_cast<int32_t*>(base);
+  int32_t* err = static_cast<int32_t*>(base);
+  int32_t* ctr = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + kErrSlot);
   float* partials = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + ctr_bytes);
 
   // same split policy as kvq_decode_attn, sized from the caller's length bound
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t max_p = max_seq_len / kvq::kPageTokens;
   const int64_t stride = records / pairs;  // CUDA-core kernel: records per (sequence, head)
   const int64_t chunk = stride >= 1 ? kvq::choose_chunk(sms, max_p * pairs, max_p, stride) : max_p + 1;
   const int splits = max_p > 0 ? (int)((max_p + chunk - 1) / chunk) : 1;
-  const int64_t n_units = pairs * (max_p + 1 + kvq::seg_overhead_units());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the merge counters must start at zero; the array keeps the last call's contents
   cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)pairs * 4, s);
@@ -130,7 +134,8 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.chunk = (int)chunk;
   p.splits_stride = (int)std::max<int64_t>(stride, 1);
   p.batch = batch;
-  p.n_units = (int)std::min<int64_t>(n_units, INT32_MAX);
+  p.n_units = (int)n_units;
+  p.err = err;
   p.max_ctas = (int)std::min<int64_t>(
       (int64_t)((kScratchBytes - ctr_bytes) / ((size_t)kvq::split_record_floats(G, head_dim) * 4)) / 2, INT32_MAX);
   p.sm_count = sms;
@@ -138,5 +143,20 @@ extern "C" kvq_status kvq_decode_attn_noalloc(kvq_pair pair, int head_dim, int n
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   e = kvq::launch_decode(pair.k_bits, pair.v_bits, head_dim, p, dim3(splits, n_kv_heads, batch), s);
   if (e != cudaSuccess) return fail(KVQ_ECUDA, std::string("decode kernel launch: ") + cudaGetErrorString(e));
+  return KVQ_OK;
+}
+
+extern "C" kvq_status kvq_noalloc_check(void) {
+  void* base = nullptr;
+  kvq_status st = scratch_address(&base);
+  if (st != KVQ_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  int32_t flag = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&flag, base, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && flag) e = cudaMemset(base, 0, 4);
+  if (e != cudaSuccess) return fail(KVQ_ECUDA, std::string("kvq_noalloc_check: ") + cudaGetErrorString(e));
+  if (flag)
+    return fail(KVQ_ECUDA, "kvq_decode_attn_noalloc: a page copy did not complete within its wait limit; "
+                           "the output of that call is wrong");
   return KVQ_OK;
 }

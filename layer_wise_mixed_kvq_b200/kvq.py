@@ -25,7 +25,7 @@ EXPORTS = (
     "kvq_cache_reset", "kvq_append", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_set_split_pages", "kvq_seq_len", "kvq_bytes",
     "kvq_export_bytes", "kvq_export_layer", "kvq_sync", "kvq_launch_count", "kvq_last_error",
     "kvq_status_string", "kvq_set_fp8_scales", "kvq_layer_error", "kvq_refresh_lengths",
-    "kvq_set_decode_mode", "kvq_decode_step",
+    "kvq_set_decode_mode", "kvq_decode_step", "kvq_noalloc_check",
 )
 
 
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "kvq_decode_attn": (c.c_int, [P, c.c_int, P, c.c_int, P, P]),
         "kvq_decode_attn_noalloc": (c.c_int, [kvq_pair, c.c_int, c.c_int, c.c_int, P, c.c_int64, P, P, c.c_int64, P,
                                               c.c_int, P, P]),
+        "kvq_noalloc_check": (c.c_int, []),
         "kvq_set_split_pages": (c.c_int, [P, c.c_int]),
         "kvq_set_decode_mode": (c.c_int, [P, c.c_int]),
         "kvq_decode_step": (c.c_int, [P, c.c_int, P, P, P, c.c_int, P, P]),
@@ -216,6 +217,12 @@ def kvq_decode_attn_noalloc(pair, head_dim, n_q_heads, n_kv_heads, pages, max_pa
                                        int(n_kv_heads), _dev_ptr(pages), int(max_pages), _dev_ptr(window),
                                        _dev_ptr(seq_len), int(max_seq_len), _dev_ptr(Q), int(Q.shape[0]),
                                        _dev_ptr(out), _stream(stream)))
+
+
+def kvq_noalloc_check() -> None:
+    """Raise if a kvq_decode_attn_noalloc call on the current device gave up on a page copy
+    (waits for the device; clears the flag)."""
+    _check(lib.kvq_noalloc_check())
 
 
 def kvq_layer_error(cache, layer):

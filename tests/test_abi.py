@@ -115,3 +115,42 @@ def test_null_cache_calls_fail_cleanly(kvq):
     assert kvq.lib.kvq_decode_step(None, 0, None, None, None, 1, None, None) == kvq.KVQ_EINVAL
     assert kvq.lib.kvq_set_decode_mode(None, -1) == kvq.KVQ_EINVAL
     kvq.kvq_cache_destroy(None)
+
+
+def test_noalloc_rejects_bad_arguments_before_touching_the_device(kvq):
+    """Every argument check of kvq_decode_attn_noalloc returns before any CUDA call
+    (this machine may have no GPU), with the status its header comment gives."""
+    import ctypes
+    f = kvq.lib.kvq_decode_attn_noalloc
+    A = 1 << 20  # a 16-byte aligned stand-in address (never dereferenced: every call below fails first)
+    good = dict(pair=(4, 4), D=128, hq=32, hkv=8, pages=A, max_pages=128, window=A, seq_len=A, max_len=4096,
+                Q=A, batch=16, out=A)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return f(kvq._pair(a["pair"]), a["D"], a["hq"], a["hkv"], ctypes.c_void_p(a["pages"]), a["max_pages"],
+                 ctypes.c_void_p(a["window"]), ctypes.c_void_p(a["seq_len"]), a["max_len"], ctypes.c_void_p(a["Q"]),
+                 a["batch"], ctypes.c_void_p(a["out"]), None)
+
+    E = kvq.KVQ_EINVAL
+    assert call(pair=(3, 4)) == E                       # unsupported bits
+    assert call(pair=(16, 8)) == E                      # mixed bf16 / int
+    assert call(pair=(16, 16, 1)) == E                  # bf16 layer with a key mode
+    assert call(pair=(8, 8, 0, 1)) == E                 # fp8 needs per-head scales (a cache)
+    assert call(pair=(4, 4, 2)) == E                    # unknown key mode
+    assert call(D=96) == E
+    assert call(hq=30) == E and call(hq=80) == E and call(hkv=0) == E
+    assert call(batch=0) == E and call(batch=1025) == E
+    assert call(max_pages=-1) == E and call(max_len=-1) == E
+    assert call(max_len=4097 + 32 * 128) == E           # max_seq_len/32 > max_pages
+    assert call(max_pages=(1 << 25) + 1, max_len=0) == E
+    for name in ("pages", "window", "seq_len", "Q", "out"):
+        assert call(**{name: 0}) == E, name
+    for name in ("pages", "window", "Q", "out"):
+        assert call(**{name: A + 8}) == E, name         # not 16-byte aligned
+    assert call(seq_len=A + 2) == E                     # not 4-byte aligned
+    # more than 2^31 units: 1024 sequences x 64 heads x (2^25/32... pages + overhead)
+    assert call(batch=1024, hq=64, hkv=64, max_pages=1 << 25, max_len=1 << 30) == E
+    assert "too many pages" in kvq.lib.kvq_last_error().decode()
+    # merge counters alone would fill the 16 MiB array
+    assert call(batch=1024, hq=8192, hkv=8192, max_len=0) == kvq.KVQ_ECAPACITY
