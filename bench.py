@@ -2,14 +2,17 @@
 
 One step = for every layer of the stack: append one new token per sequence
 and decode attention for every query head (kvq_decode_step: one fused kernel
-where the one-warp-per-segment split applies, else kvq_append then
-kvq_decode_attn), over a cache prefilled to the workload's context. Default workload: the
-Llama-3.1-8B-shaped uniform K4V4 stack (32 layers, 32 query / 8 KV heads,
-head_dim 128, batch 16, context 4096).
+per layer-step), over a cache prefilled to the workload's context with one
+full-context kvq_append per layer (timed too: append tokens/s). Default
+workload, the largest: the long-context ragged Llama-3.1-8B-shaped stack
+(32 layers, layers 0 and 31 bf16, the rest K8V8, 32 query / 8 KV heads,
+head_dim 128, batch 4, per-sequence context 8K-32K). The same line carries the
+uniform K4V4 (batch 16 x 4K), mixed 3.25-bit (batch 64, short contexts) and
+Qwen2.5-7B-shaped 4.0-bit (batch 32 x 8K) stacks under `per_config`.
 
 value = algorithmic HBM bytes per step (packed codes, fp16 scales/zeros, bf16
 window of every layer at the step's context) / device time per step, in GB/s.
-The cache (2.5 GB) is far larger than the 126 MB L2, so no flush is needed.
+Every cache is far larger than the 126 MB L2, so no flush is needed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
 """
@@ -42,8 +45,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--workload", default="llama_k4v4", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="ragged_long", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads' lines (llama_k4v4, llama_mixed325, qwen_mixed40)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the step only (no isolated-launch, end-to-end or graph pass; for profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--layers", type=int, default=0,
                     help="profile a truncated stack (N layers from --first-layer); 0 = the workload's full stack")
@@ -61,25 +68,26 @@ def peaks():
 
 
 def kernel_source_hash():
+    """Hash of the sources the decode step kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "layer_wise_mixed_kvq_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("kvq_decode") and name.endswith(".cu"):
+        if (name.startswith("kvq_decode") and name.endswith(".cu")) or name.endswith(".cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_from_profile(workload):
-    """dram bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source."""
+    """DRAM bytes per decode launch from the committed ncu summary, only if its
+    counters were taken on the current kernel source (else None)."""
     path = os.path.join(PROFILES, "decode_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("kernel_hash") != kernel_source_hash():
+    if not e or e.get("counters_taken_at") != kernel_source_hash():
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -211,7 +219,8 @@ def workload_config(w, equiv_bits, world):
     """The `config` object both arms print (the GPU arm's workload, whatever the arm samples)."""
     return {"workload": w.name, "layers": w.n_layers, "layer_map_equiv_bits": equiv_bits, "batch": w.batch,
             "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-            "context": int(synth.context_lengths(w).max()), "parallelism": f"replicas x{world}",
+            "context": int(synth.context_lengths(w).max()),
+            "context_min": int(synth.context_lengths(w).min()), "parallelism": f"replicas x{world}",
             "l2": "cache larger than L2 (no flush)"}
 
 
@@ -241,44 +250,64 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------ GPU --
-def run_gpu(args, w):
-    import torch
-    import torch.distributed as dist
-    rank, world, local = replicas.world()
-    if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", init_method="env://",
-                                timeout=__import__("datetime").timedelta(seconds=120))
-    dev = torch.device("cuda", torch.cuda.current_device())
-    from layer_wise_mixed_kvq_b200 import kvq
+PER_CONFIG = ("llama_k4v4", "llama_mixed325", "qwen_mixed40")
 
+
+def prefill_bytes(w, kvq, lens):
+    """Algorithmic bytes of prefilling every layer from empty with one kvq_append:
+    the bf16 keys and values read, the pages and window rows written."""
+    total = 0
+    for pair in w.layer_map:
+        pb = kvq.kvq_page_bytes(pair, w.head_dim)
+        for T in lens:
+            T = int(T)
+            total += w.n_kv_heads * (T * 4 * w.head_dim + (T // 32) * pb + (T % 32) * 4 * w.head_dim)
+    return total
+
+
+def measure(w, args, world, full):
+    """Prefill the workload's cache, then time K decode steps (kvq_decode_step for
+    every layer: one kernel per layer-step). `full` adds the event-per-launch pass,
+    the end-to-end and CUDA-graph measurements and the clock record."""
+    import torch
+    from layer_wise_mixed_kvq_b200 import kvq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    rank = replicas.world()[0]
     B, Hq, Hkv, D, NL = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.n_layers
     lens = synth.context_lengths(w)
     total_steps = args.warmup + args.steps
     graph_steps = max(3, min(args.steps, 20))
-    # + kernel-timing, end-to-end and graph steps
-    max_tokens = int(lens.max()) + total_steps + args.steps + 32 + graph_steps + 2
+    extra = (args.steps + graph_steps + 2) if full else 0
+    max_tokens = int(lens.max()) + total_steps + extra + 32
     cache = kvq.kvq_cache_create(list(w.layer_map), Hq, Hkv, D, B, max_tokens)
     for layer, pair in enumerate(w.layer_map):
         if len(pair) > 3 and pair[3]:
             kvq.kvq_set_fp8_scales(cache, layer, w.fp8_scales[0], w.fp8_scales[1])
     gen = torch.Generator(device=dev)
     gen.manual_seed(w.seed * 1000 + rank)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = peaks()
 
-    # prefill every layer (timed separately: append tokens/s)
+    # ---- prefill: one kvq_append of the full context per layer (append tokens/s)
     pre_ms = 0.0
     for layer in range(NL):
         K, V = synth.torch_kv_tokens(w, layer, int(lens.sum()), dev, gen)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        kvq.kvq_append(cache, layer, K, V, [int(x) for x in lens])
-        e1.record()
+        e0.record(stream)
+        kvq.kvq_append(cache, layer, K, V, [int(x) for x in lens], stream)
+        e1.record(stream)
         torch.cuda.synchronize()
         pre_ms += e0.elapsed_time(e1)
         del K, V
-    prefill_tokens = int(lens.sum()) * NL
+    pre_bytes = prefill_bytes(w, kvq, lens)
+    pre_gbs = pre_bytes / (pre_ms / 1e3) / 1e9
+    append = {"tokens_per_s": int(lens.sum()) * NL / (pre_ms / 1e3), "unit": "token-layers/s",
+              "roofline": {"bound": "hbm", "achieved": pre_gbs, "peak": peak, "unit": "GB/s", "frac": pre_gbs / peak,
+                           "peak_kind": peak_kind, "bytes": pre_bytes,
+                           "kernel": "append_kernel, full-context prefill of every layer (bf16 K, V in; pages "
+                                     "and window rows out), CUDA events around each launch"}}
 
-    # per-step inputs resident in HBM
+    # ---- per-step inputs resident in HBM
     steps_K, steps_V, steps_Q = [], [], []
     for s in range(total_steps):
         kl, vl, ql = [], [], []
@@ -291,39 +320,30 @@ def run_gpu(args, w):
         steps_V.append(vl)
         steps_Q.append(ql)
     outs = [torch.empty((B, Hq, D), device=dev, dtype=torch.float32) for _ in range(NL)]
-    ones = [1] * B
-    stream = torch.cuda.current_stream()
 
     def step(s, events=None):
-        # one decode step per layer through the public call (kvq_decode_step: the
-        # append fused into the attention kernel where the one-warp-per-segment
-        # split applies, the two kernels otherwise); the kernel-timing pass calls
-        # them separately so the events bracket the decode attention kernel alone
+        # one decode step per layer through the public call: kvq_decode_step appends
+        # the layer's new token and attends, in one kernel
         for layer in range(NL):
-            if events is None:
-                kvq.kvq_decode_step(cache, layer, steps_K[s][layer], steps_V[s][layer], steps_Q[s][layer],
-                                    outs[layer], stream)
-                continue
-            kvq.kvq_append(cache, layer, steps_K[s][layer], steps_V[s][layer], ones, stream)
-            events[layer][0].record(stream)
-            kvq.kvq_decode_attn(cache, layer, steps_Q[s][layer], outs[layer], stream)
-            events[layer][1].record(stream)
-
-    for s in range(args.warmup):
-        step(s)
-    torch.cuda.synchronize()
+            if events is not None:
+                events[layer][0].record(stream)
+            kvq.kvq_decode_step(cache, layer, steps_K[s][layer], steps_V[s][layer], steps_Q[s][layer],
+                                outs[layer], stream)
+            if events is not None:
+                events[layer][1].record(stream)
 
     def step_bytes():
         return sum(kvq.kvq_bytes(cache, layer, B, True) for layer in range(NL))
 
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
     bytes_before = step_bytes()
     launches0 = kvq.kvq_launch_count(cache)
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(NL)]
-          for _ in range(args.steps)]
     with ClockSampler(dev.index) as clk:
-        # The whole-step timed region: K steps enqueued back to back, with no
-        # event between kernels (an event between two launches stops the next
-        # one from starting under the tail of the previous one).
+        # The timed region: K steps enqueued back to back with no event between
+        # kernels (an event between two launches stops the next one from starting
+        # under the tail of the previous one). Every launch is the fused decode kernel.
         replicas.barrier()
         torch.cuda.synchronize()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -333,143 +353,181 @@ def run_gpu(args, w):
         t1.record(stream)
         torch.cuda.synchronize()
         replicas.barrier()
-        launches = kvq.kvq_launch_count(cache) - launches0
-        bytes_after = step_bytes()
-        # The decode kernel's own duration: the same K steps again (same inputs,
-        # one token later), an event pair around every decode launch.
+    launches = kvq.kvq_launch_count(cache) - launches0
+    bytes_after = step_bytes()
+    # the step at context c reads the cache after its own append
+    bytes_per_step = (bytes_before + bytes_after) / 2.0
+    local_ms = t0.elapsed_time(t1)
+    total_bytes, max_ms, _ = replicas.aggregate(bytes_per_step * args.steps, local_ms)
+    ms_per_step = max_ms / args.steps
+    value = total_bytes / (max_ms / 1e3) / 1e9
+    launch_us = local_ms * 1e3 / (args.steps * NL)
+    traffic = traffic_from_profile(w.name)
+    res = {
+        "value": value, "unit": "GB/s", "ms_per_step": ms_per_step, "decode_steps_per_s": 1e3 / ms_per_step,
+        "tokens_per_s": B * world * 1e3 / ms_per_step, "bytes_per_step": bytes_per_step,
+        "append_prefill_tokens_per_s": append["tokens_per_s"], "append": append,
+        "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
+                     "frac": value / world / peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "avg_launch_us": launch_us, "algorithmic_bytes_per_launch": bytes_per_step / NL,
+                     "kernel": "fused decode step (decode_mma_kernel / decode_warp_kernel with the one-token "
+                               "append): every launch of the timed region, average duration = region / launches"},
+        "gpu_launches": launches, "clocks": clk.summary(),
+    }
+    if full:
+        # each launch alone: an event pair around every decode step kernel (no
+        # overlap with its neighbours), the same K steps one token later
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(NL)]
+              for _ in range(args.steps)]
+        b0 = step_bytes()
         torch.cuda.synchronize()
         for s in range(args.steps):
             step(args.warmup + s, ev[s])
         torch.cuda.synchronize()
+        iso_us = float(np.mean([ev[s][l][0].elapsed_time(ev[s][l][1]) for s in range(args.steps)
+                                for l in range(NL)])) * 1e3
+        iso_gbs = ((b0 + step_bytes()) / 2.0 / NL) / (iso_us / 1e6) / 1e9
+        res["roofline"]["isolated_launch"] = {"avg_us": iso_us, "achieved": iso_gbs, "frac": iso_gbs / peak}
+
+        # ---- end to end through the public API with host buffers: every step copies
+        # that step's K, V and Q for all layers from one pinned buffer to the device,
+        # runs the layer-steps on views of it, and copies all outputs back
+        e2e_steps = max(3, min(args.steps, 20))
+        n_kv = B * Hkv * D
+        row = 2 * n_kv + B * Hq * D
+        dstage = torch.empty((NL, row), device=dev, dtype=torch.bfloat16)
+        dK = [dstage[layer, :n_kv].view(B, Hkv, D) for layer in range(NL)]
+        dV = [dstage[layer, n_kv:2 * n_kv].view(B, Hkv, D) for layer in range(NL)]
+        dQ = [dstage[layer, 2 * n_kv:].view(B, Hq, D) for layer in range(NL)]
+        hstage = []
+        for s in range(e2e_steps):
+            src = s % total_steps
+            hs = torch.empty((NL, row), dtype=torch.bfloat16).pin_memory()
+            for layer in range(NL):
+                hs[layer, :n_kv].copy_(steps_K[src][layer].reshape(-1).cpu())
+                hs[layer, n_kv:2 * n_kv].copy_(steps_V[src][layer].reshape(-1).cpu())
+                hs[layer, 2 * n_kv:].copy_(steps_Q[src][layer].reshape(-1).cpu())
+            hstage.append(hs)
+        douts = torch.empty((NL, B, Hq, D), device=dev, dtype=torch.float32)
+        hout = torch.empty((NL, B, Hq, D), dtype=torch.float32).pin_memory()
+        h2d = hstage[0].numel() * hstage[0].element_size()
+        d2h = hout.numel() * hout.element_size()
+        e2e_bytes0 = step_bytes()
         replicas.barrier()
-    bytes_kernel_pass = step_bytes()
-    # the step at context c reads the cache after its own append
-    bytes_per_step = (bytes_before + bytes_after) / 2.0
-    local_ms = t0.elapsed_time(t1)
-    attn_ms = [ev[s][l][0].elapsed_time(ev[s][l][1]) for s in range(args.steps) for l in range(NL)]
-    total_bytes, max_ms, _ = replicas.aggregate(bytes_per_step * args.steps, local_ms)
-    ms_per_step = max_ms / args.steps
-    value = total_bytes / (max_ms / 1e3) / 1e9
-    attn_avg_ms = float(np.mean(attn_ms))
-    attn_gbs = ((bytes_after + bytes_kernel_pass) / 2.0 / NL) / (attn_avg_ms / 1e3) / 1e9
-    peak, peak_kind = peaks()
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for s in range(e2e_steps):
+            dstage.copy_(hstage[s], non_blocking=True)
+            for layer in range(NL):
+                kvq.kvq_decode_step(cache, layer, dK[layer], dV[layer], dQ[layer], douts[layer], stream)
+            hout.copy_(douts, non_blocking=True)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        replicas.barrier()
+        e2e_bytes = (e2e_bytes0 + step_bytes()) / 2.0
+        e2e_total, e2e_max, _ = replicas.aggregate(e2e_bytes * e2e_steps, a.elapsed_time(b_))
+        res["e2e"] = {"value": e2e_total / (e2e_max / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_max / e2e_steps}
 
-    # ---- end to end through the public API with host buffers ----
-    # Every step copies that step's inputs for all layers (K, V, Q; one pinned
-    # staging buffer, one copy) to the device, runs the 32 layer-steps on views
-    # of it, and reads all outputs back (one copy).
-    e2e_steps = max(3, min(args.steps, 20))
-    n_kv = B * Hkv * D
-    row = 2 * n_kv + B * Hq * D
-    dstage = torch.empty((NL, row), device=dev, dtype=torch.bfloat16)
-    dK = [dstage[layer, :n_kv].view(B, Hkv, D) for layer in range(NL)]
-    dV = [dstage[layer, n_kv:2 * n_kv].view(B, Hkv, D) for layer in range(NL)]
-    dQ = [dstage[layer, 2 * n_kv:].view(B, Hq, D) for layer in range(NL)]
-    hstage = []
-    for s in range(e2e_steps):
-        src = s % total_steps
-        hs = torch.empty((NL, row), dtype=torch.bfloat16).pin_memory()
-        for layer in range(NL):
-            hs[layer, :n_kv].copy_(steps_K[src][layer].reshape(-1).cpu())
-            hs[layer, n_kv:2 * n_kv].copy_(steps_V[src][layer].reshape(-1).cpu())
-            hs[layer, 2 * n_kv:].copy_(steps_Q[src][layer].reshape(-1).cpu())
-        hstage.append(hs)
-    douts = torch.empty((NL, B, Hq, D), device=dev, dtype=torch.float32)
-    hout = torch.empty((NL, B, Hq, D), dtype=torch.float32).pin_memory()
-    h2d = hstage[0].numel() * hstage[0].element_size()
-    d2h = hout.numel() * hout.element_size()
-    e2e_bytes0 = step_bytes()
-    replicas.barrier()
-    torch.cuda.synchronize()
-    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for s in range(e2e_steps):
-        dstage.copy_(hstage[s], non_blocking=True)
-        for layer in range(NL):
-            kvq.kvq_decode_step(cache, layer, dK[layer], dV[layer], dQ[layer], douts[layer], stream)
-        hout.copy_(douts, non_blocking=True)
-    b_.record(stream)
-    torch.cuda.synchronize()
-    replicas.barrier()
-    e2e_local = a.elapsed_time(b_)
-    e2e_bytes = (e2e_bytes0 + step_bytes()) / 2.0
-    e2e_total, e2e_max, _ = replicas.aggregate(e2e_bytes * e2e_steps, e2e_local)
-    e2e_value = e2e_total / (e2e_max / 1e3) / 1e9
-
-    # ---- the same step captured once in a CUDA graph and replayed ----
-    # (one-token appends and decode attention enqueue kernels only; the inputs
-    # sit in static buffers, the step's kernels are the ones timed above)
-    gK = [t.clone() for t in steps_K[0]]
-    gV = [t.clone() for t in steps_V[0]]
-    gQ = [t.clone() for t in steps_Q[0]]
-    gstream = torch.cuda.Stream()
-    gstream.wait_stream(stream)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=gstream):
-        for layer in range(NL):
-            kvq.kvq_decode_step(cache, layer, gK[layer], gV[layer], gQ[layer], outs[layer])
-    stream.wait_stream(gstream)
-    graph.replay()                      # warm-up replay
-    torch.cuda.synchronize()
-    g_bytes0 = step_bytes()             # host mirror: includes the step recorded at capture
-    replicas.barrier()
-    torch.cuda.synchronize()
-    ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ga.record(stream)
-    for _ in range(graph_steps):
-        graph.replay()
-    gb.record(stream)
-    torch.cuda.synchronize()
-    replicas.barrier()
-    g_local = ga.elapsed_time(gb)
-    kvq.kvq_refresh_lengths(cache)
-    g_bytes = (g_bytes0 + step_bytes()) / 2.0
-    g_total, g_max, _ = replicas.aggregate(g_bytes * graph_steps, g_local)
+        # ---- the same step captured once in a CUDA graph and replayed (device
+        # lengths; inputs in static buffers)
+        gK = [t.clone() for t in steps_K[0]]
+        gV = [t.clone() for t in steps_V[0]]
+        gQ = [t.clone() for t in steps_Q[0]]
+        gstream = torch.cuda.Stream()
+        gstream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gstream):
+            for layer in range(NL):
+                kvq.kvq_decode_step(cache, layer, gK[layer], gV[layer], gQ[layer], outs[layer])
+        stream.wait_stream(gstream)
+        graph.replay()                      # warm-up replay
+        torch.cuda.synchronize()
+        g_bytes0 = step_bytes()             # host mirror: includes the step recorded at capture
+        replicas.barrier()
+        torch.cuda.synchronize()
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for _ in range(graph_steps):
+            graph.replay()
+        gb.record(stream)
+        torch.cuda.synchronize()
+        replicas.barrier()
+        kvq.kvq_refresh_lengths(cache)
+        g_bytes = (g_bytes0 + step_bytes()) / 2.0
+        g_total, g_max, _ = replicas.aggregate(g_bytes * graph_steps, ga.elapsed_time(gb))
+        kvq.kvq_sync(cache)
+        del graph
+        res["graph"] = {"value": g_total / (g_max / 1e3) / 1e9, "unit": "GB/s", "steps": graph_steps,
+                        "ms_per_step": g_max / graph_steps, "decode_steps_per_s": graph_steps / (g_max / 1e3) * world,
+                        "note": "same step (kvq_decode_step per layer) captured in one CUDA graph, inputs resident"}
     kvq.kvq_sync(cache)
-    del graph
-    graph_result = {"value": g_total / (g_max / 1e3) / 1e9, "unit": "GB/s", "steps": graph_steps,
-                    "ms_per_step": g_max / graph_steps, "decode_steps_per_s": graph_steps / (g_max / 1e3) * world,
-                    "note": "same step (kvq_decode_step per layer) captured in one CUDA graph, inputs resident"}
+    kvq.kvq_cache_destroy(cache)
+    return res
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = replicas.world()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    from layer_wise_mixed_kvq_b200 import kvq
+
+    head = measure(w, args, world, full=not args.no_extras)
+    per_config = {}
+    if not args.no_per_config and not args.layers:
+        for name in PER_CONFIG:
+            if name == w.name:
+                continue
+            r = measure(synth.WORKLOADS[name], args, world, full=False)
+            per_config[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "decode_steps_per_s",
+                                                  "append_prefill_tokens_per_s", "bytes_per_step", "gpu_launches")}
+            per_config[name]["roofline"] = {k: r["roofline"][k] for k in ("achieved", "frac", "traffic",
+                                                                          "avg_launch_us")}
+            per_config[name]["append_roofline_frac"] = r["append"]["roofline"]["frac"]
+            per_config[name]["clocks"] = r["clocks"]
+            per_config[name]["config"] = workload_config(synth.WORKLOADS[name],
+                                                         kvq.kvq_equiv_bits(list(synth.WORKLOADS[name].layer_map)),
+                                                         world)
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baselines(w, args.cpu_seconds)
 
-    traffic = traffic_from_profile(w.name)
-    clocks = clk.summary()
     result = {
         "metric": METRIC,
-        "value": value,
+        "value": head["value"],
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_per_step,
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
-        "operands": "f16 tensor-core operands (integer codes and e4m3 as exact f16, q and p as hi+lo f16 pairs)",
+        "operands": "f16 tensor-core operands (integer codes and e4m3 as exact f16, q * scale and p as exact or "
+                    "hi+lo f16 pairs)",
         "data": "synthetic",
         "config": workload_config(w, kvq.kvq_equiv_bits(list(w.layer_map)), world),
-        "pct_of_peak": value / peak,
-        "decode_steps_per_s": 1e3 / ms_per_step,
-        "tokens_per_s": B * world * 1e3 / ms_per_step,
-        "append_prefill_tokens_per_s": prefill_tokens / (pre_ms / 1e3),
-        "bytes_per_step": bytes_per_step,
-        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": attn_gbs / peak, "traffic": traffic,
-                     "kernel": "decode attention (kvq_decode_attn): mean CUDA-event duration over a second pass "
-                               "of the K timed steps with an event pair around every decode launch",
-                     "peak_kind": peak_kind, "avg_launch_us": attn_avg_ms * 1e3},
+        "pct_of_peak": head["roofline"]["frac"],
+        "decode_steps_per_s": head["decode_steps_per_s"],
+        "tokens_per_s": head["tokens_per_s"],
+        "append_prefill_tokens_per_s": head["append_prefill_tokens_per_s"],
+        "append": head["append"],
+        "bytes_per_step": head["bytes_per_step"],
+        "roofline": head["roofline"],
         "cpu_baseline": cb,
-        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps, "ms_per_step": e2e_max / e2e_steps},
-        "graph": graph_result,
-        "gpu_launches": launches,
-        "clocks": clocks,
+        "e2e": head.get("e2e"),
+        "graph": head.get("graph"),
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "per_config": per_config,
     }
-    kvq.kvq_cache_destroy(cache)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:

@@ -244,7 +244,7 @@ kvq_status kvq_decode_step(kvq_cache* cache, int layer, const void* K, const voi
  * (sequence, KV head) and split-K records of (n_q_heads / n_kv_heads) *
  * (head_dim + 2) * 4 bytes; KVQ_ECAPACITY when the counters leave no room for
  * two records in 16 MiB; KVQ_EINVAL for bad arguments (including more than
- * 2^31 units of work: batch * n_kv_heads * (max_seq_len/32 + 17)). Nothing is
+ * 2^31 units of work: batch * n_kv_heads * (max_seq_len/32 + 33)). Nothing is
  * launched on error. A call whose kernel gave up waiting for a page copy (its
  * output is then wrong) raises an error word in the same array; read it with
  * kvq_noalloc_check. */

@@ -159,7 +159,7 @@ cudaError_t launch_decode(int kb, int vb, int D, const DecodeParams& p, dim3 gri
 int seg_overhead_units() {
   static const int v = [] {
     const char* e = std::getenv("KVQ_SEG_OVERHEAD_UNITS");
-    int x = e ? std::atoi(e) : 16;
+    int x = e ? std::atoi(e) : 32;
     return x < 0 ? 0 : (x > 256 ? 256 : x);
   }();
   return v;

@@ -249,7 +249,8 @@ struct Cfg {
   // shared memory layout
   static constexpr int RING = kWarps * R * STAGE;
   static constexpr int MBAR_OFF = RING;
-  static constexpr int MBAR_BYTES = ((kWarps * R + 2) * 8 + 127) / 128 * 128;  // + 2 query-row barriers
+  // ring + 2 query-row barriers, then each warp's stage part tags [kWarps][4] and the page counter
+  static constexpr int MBAR_BYTES = ((kWarps * R + 2) * 8 + kWarps * 16 + 16 + 127) / 128 * 128;
   // per-warp scratch: value scales and zeros, per-token key scales and zeros
   // (4 x 32 floats), or a flush's quantizer parameters (2 D + 64 floats)
   static constexpr int WSCR_FLOATS = 2 * D + 64 > 128 ? 2 * D + 64 : 128;
@@ -257,13 +258,14 @@ struct Cfg {
   static constexpr int WSCR_STRIDE = (WSCR_FLOATS * 4 + 127) / 128 * 128;
   static constexpr int QZ_OFF = WSCR_OFF + kWarps * WSCR_STRIDE;
   static constexpr int QZ_BYTES = KS * 32 * 16;            // head rows: query operand table
-  static constexpr int QBUF_BYTES = 2 * kMaxGqa * D * 2;   // 2 x [8][D] bf16 query rows
+  // 2 x [G][D] bf16 query rows (G <= 4 with token rows, <= 8 with head rows)
+  static constexpr int qbuf_bytes(bool tok) { return 2 * (tok ? 4 : kMaxGqa) * D * 2; }
   static constexpr int qbuf_off(bool tok) { return tok ? QZ_OFF : QZ_OFF + QZ_BYTES; }
-  static constexpr int merge_off(bool tok) { return qbuf_off(tok) + QBUF_BYTES; }
-  // then: merge area [kWarps][G][D] + m, l [kWarps][8] floats, unit starts [batch + 1] and
-  // lengths [batch] ints
+  static constexpr int merge_off(bool tok) { return qbuf_off(tok) + qbuf_bytes(tok); }
+  // then: merge area [kWarps + 1][G][D] + m, l [kWarps + 1][8] floats (one slot per warp and
+  // one for the window), unit starts [batch + 1] and lengths [batch] ints
   static int smem_bytes(bool tok, int G, int batch) {
-    return merge_off(tok) + (kWarps * G * D + 2 * kWarps * kMaxGqa) * 4 + (2 * batch + 1) * 4;
+    return merge_off(tok) + ((kWarps + 1) * G * D + 2 * (kWarps + 1) * kMaxGqa) * 4 + (2 * batch + 1) * 4;
   }
   static_assert(PB % 16 == 0, "bulk copies need 16-byte multiples");
 };
@@ -1474,32 +1476,36 @@ struct Slicer {
   }
 };
 
-// Walks the page units of one warp in the order the warp consumes them:
-// within each segment part [a, e) of the CTA slice, units a + warp + 4j.
-struct PageCursor {
-  int u, e;          // candidate unit, end of the current segment part
-  int first, P;      // current segment's first page unit and page count
-  const uint8_t* base;  // pages of the current (b, h)
+// The pages of a CTA's slice, numbered in unit order (ordinals), are handed to
+// the CTA's warps by a shared-memory counter, so a warp that runs ahead (or one
+// that spent its time on the tail unit) takes more or fewer of them and the
+// warps finish a part together. Each warp's producer (lane 0) walks the slice's
+// segment parts forward to the part holding the ordinal it drew.
+struct PageWalk {
+  int a, e;             // segment part [a, e) of the slice
+  int k0, n;            // its first page index in the segment and its page count
+  int ord0;             // ordinal of its first page
+  const uint8_t* base;  // pages of its (b, h)
 };
 
-__device__ __forceinline__ bool cursor_next(PageCursor& c, const DecodeParams& p, const int* ustart, const int* slen,
-                                            int B, int u1, int warp) {
-  for (;;) {
-    if (c.u < c.e) {
-      const int k = c.u - c.first;
-      if (k >= 0 && k < c.P) return true;
-      c.u += kWarps;  // overhead units and the tail unit lead a segment
-      continue;
-    }
-    if (c.e >= u1) return false;
-    const int a = c.e;
+// Advance w to the part holding ordinal o; false when the slice has no page o.
+__device__ __forceinline__ bool walk_to(PageWalk& w, int o, const DecodeParams& p, const int* ustart, const int* slen,
+                                        int B, int u1) {
+  while (o >= w.ord0 + w.n) {
+    if (w.e >= u1) return false;
+    const int a = w.e;
     const Seg sg = seg_of(ustart, B, p.n_kv_heads, a);
-    c.first = sg.start + p.seg_overhead + 1;
-    c.e = min(sg.start + sg.n, u1);
-    c.P = slen[sg.b] / kPageTokens;
-    c.base = p.pages + ((int64_t)(sg.b * p.n_kv_heads + sg.h) * p.max_pages) * p.page_bytes;
-    c.u = a + warp;
+    const int first = sg.start + p.seg_overhead + 1;  // first page unit (after the overhead and tail units)
+    const int e = min(sg.start + sg.n, u1);
+    const int lo = max(a, first);
+    w.ord0 += w.n;
+    w.a = a;
+    w.e = e;
+    w.k0 = lo - first;
+    w.n = max(0, e - lo);
+    w.base = p.pages + ((int64_t)(sg.b * p.n_kv_heads + sg.h) * p.max_pages) * p.page_bytes;
   }
+  return true;
 }
 
 template <int KB, int VB, int D, bool TOK, bool PT, bool F8, bool AP>
@@ -1519,13 +1525,16 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + warp * C::R;
   float* wscr = reinterpret_cast<float*>(smem + C::WSCR_OFF + warp * C::WSCR_STRIDE);
   uint32_t* qtab = reinterpret_cast<uint32_t*>(smem + C::QZ_OFF);
-  float* mo = reinterpret_cast<float*>(smem + C::merge_off(TOK));   // [kWarps][G][D]
-  float* mm = mo + kWarps * G * D;                                   // [kWarps][8]
-  float* ml = mm + kWarps * kMaxGqa;                                 // [kWarps][8]
-  int* ustart = reinterpret_cast<int*>(ml + kWarps * kMaxGqa);       // [B + 1]
+  float* mo = reinterpret_cast<float*>(smem + C::merge_off(TOK));   // [kWarps + 1][G][D]
+  float* mm = mo + (kWarps + 1) * G * D;                             // [kWarps + 1][8]
+  float* ml = mm + (kWarps + 1) * kMaxGqa;                           // [kWarps + 1][8]
+  int* ustart = reinterpret_cast<int*>(ml + (kWarps + 1) * kMaxGqa); // [B + 1]
   int* slen = ustart + B + 1;                                        // [B]: lengths before this call's append
-  __nv_bfloat16* qbuf = reinterpret_cast<__nv_bfloat16*>(smem + C::qbuf_off(TOK));  // [2][8][D]
+  __nv_bfloat16* qbuf = reinterpret_cast<__nv_bfloat16*>(smem + C::qbuf_off(TOK));  // [2][G][D]
+  constexpr int QROWS = TOK ? 4 : kMaxGqa;  // rows per query buffer
   uint64_t* qbars = reinterpret_cast<uint64_t*>(smem + C::MBAR_OFF) + kWarps * C::R;
+  int* stage_part = reinterpret_cast<int*>(qbars + 2) + warp * 4;  // [4]: first unit of the part a stage holds
+  int* s_taken = reinterpret_cast<int*>(qbars + 2) + kWarps * 4;   // pages of the slice handed out
 
   // ---- units per sequence: exclusive scan (warp 0), n_b = H * (V + 1 + P_b)
   auto scan_units = [&](bool host) {
@@ -1556,6 +1565,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     if (warp == 0) {
       mbar_init(&qbars[0], 1);
       mbar_init(&qbars[1], 1);
+      *s_taken = 0;
     }
     mbar_init_fence();
   }
@@ -1587,42 +1597,49 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     work = u1 > s0.start + p.seg_overhead;
   }
 
-  // ---- producer: the first R page units of this warp (pages below the lengths
-  // the slices were cut from are never written by the preceding kernel when
-  // `early` is set, so they may stream in under its tail)
-  PageCursor cur;
-  cur.u = u0;  // >= e: the first call looks up the segment of u0
-  cur.e = u0;
-  cur.first = 0;
-  cur.P = 0;
-  cur.base = nullptr;
+  // ---- producer: the first R pages of this warp (pages below the lengths the
+  // slices were cut from are never written by the preceding kernel when `early`
+  // is set, so they may stream in under its tail)
+  PageWalk pw;
+  pw.a = pw.e = u0;
+  pw.k0 = pw.n = pw.ord0 = 0;
+  pw.base = nullptr;
   int issued = 0;
+  bool pdone = false;  // lane 0: the slice has no more pages for this warp
   const uint64_t pol = l2_evict_first_policy();
-  auto issue_first = [&]() {
-    if (lane == 0 && work) {
-      for (int r = 0; r < C::R; ++r) {
-        if (!cursor_next(cur, p, ustart, slen, B, u1, warp)) break;
-        mbar_expect_tx(&bars[r], C::PB);
-        bulk_load_once(ring + r * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes, C::PB, &bars[r],
-                       pol);
-        cur.u += kWarps;
-        ++issued;
-      }
+  auto grab = [&](int stage) {
+    const int o = atomicAdd(s_taken, 1);
+    if (!walk_to(pw, o, p, ustart, slen, B, u1)) {
+      pdone = true;
+      return;
     }
+    stage_part[stage] = pw.a;
+    mbar_expect_tx(&bars[stage], C::PB);
+    bulk_load_once(ring + stage * C::STAGE, pw.base + (int64_t)(pw.k0 + (o - pw.ord0)) * p.page_bytes, C::PB,
+                   &bars[stage], pol);
+    ++issued;
+  };
+  auto issue_first = [&]() {
+    if (lane == 0 && work)
+      for (int r = 0; r < C::R && !pdone; ++r) grab(r);
   };
   if (p.host_units && p.early) issue_first();
   if (p.host_units) pdl_enter();
   if (!(p.host_units && p.early)) issue_first();
   if (!work) return;  // no copy was issued
+  issued = __shfl_sync(0xffffffffu, issued, 0);
+  __syncwarp();  // the stage tags are visible to the warp
 
-  // ---- query rows arrive by bulk copy (the first one ahead of the page stream)
+  // ---- query rows: the first part's straight from global memory (a bulk copy
+  // would queue behind the page copies), the later parts' by bulk copy into a
+  // shared double buffer one part ahead
   const uint32_t qbytes = (uint32_t)(G * D * 2);
   auto issue_q = [&](int unit, int buf) {
     const Seg qs = seg_of(ustart, B, H, unit);
+    fence_proxy_async();  // the buffer's previous rows were read through the generic proxy
     mbar_expect_tx(&qbars[buf], qbytes);
-    bulk_load(qbuf + buf * kMaxGqa * D, p.Q + (int64_t)(qs.b * H + qs.h) * G * D, qbytes, &qbars[buf]);
+    bulk_load(qbuf + buf * QROWS * D, p.Q + (int64_t)(qs.b * H + qs.h) * G * D, qbytes, &qbars[buf]);
   };
-  if (threadIdx.x == 0) issue_q(u0, 0);
 
   bool ok = true;
   int consumed = 0;
@@ -1641,31 +1658,36 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
       prefetch_l2(win, (uint32_t)((T % kPageTokens) * D * 2));
       prefetch_l2(win + kPageTokens * D, (uint32_t)((T % kPageTokens) * D * 2));
     }
-    // ---- the tail unit (its warp: the one whose turn it is at unit tu): the
-    // fused step's append happens here, before the query operands are live; its
+    // ---- the tail unit (its warp: part index mod 4): the fused step's append
+    // happens here, before the query operands are live; its
     // window, or the page it completed, is attended after the warp's pages
-    int tail_w = 0;          // tokens of the window this warp attends after its pages
-    bool tail_page = false;  // the page the new token completed, attended after the pages
-    if (a <= tu && tu < e && (tu - a) % kWarps == warp) {
-      tail_w = T % kPageTokens;
-      if constexpr (AP) {
-        if (!p.host_units && T >= p.max_tokens) {
+    const bool has_tail = a <= tu;  // (e > tu: a part never ends inside the overhead units)
+    const bool appends = AP && (p.host_units || T < p.max_tokens);  // device lengths: a full sequence is left as is
+    const int win_tokens = appends ? (T + 1) % kPageTokens : T % kPageTokens;
+    const bool has_win = has_tail && win_tokens > 0;
+    const bool tail_warp = has_tail && segi % kWarps == warp;
+    bool tail_page = false;  // the page the new token completed (attended first by the tail warp)
+    if constexpr (AP) {
+      if (tail_warp) {
+        if (!appends) {
           if (lane == 0 && p.err) atomicExch(p.err, 2);
         } else {
           tail_page = append_token<KB, VB, D, PT, F8>(p, seg, sg.h, T, wscr, lane);
-          tail_w = (T + 1) % kPageTokens;
           if (p.host_units && sg.h == 0 && lane == 0) p.step_len[sg.b] = T + 1;
         }
       }
     }
     const bool qvalid = qh < G;
-    {
-      const bool got = mbar_wait(&qbars[segi & 1], (uint32_t)((segi >> 1) & 1));
+    const __nv_bfloat16* qrow;
+    if (segi == 0) {
+      qrow = p.Q + ((int64_t)seg * G + (qvalid ? qh : 0)) * D;
+    } else {
+      const bool got = mbar_wait(&qbars[segi & 1], (uint32_t)(((segi - 1) >> 1) & 1));
       if (!__all_sync(0xffffffffu, got)) ok = false;
-      // prefetch the next segment's query row (unless that part is overhead units only)
-      if (threadIdx.x == 0 && e < u1 && u1 > e + p.seg_overhead) issue_q(e, (segi + 1) & 1);
+      qrow = qbuf + (segi & 1) * QROWS * D + (qvalid ? qh : 0) * D;
     }
-    const __nv_bfloat16* qrow = qbuf + (segi & 1) * kMaxGqa * D + (qvalid ? qh : 0) * D;
+    // prefetch the next part's query rows (unless that part is overhead units only)
+    if (threadIdx.x == 0 && e < u1 && u1 > e + p.seg_overhead) issue_q(e, (segi + 1) & 1);
 
     // ---- query operands
     const float ksc = F8 ? p.fp8_scales[sg.h] : 1.f;
@@ -1683,6 +1705,57 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     auto load_qbp = [&]() { load_qb<D>(qrow, qvalid && (!TOK || (g & 1) == 0), t, qb); };
     if constexpr (C::kBf16) load_qbp();
 
+    // a state (true units: the bf16 MMAs) into merge slot `slot`
+    auto store_state = [&](St& x, int slot) {
+      if constexpr (TOK) {
+        float l = x.l, vz = x.vz;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          l += __shfl_xor_sync(0xffffffffu, l, o);
+          vz += __shfl_xor_sync(0xffffffffu, vz, o);
+        }
+        if (t < G) {
+          float* dst = mo + (slot * G + t) * D;
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j) {
+            dst[16 * j + g] = x.o[j][0] + x.o[j][1] + vz;
+            dst[16 * j + 8 + g] = x.o[j][2] + x.o[j][3] + vz;
+          }
+          if (g == 0) {
+            mm[slot * kMaxGqa + t] = x.m;
+            ml[slot * kMaxGqa + t] = l;
+          }
+        }
+      } else {
+        float l = x.l + __shfl_xor_sync(0xffffffffu, x.l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        float vz = x.vz + __shfl_xor_sync(0xffffffffu, x.vz, 1);
+        vz += __shfl_xor_sync(0xffffffffu, vz, 2);
+        if (g < G) {
+          float* dst = mo + (slot * G + g) * D;
+#pragma unroll
+          for (int j = 0; j < D / 8; ++j) {
+            dst[8 * j + 2 * t] = x.o[j][0] + x.o[j][2] + vz;
+            dst[8 * j + 2 * t + 1] = x.o[j][1] + x.o[j][3] + vz;
+          }
+          if (t == 0) {
+            mm[slot * kMaxGqa + g] = x.m;
+            ml[slot * kMaxGqa + g] = l;
+          }
+        }
+      }
+    };
+    // the bf16 window, by the tail warp before its pages (its L2 reads overlap the
+    // other warps' page stream), into the window's merge slot
+    if (tail_warp && win_tokens > 0) {
+      St wst;
+      state_init(wst);
+      if constexpr (!C::kBf16) load_qbp();
+      if constexpr (TOK) attend_window_tok<D>(win, win_tokens, wst, qb, p.scale_log2, lane);
+      else attend_window<D>(win, win_tokens, wst, qb, p.scale_log2, lane);
+      store_state(wst, kWarps);
+    }
+
     St st;
     state_init(st);
     auto attend_page = [&](const uint8_t* page) {
@@ -1699,91 +1772,43 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
       }
     };
 
-    // ---- this warp's page units of the segment part [a, e)
-    for (int u = a + warp; u < e; u += kWarps) {
-      const int k = u - tu - 1;
-      if (k < 0) continue;  // overhead units and the tail unit
-      if (k < P && ok) {
-        const int stage = consumed % C::R;
-        const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
-        if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
-          ok = false;
-        } else {
-          attend_page(ring + stage * C::STAGE);
-          ++consumed;
-          __syncwarp();
-          if (lane == 0 && cursor_next(cur, p, ustart, slen, B, u1, warp)) {
-            fence_proxy_async();
-            mbar_expect_tx(&bars[stage], C::PB);
-            bulk_load_once(ring + stage * C::STAGE, cur.base + (int64_t)(cur.u - cur.first) * p.page_bytes, C::PB,
-                           &bars[stage], pol);
-            cur.u += kWarps;
-            ++issued;
-          }
-        }
+    // the page the new token completed (generic loads: it never went through the async proxy)
+    if (tail_page) attend_page(p.pages + ((int64_t)seg * p.max_pages + P) * p.page_bytes);
+
+    // ---- this warp's pages of the segment part [a, e): the ring in order, while
+    // its stages hold pages of this part
+    for (;;) {
+      if (!ok || consumed == issued) break;  // a lost copy, or no more pages for this warp
+      const int stage = consumed % C::R;
+      if (stage_part[stage] != a) break;     // the next page belongs to a later part
+      const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
+      if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
+        ok = false;
+        break;
       }
-    }
-    if (tail_page) {
-      // the page this warp has just written (generic loads: it never went through the async proxy)
-      attend_page(p.pages + ((int64_t)seg * p.max_pages + P) * p.page_bytes);
+      attend_page(ring + stage * C::STAGE);
+      ++consumed;
+      __syncwarp();
+      if (lane == 0 && !pdone) {
+        fence_proxy_async();
+        grab(stage);
+      }
+      issued = __shfl_sync(0xffffffffu, issued, 0);
+      __syncwarp();  // the stage tag is visible to the warp
     }
     to_true_units<VB, TOK, F8>(st, F8 ? p.fp8_scales[H + sg.h] : 1.f);
-    if (tail_w > 0) {
-      if constexpr (!C::kBf16) load_qbp();
-      if constexpr (TOK) attend_window_tok<D>(win, tail_w, st, qb, p.scale_log2, lane);
-      else attend_window<D>(win, tail_w, st, qb, p.scale_log2, lane);
-    }
-
-    // ---- warps -> shared memory, CTA merge
-    if constexpr (TOK) {
-      float l = st.l, vz = st.vz;
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        l += __shfl_xor_sync(0xffffffffu, l, o);
-        vz += __shfl_xor_sync(0xffffffffu, vz, o);
-      }
-      if (t < G) {
-        float* dst = mo + (warp * G + t) * D;
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          dst[16 * j + g] = st.o[j][0] + st.o[j][1] + vz;
-          dst[16 * j + 8 + g] = st.o[j][2] + st.o[j][3] + vz;
-        }
-        if (g == 0) {
-          mm[warp * kMaxGqa + t] = st.m;
-          ml[warp * kMaxGqa + t] = l;
-        }
-      }
-    } else {
-      float l = st.l + __shfl_xor_sync(0xffffffffu, st.l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      float vz = st.vz + __shfl_xor_sync(0xffffffffu, st.vz, 1);
-      vz += __shfl_xor_sync(0xffffffffu, vz, 2);
-      if (g < G) {
-        float* dst = mo + (warp * G + g) * D;
-#pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-          dst[8 * j + 2 * t] = st.o[j][0] + st.o[j][2] + vz;
-          dst[8 * j + 2 * t + 1] = st.o[j][1] + st.o[j][3] + vz;
-        }
-        if (t == 0) {
-          mm[warp * kMaxGqa + g] = st.m;
-          ml[warp * kMaxGqa + g] = l;
-        }
-      }
-    }
+    store_state(st, warp);
     __syncthreads();
-    const bool whole = (a <= tu) && (e == sg.start + sg.n);
+    const bool whole = has_tail && (e == sg.start + sg.n);
     float* outp = p.out + (int64_t)seg * G * D;
     float* part = p.partials + ((int64_t)blockIdx.x * 2 + (a == u0 ? 0 : 1)) * split_record_floats(G, D);
+    const int nslots = kWarps + (has_win ? 1 : 0);
     for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
       const int gg = idx / D, d = idx % D;
       float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * kMaxGqa + gg]);
+      for (int w = 0; w < nslots; ++w) M = fmaxf(M, mm[w * kMaxGqa + gg]);
       float L = 0.f, O = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
+      for (int w = 0; w < nslots; ++w) {
         const float mw = mm[w * kMaxGqa + gg];
         const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
         L = fmaf(f, ml[w * kMaxGqa + gg], L);

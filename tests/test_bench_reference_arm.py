@@ -21,5 +21,7 @@ def test_reference_arm_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     cfg = line["config"]
-    assert cfg["workload"] == "llama_k4v4" and cfg["batch"] == 16 and cfg["layers"] == 32
-    assert cfg["layer_map_equiv_bits"] == 4.0 and cfg["context"] == 4096
+    # the default workload is the largest: the long-context ragged stack (bf16 layers 0 and 31, K8V8 between)
+    assert cfg["workload"] == "ragged_long" and cfg["batch"] == 4 and cfg["layers"] == 32
+    assert cfg["layer_map_equiv_bits"] == 8.5 and 8192 <= cfg["context_min"] <= cfg["context"] <= 32768
+    assert line["ms_per_step"] > 0
