@@ -80,6 +80,96 @@ __device__ __forceinline__ uint4 load8(const void* base, int64_t idx) {
   }
 }
 
+// Integer code blocks, tile by tile. A block's 16-byte vector vi of lane
+// (g, t) holds 16/BITS consecutive 16x16 tiles f (tile row dt = f/2, token
+// half tt = f%2); element (p, j) of a tile sits at row g + 8(p&1), column
+// 2t + j + 8(p>>1), rows being tokens for keys and channels for values. The
+// element's code goes to nibble p + 4j of word f (4-bit), to bits
+// 2(4u + p + 8j) of word f/2 with u = f%2 (2-bit), or to byte 2(p&1) + j of
+// word 2f + p/2 (8-bit): the same layout as lane_word, produced tile by tile so
+// that a tile's values and quantizer parameters are loaded once.
+//   code(r, p, j, x, i): code of the element with value x and parameter index i.
+template <int BITS>
+__device__ __forceinline__ void place_tile(uint32_t (&words)[4], int i, const uint32_t (&c)[4][2]) {
+  if constexpr (BITS == 4) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) w |= c[p][j] << (4 * (p + 4 * j));
+    words[i] = w;
+  } else if constexpr (BITS == 2) {
+    const int u = i & 1;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) words[i >> 1] |= c[p][j] << (2 * (4 * u + p + 8 * j));
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      words[2 * i + h] = c[2 * h][0] | (c[2 * h][1] << 8) | (c[2 * h + 1][0] << 16) | (c[2 * h + 1][1] << 24);
+  }
+}
+
+// Vector vi of lane `lane` of the key block (r = 0) or value block (r = 1).
+// xs: [32][RS] bf16 rows of the group (tokens); pz, pr: quantizer zero points and
+// reciprocals by channel (per-channel keys) or by token (values, per-token keys).
+template <int BITS, int RS, typename Code>
+__device__ __forceinline__ uint4 pack_vector(int r, bool by_token, int lane, int vi,
+                                             const __nv_bfloat16 (*xs)[RS], Code code) {
+  constexpr int TPV = 16 / BITS;  // tiles per 16-byte vector
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < TPV; ++i) {
+    const int f = vi * TPV + i, dt = f >> 1, tt = f & 1;
+    uint32_t c[4][2];
+    if (r == 0) {
+      // keys: rows are tokens 16tt + g (+8), columns channels 16dt + 2t (+1) (+8)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int tok = 16 * tt + g + 8 * (p & 1), dim = 16 * dt + 2 * t + 8 * (p >> 1);
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[tok][dim]));
+        c[p][0] = code(p, 0, x.x, by_token ? tok : dim);
+        c[p][1] = code(p, 1, x.y, by_token ? tok : dim + 1);
+      }
+    } else {
+      // values: rows are channels 16dt + g (+8), columns tokens 16tt + 2t (+1) (+8)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int dim = 16 * dt + g + 8 * (p & 1), tok = 16 * tt + 2 * t + 8 * (p >> 1);
+        c[p][0] = code(p, 0, __bfloat162float(xs[tok][dim]), tok);
+        c[p][1] = code(p, 1, __bfloat162float(xs[tok + 1][dim]), tok + 1);
+      }
+    }
+    place_tile<BITS>(words, i, c);
+  }
+  return make_uint4(words[0], words[1], words[2], words[3]);
+}
+
+// One integer code block (R = 0 keys, 1 values) of BITS-bit codes, with this
+// thread's share of the error report terms.
+template <int R, int BITS, int D, int RS>
+__device__ __forceinline__ void emit_block(uint8_t* blk, bool per_token_keys, const __nv_bfloat16 (*xs)[RS],
+                                           const float* pz, const float* pr, const float* ps, double (&err)[4]) {
+  constexpr int qmax = (1 << BITS) - 1;
+  const bool by_token = R == 1 || per_token_keys;
+  auto code = [&](int, int, float x, int i) -> uint32_t {
+    QParams q;
+    q.z = pz[i];
+    q.r = pr[i];
+    q.zero_scale = (q.r == 0.0f);
+    const uint32_t c = quant_code(x, q, qmax);
+    const double dx = (double)x - ((double)c * (double)ps[i] + (double)q.z);
+    err[2 * R] += dx * dx;
+    err[2 * R + 1] += (double)x * (double)x;
+    return c;
+  };
+  constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
+  for (int v = threadIdx.x; v < kVectors; v += kThreads)
+    reinterpret_cast<uint4*>(blk)[v] = pack_vector<BITS, RS>(R, by_token, v & 31, v >> 5, xs, code);
+}
+
 template <int KB, int VB, int D, bool F32IN>
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
   pdl_enter();
@@ -238,21 +328,8 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         quantize_tokens(1, (1 << VB) - 1, vscale, vzero);
         __syncthreads();
         // codes, each element quantized as it is packed, and its error report terms
-        auto code = [&](int r, int i, float x, int qmax) -> uint32_t {
-          QParams q;
-          q.z = pz[r][i];
-          q.r = pr[r][i];
-          q.zero_scale = (q.r == 0.0f);
-          const uint32_t c = quant_code(x, q, qmax);
-          add_err(r, x, (double)c * (double)ps[r][i] + (double)q.z);
-          return c;
-        };
-        store_block<KB, D>(page, false, [&](int tok, int dim) {
-          return code(0, per_token_keys ? tok : dim, __bfloat162float(xs[0][tok][dim]), (1 << KB) - 1);
-        });
-        store_block<VB, D>(vblk, true, [&](int tok, int dim) {
-          return code(1, tok, __bfloat162float(xs[1][tok][dim]), (1 << VB) - 1);
-        });
+        emit_block<0, KB, D, RS>(page, per_token_keys, xs[0], pz[0], pr[0], ps[0], err);
+        emit_block<1, VB, D, RS>(vblk, true, xs[1], pz[1], pr[1], ps[1], err);
       }
       // this flush's error sums: warp shuffles, then one fp64 atomic per sum into
       // one of the layer's bins

@@ -353,6 +353,26 @@ __device__ __forceinline__ void load_tile_words(const uint8_t* blk, int lane, in
   }
 }
 
+// The same words through a 16-byte vector per lane shared by consecutive tile
+// rows: 4-bit blocks hold 2 tile rows per vector, 2-bit blocks 4. Called with
+// dt = 0, 1, ... in order (unrolled), it loads a vector only at a vector's first
+// tile row, so a warp reads whole 512-byte rows (no bank conflicts) with half or
+// a quarter of the loads.
+template <int BITS>
+__device__ __forceinline__ void tile_words(const uint8_t* blk, int lane, int dt, uint4& vec,
+                                           uint32_t (&w)[TileWords<BITS>::N]) {
+  constexpr int N = TileWords<BITS>::N;
+  if constexpr (N >= 4) {
+    load_tile_words<BITS>(blk, lane, dt, w);
+  } else {
+    const int word0 = dt * N;
+    if (word0 % 4 == 0) vec = *reinterpret_cast<const uint4*>(blk + ((word0 / 4) * 32 + lane) * 16);
+    const uint32_t c[4] = {vec.x, vec.y, vec.z, vec.w};
+#pragma unroll
+    for (int i = 0; i < N; ++i) w[i] = c[word0 % 4 + i];
+  }
+}
+
 // B fragments of tile (dt, tt): b[0..1] for the even n-tile (key tokens
 // 16tt..16tt+7, or value channels 16dt..16dt+7), b[2..3] for the odd one.
 template <int BITS>
@@ -619,10 +639,11 @@ __device__ __forceinline__ void tok_pv_frags(const float (&pv)[4], uint32_t (&b)
 // PV of one integer / fp8 / bf16 value block with the B fragments above.
 template <int VB, int D, bool F8>
 __device__ __forceinline__ void tok_pv(const uint8_t* vblk, TokState<D>& st, const uint32_t (&b)[2][2], int lane) {
+  uint4 vec;
 #pragma unroll
   for (int dt = 0; dt < D / 16; ++dt) {
     uint32_t w[TileWords<VB>::N];
-    load_tile_words<VB>(vblk, lane, dt, w);
+    tile_words<VB>(vblk, lane, dt, vec, w);
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
       uint32_t a[4];
@@ -685,10 +706,11 @@ __device__ __forceinline__ void attend_qpage_tok(const uint8_t* page, TokState<D
     for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
   const uint2* srow = reinterpret_cast<const uint2*>(kscale + t * (D / 4));   // channels 2t, 2t+1, 2t+8, 2t+9 per tile
   const uint2* zrow = reinterpret_cast<const uint2*>(kzero + t * (D / 4));
+  uint4 vec;
 #pragma unroll
   for (int dt = 0; dt < C::KS; ++dt) {
     uint32_t w[TileWords<KB>::N];
-    load_tile_words<KB>(page, lane, dt, w);
+    tile_words<KB>(page, lane, dt, vec, w);
     const uint2 s = srow[dt];
     const uint32_t h0 = hmul2(ops.q2[2 * dt], s.x), h1 = hmul2(ops.q2[2 * dt + 1], s.y);
     const uint32_t b0 = hfma2(ops.q2[2 * dt], s.x, hmul2(h0, ops.npart));
@@ -738,10 +760,11 @@ __device__ __forceinline__ void attend_qpage_tok_pt(const uint8_t* page, TokStat
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int k = 0; k < 4; ++k) s2[mt][k] = 0.f;
+  uint4 vec;
 #pragma unroll
   for (int dt = 0; dt < C::KS; ++dt) {
     uint32_t w[TileWords<KB>::N];
-    load_tile_words<KB>(page, lane, dt, w);
+    tile_words<KB>(page, lane, dt, vec, w);
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
       uint32_t a[4];
@@ -940,10 +963,11 @@ __device__ __forceinline__ void prep_head_ops(HeadOps& ops, uint32_t* qtab, bool
 // PV of head rows: A = p' (hi/lo) per 16-token k-step, B = value codes.
 template <int VB, int D, bool F8>
 __device__ __forceinline__ void head_pv(const uint8_t* vblk, WarpState<D>& st, const uint32_t (&pa)[2][4], int lane) {
+  uint4 vec;
 #pragma unroll
   for (int dt = 0; dt < D / 16; ++dt) {
     uint32_t w[TileWords<VB>::N];
-    load_tile_words<VB>(vblk, lane, dt, w);
+    tile_words<VB>(vblk, lane, dt, vec, w);
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
       uint32_t b[4];
@@ -1004,10 +1028,11 @@ __device__ __forceinline__ void attend_qpage(const uint8_t* page, WarpState<D>& 
     for (int k = 0; k < 4; ++k) s4[j][k] = 0.f;
   const uint2* srow = reinterpret_cast<const uint2*>(kscale + t * (D / 4));
   const uint2* zrow = reinterpret_cast<const uint2*>(kzero + t * (D / 4));
+  uint4 vec;
 #pragma unroll
   for (int dt = 0; dt < C::KS; ++dt) {
     uint32_t w[TileWords<KB>::N];
-    load_tile_words<KB>(page, lane, dt, w);
+    tile_words<KB>(page, lane, dt, vec, w);
     const uint4 q = *reinterpret_cast<const uint4*>(qtab + (dt * 32 + lane) * 4);
     const uint2 s = srow[dt];
     const uint32_t h01 = hmul2(q.x, s.x), h89 = hmul2(q.y, s.y);
@@ -1060,10 +1085,11 @@ __device__ __forceinline__ void attend_qpage_pt(const uint8_t* page, WarpState<D
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int k = 0; k < 4; ++k) s4[j][k] = 0.f;
+  uint4 vec;
 #pragma unroll
   for (int dt = 0; dt < C::KS; ++dt) {
     uint32_t w[TileWords<KB>::N];
-    load_tile_words<KB>(page, lane, dt, w);
+    tile_words<KB>(page, lane, dt, vec, w);
     const uint2 q = *reinterpret_cast<const uint2*>(qtab + (dt * 32 + lane) * 4);
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
@@ -1643,6 +1669,8 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
 
   bool ok = true;
   int consumed = 0;
+  int cstage = 0;       // consumed % R
+  uint32_t cphase = 0;  // (consumed / R) & 1
   int segi = 0;
   for (int a = u0; a < u1; ++segi) {
     const Seg sg = seg_of(ustart, B, H, a);
@@ -1779,15 +1807,19 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     // its stages hold pages of this part
     for (;;) {
       if (!ok || consumed == issued) break;  // a lost copy, or no more pages for this warp
-      const int stage = consumed % C::R;
+      const int stage = cstage;
       if (stage_part[stage] != a) break;     // the next page belongs to a later part
-      const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
+      const bool arrived = mbar_wait(&bars[stage], cphase);
       if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform verdict
         ok = false;
         break;
       }
       attend_page(ring + stage * C::STAGE);
       ++consumed;
+      if (++cstage == C::R) {
+        cstage = 0;
+        cphase ^= 1u;
+      }
       __syncwarp();
       if (lane == 0 && !pdone) {
         fence_proxy_async();
