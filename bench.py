@@ -288,11 +288,16 @@ def measure(w, args, world, full):
     stream = torch.cuda.current_stream()
     peak, peak_kind = peaks()
 
-    # ---- prefill: one kvq_append of the full context per layer (append tokens/s)
+    # ---- prefill: one kvq_append of the full context per layer (append tokens/s).
+    # A ~1 ms device-side sleep ahead of the start event keeps the stream busy
+    # while the host prepares and launches the append, so the events time the
+    # device work only.
     pre_ms = 0.0
     for layer in range(NL):
         K, V = synth.torch_kv_tokens(w, layer, int(lens.sum()), dev, gen)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)
         e0.record(stream)
         kvq.kvq_append(cache, layer, K, V, [int(x) for x in lens], stream)
         e1.record(stream)

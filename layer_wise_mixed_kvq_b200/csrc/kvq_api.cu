@@ -165,6 +165,15 @@ int seg_overhead_units() {
   return v;
 }
 
+int append_groups_per_cta() {
+  static const int v = [] {
+    const char* e = std::getenv("KVQ_APPEND_GROUPS_PER_CTA");
+    const int n = e ? std::atoi(e) : 0;
+    return n >= 1 && n <= 1024 ? n : 8;
+  }();
+  return v;
+}
+
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_p, int64_t stride) {
   const int64_t target_ctas = (int64_t)sm_count * 3;
   int64_t chunk = std::max<int64_t>(8, (total_pages + target_ctas - 1) / target_ctas);
@@ -452,7 +461,10 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
     c->plan_pending = true;
     p.plan = c->plan_dev;
   }
-  dim3 grid(all_one ? 1 : max_items, c->n_kv_heads, batch);
+  // multi-token appends: each CTA quantizes up to append_groups_per_cta() of a
+  // sequence-head's completed groups, staging the next while it quantizes one
+  const int gpc = kvq::append_groups_per_cta();
+  dim3 grid(all_one ? 1 : (max_items + gpc - 1) / gpc, c->n_kv_heads, batch);
   cudaError_t e = kvq::launch_append(L.kb, L.vb, c->head_dim, dtype, p, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
   c->launches += 1;

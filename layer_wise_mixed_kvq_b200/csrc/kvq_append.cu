@@ -57,6 +57,19 @@ __device__ __forceinline__ void store_block(uint8_t* blk, bool is_value, Get val
   }
 }
 
+// Asynchronous 16-byte global -> shared copies (L2 only), committed and
+// waited for in groups.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
 template <bool F32IN>
 __device__ __forceinline__ __nv_bfloat16 load_in(const void* base, int64_t idx) {
   if constexpr (F32IN) return __float2bfloat16_rn(reinterpret_cast<const float*>(base)[idx]);
@@ -80,106 +93,172 @@ __device__ __forceinline__ uint4 load8(const void* base, int64_t idx) {
   }
 }
 
-// Integer code blocks, tile by tile. A block's 16-byte vector vi of lane
-// (g, t) holds 16/BITS consecutive 16x16 tiles f (tile row dt = f/2, token
-// half tt = f%2); element (p, j) of a tile sits at row g + 8(p&1), column
-// 2t + j + 8(p>>1), rows being tokens for keys and channels for values. The
-// element's code goes to nibble p + 4j of word f (4-bit), to bits
-// 2(4u + p + 8j) of word f/2 with u = f%2 (2-bit), or to byte 2(p&1) + j of
-// word 2f + p/2 (8-bit): the same layout as lane_word, produced tile by tile so
-// that a tile's values and quantizer parameters are loaded once.
-//   code(r, p, j, x, i): code of the element with value x and parameter index i.
-template <int BITS>
-__device__ __forceinline__ void place_tile(uint32_t (&words)[4], int i, const uint32_t (&c)[4][2]) {
-  if constexpr (BITS == 4) {
-    uint32_t w = 0;
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) w |= c[p][j] << (4 * (p + 4 * j));
-    words[i] = w;
-  } else if constexpr (BITS == 2) {
-    const int u = i & 1;
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) words[i >> 1] |= c[p][j] << (2 * (4 * u + p + 8 * j));
-  } else {
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      words[2 * i + h] = c[2 * h][0] | (c[2 * h][1] << 8) | (c[2 * h + 1][0] << 16) | (c[2 * h + 1][1] << 24);
-  }
+// Fragment loads from the staged rows: matrix m of an x4 load takes its eight
+// row addresses from lanes 8m..8m+7, and lane (g, t) = (lane/4, lane%4)
+// receives row g, columns 2t and 2t+1 of each matrix (rows and columns
+// swapped with .trans).
+__device__ __forceinline__ void ldsm_x4(uint32_t (&a)[4], const void* p) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]) : "r"(s));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&a)[4], const void* p) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]) : "r"(s));
 }
 
-// Vector vi of lane `lane` of the key block (r = 0) or value block (r = 1).
-// xs: [32][RS] bf16 rows of the group (tokens); pz, pr: quantizer zero points and
-// reciprocals by channel (per-channel keys) or by token (values, per-token keys).
-template <int BITS, int RS, typename Code>
-__device__ __forceinline__ uint4 pack_vector(int r, bool by_token, int lane, int vi,
-                                             const __nv_bfloat16 (*xs)[RS], Code code) {
+// Tile (dt, tt) of a code block for this lane: register p holds elements
+// (p, 0) and (p, 1) (low, high half), element (p, j) sitting at row g + 8(p&1),
+// column 2t + j + 8(p>>1) of the 16x16 tile. Rows are tokens 16tt.. for keys
+// (is_value false) and channels 16dt.. for values; xs rows are tokens.
+template <int RS>
+__device__ __forceinline__ void load_tile(uint32_t (&a)[4], const __nv_bfloat16 (*xs)[RS], bool is_value,
+                                          int dt, int tt, int lane) {
+  const int m = lane >> 3, r = lane & 7;
+  if (is_value) ldsm_x4_trans(a, &xs[16 * tt + 8 * (m >> 1) + r][16 * dt + 8 * (m & 1)]);
+  else ldsm_x4(a, &xs[16 * tt + r + 8 * (m & 1)][16 * dt + 8 * (m >> 1)]);
+}
+
+// One element's code, as the bits of the fp32 number 1.5 * 2^23 + code: for y in
+// [0, qmax] the single rounding of the addition is rint(y), round-half-even.
+// The clamp to [0, qmax] first gives clamp(rint(y), 0, qmax) for every y
+// (fmaxf also maps a NaN to 0), and a zero reciprocal (constant set) gives 0.
+constexpr uint32_t kRintBias = 0x4B400000u;  // bits of 1.5 * 2^23
+__device__ __forceinline__ uint32_t code_bits(float x, float z, float r, float qmax) {
+  const float y = fminf(fmaxf(__fmul_rn(__fsub_rn(x, z), r), 0.0f), qmax);
+  return __float_as_uint(__fadd_rn(y, 12582912.0f));
+}
+
+// Error report terms of one element: (x - x_hat)^2 and x^2 in fp64, with
+// x_hat = code * s + z exact in fp64 (code < 2^8, s and z fp16 values).
+// The code becomes a double through the bits of 2^52 + (code bits).
+__device__ __forceinline__ void add_error(double (&e)[2], float x, uint32_t bits, double2 zs) {
+  const double c = __hiloint2double(0x43300000, (int)bits) - (4503599627370496.0 + (double)kRintBias);
+  const double xd = (double)x;
+  const double dx = xd - fma(c, zs.y, zs.x);
+  e[0] = fma(dx, dx, e[0]);
+  e[1] = fma(xd, xd, e[1]);
+}
+
+// Quantizer parameters of one index (a channel or a token): z and 1/s in fp32
+// for the code, z and s in fp64 for the error report.
+struct QTab {
+  const float2* zr;
+  const double2* zs;
+};
+
+// Integer code block of BITS-bit codes. Lane l's 16-byte vector vi holds tiles
+// f = vi * 16/BITS .. (tile row dt = f/2, token half tt = f%2). Element (p, j)
+// of tile f goes to nibble p + 4j of word f (4-bit), to bits 2(4u + p + 8j) of
+// word f/2 with u = f%2 (2-bit), or to byte 2(p&1) + j of word 2f + p/2 (8-bit).
+// MODE 0: keys, one parameter set per channel; 1: keys, one per token;
+// 2: values, one per token. e: this thread's error terms of the block.
+template <int BITS, int D, int RS, int MODE>
+__device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*xs)[RS], QTab q, double (&e)[2]) {
   constexpr int TPV = 16 / BITS;  // tiles per 16-byte vector
-  const int g = lane >> 2, t = lane & 3;
-  uint32_t words[4] = {0u, 0u, 0u, 0u};
+  constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
+  constexpr float qmax = (float)((1 << BITS) - 1);
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  for (int v = threadIdx.x; v < kVectors; v += kThreads) {
+    const int vi = v >> 5;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    // one element: quantize, add its error terms, add its code into its field
+    auto put = [&](int i, int p, int j, float x, float2 zr, double2 zs) {
+      const uint32_t bits = code_bits(x, zr.x, zr.y, qmax);
+      add_error(e, x, bits, zs);
+      // (bits - bias) << shift is the code in place; words only gain disjoint fields
+      if constexpr (BITS == 4) w[i] += (bits - kRintBias) << (4 * (p + 4 * j));
+      else if constexpr (BITS == 2) w[i >> 1] += (bits - kRintBias) << (2 * (4 * (i & 1) + p + 8 * j));
+      else w[2 * i + (p >> 1)] += (bits - kRintBias) << (8 * (2 * (p & 1) + j));
+    };
+    auto elem = [](const uint32_t (&a)[4], int p, int j) {
+      return __uint_as_float(j ? (a[p] & 0xFFFF0000u) : (a[p] << 16));
+    };
+    if constexpr (MODE == 0) {
+      // parameters by channel 16dt + 2t + j + 8(p>>1): shared by both token halves
 #pragma unroll
-  for (int i = 0; i < TPV; ++i) {
-    const int f = vi * TPV + i, dt = f >> 1, tt = f & 1;
-    uint32_t c[4][2];
-    if (r == 0) {
-      // keys: rows are tokens 16tt + g (+8), columns channels 16dt + 2t (+1) (+8)
+      for (int d2 = 0; d2 < TPV / 2; ++d2) {
+        const int dt = vi * (TPV / 2) + d2;
+        float2 zr[2][2];
+        double2 zs[2][2];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int tok = 16 * tt + g + 8 * (p & 1), dim = 16 * dt + 2 * t + 8 * (p >> 1);
-        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[tok][dim]));
-        c[p][0] = code(p, 0, x.x, by_token ? tok : dim);
-        c[p][1] = code(p, 1, x.y, by_token ? tok : dim + 1);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            zr[h][j] = q.zr[16 * dt + 2 * t + j + 8 * h];
+            zs[h][j] = q.zs[16 * dt + 2 * t + j + 8 * h];
+          }
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          uint32_t a[4];
+          load_tile<RS>(a, xs, false, dt, tt, lane);
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) put(2 * d2 + tt, p, j, elem(a, p, j), zr[p >> 1][j], zs[p >> 1][j]);
+        }
       }
     } else {
-      // values: rows are channels 16dt + g (+8), columns tokens 16tt + 2t (+1) (+8)
+      // parameters by token: 16tt + g + 8(p&1) (keys, MODE 1) or 16tt + 2t + j + 8(p>>1)
+      // (values), shared by every tile row of a token half
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int dim = 16 * dt + g + 8 * (p & 1), tok = 16 * tt + 2 * t + 8 * (p >> 1);
-        c[p][0] = code(p, 0, __bfloat162float(xs[tok][dim]), tok);
-        c[p][1] = code(p, 1, __bfloat162float(xs[tok + 1][dim]), tok + 1);
+      for (int tt = 0; tt < 2; ++tt) {
+        float2 zr[2][2];
+        double2 zs[2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int i = MODE == 1 ? 16 * tt + g + 8 * h : 16 * tt + 2 * t + j + 8 * h;
+            zr[h][j] = q.zr[i];
+            zs[h][j] = q.zs[i];
+          }
+#pragma unroll
+        for (int d2 = 0; d2 < TPV / 2; ++d2) {
+          const int dt = vi * (TPV / 2) + d2;
+          uint32_t a[4];
+          load_tile<RS>(a, xs, MODE == 2, dt, tt, lane);
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int h = MODE == 1 ? (p & 1) : (p >> 1), jj = MODE == 1 ? 0 : j;
+              put(2 * d2 + tt, p, j, elem(a, p, j), zr[h][jj], zs[h][jj]);
+            }
+        }
       }
     }
-    place_tile<BITS>(words, i, c);
+    reinterpret_cast<uint4*>(blk)[v] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  return make_uint4(words[0], words[1], words[2], words[3]);
 }
 
-// One integer code block (R = 0 keys, 1 values) of BITS-bit codes, with this
-// thread's share of the error report terms.
-template <int R, int BITS, int D, int RS>
-__device__ __forceinline__ void emit_block(uint8_t* blk, bool per_token_keys, const __nv_bfloat16 (*xs)[RS],
-                                           const float* pz, const float* pr, const float* ps, double (&err)[4]) {
-  constexpr int qmax = (1 << BITS) - 1;
-  const bool by_token = R == 1 || per_token_keys;
-  auto code = [&](int, int, float x, int i) -> uint32_t {
-    QParams q;
-    q.z = pz[i];
-    q.r = pr[i];
-    q.zero_scale = (q.r == 0.0f);
-    const uint32_t c = quant_code(x, q, qmax);
-    const double dx = (double)x - ((double)c * (double)ps[i] + (double)q.z);
-    err[2 * R] += dx * dx;
-    err[2 * R + 1] += (double)x * (double)x;
-    return c;
-  };
-  constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
-  for (int v = threadIdx.x; v < kVectors; v += kThreads)
-    reinterpret_cast<uint4*>(blk)[v] = pack_vector<BITS, RS>(R, by_token, v & 31, v >> 5, xs, code);
+// bf16 block (a bf16 layer): the tile registers are the block's words.
+template <int D, int RS>
+__device__ __forceinline__ void emit_bf16(uint8_t* blk, const __nv_bfloat16 (*xs)[RS], bool is_value) {
+  constexpr int kVectors = (int)(code_block_bytes(16, D) / 16);
+  const int lane = threadIdx.x & 31;
+  for (int v = threadIdx.x; v < kVectors; v += kThreads) {
+    const int f = v >> 5;
+    uint32_t a[4];
+    load_tile<RS>(a, xs, is_value, f >> 1, f & 1, lane);
+    reinterpret_cast<uint4*>(blk)[v] = make_uint4(a[0], a[1], a[2], a[3]);
+  }
 }
 
 template <int KB, int VB, int D, bool F32IN>
-__global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
+__global__ void __launch_bounds__(kThreads, (KB == 2 || VB == 2) ? 3 : 4) append_kernel(AppendParams a) {
   pdl_enter();
   constexpr bool kBf16Layer = (KB == 16);
   constexpr int RS = D + 8;          // bf16 row stride of the staged rows (16-byte rows, staggered banks)
   constexpr int NP = D > 32 ? D : 32;
   const int b = blockIdx.z, h = blockIdx.y, item = blockIdx.x;
   const int H = a.n_kv_heads;
-  __shared__ __align__(16) __nv_bfloat16 xs[2][kPageTokens][RS];  // keys, values of the group
-  __shared__ float pz[2][NP], pr[2][NP], ps[2][NP];  // quantizer zero, reciprocal, scale: keys, values
+  __shared__ __align__(16) __nv_bfloat16 xsb[2][2][kPageTokens][RS];  // two groups' key and value rows
+  __shared__ __align__(16) float2 qzr[2][NP];   // quantizer z, 1/s by index: keys, values
+  __shared__ __align__(16) double2 qzs[2][NP];  // z, s in fp64 (error report)
+  constexpr int KP = D / 2, KS = kThreads / KP;  // key channel pairs, token splits of the key pass
+  __shared__ __nv_bfloat162 kpart[KS][2][KP];   // per-split min, max of each key channel pair
   __shared__ double red[kThreads / 32][4];
   __shared__ int s_T0;
   __nv_bfloat16 k_new, v_new;  // one-token mode: this thread's channel of the new row
@@ -231,107 +310,150 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
   __nv_bfloat16* win = a.window + ((int64_t)(b * H + h) * 2) * kPageTokens * D;
 
   if (ng > 0) {
-    const int g = g0 + item;
-    uint8_t* page = a.pages + ((int64_t)(b * H + h) * a.max_pages + g) * a.page_bytes;
-    // the group's 32 key and value rows, old window slots first, as 16-byte vectors
+    // this CTA's groups are item, item + gridDim.x, ...; the next group's rows
+    // are staged (asynchronous 16-byte copies for bf16 inputs) while one group
+    // is quantized
     constexpr int VPR = D / 8;
-    for (int v = threadIdx.x; v < 2 * kPageTokens * VPR; v += kThreads) {
-      const int r = v / (kPageTokens * VPR), rem = v % (kPageTokens * VPR);
-      const int tk = rem / VPR, c8 = (rem % VPR) * 8;
-      const int tau = g * kPageTokens + tk;
-      uint4 x;
-      if (tau < T0) {
-        x = *reinterpret_cast<const uint4*>(win + (r * kPageTokens + (tau % kPageTokens)) * D + c8);
-      } else {
-        const int64_t row = off + (tau - T0);
-        x = load8<F32IN>(r ? a.V : a.K, (row * H + h) * D + c8);
+    auto stage = [&](int it, int buf) {
+      const int g = g0 + it;
+      for (int v = threadIdx.x; v < 2 * kPageTokens * VPR; v += kThreads) {
+        const int r = v / (kPageTokens * VPR), rem = v % (kPageTokens * VPR);
+        const int tk = rem / VPR, c8 = (rem % VPR) * 8;
+        const int tau = g * kPageTokens + tk;  // old window slots first
+        const bool from_win = tau < T0;
+        const int64_t idx = ((off + (tau - T0)) * H + h) * D + c8;
+        const __nv_bfloat16* wsrc = win + (r * kPageTokens + (tau % kPageTokens)) * D + c8;
+        if constexpr (F32IN) {
+          *reinterpret_cast<uint4*>(&xsb[buf][r][tk][c8]) =
+              from_win ? *reinterpret_cast<const uint4*>(wsrc) : load8<true>(r ? a.V : a.K, idx);
+        } else {
+          cp_async16(&xsb[buf][r][tk][c8],
+                     from_win ? wsrc : reinterpret_cast<const __nv_bfloat16*>(r ? a.V : a.K) + idx);
+        }
       }
-      *reinterpret_cast<uint4*>(&xs[r][tk][c8]) = x;
-    }
-    __syncthreads();
-    if constexpr (kBf16Layer) {
-      store_block<16, D>(page, false, [&](int tok, int dim) { return (uint32_t)__bfloat16_as_ushort(xs[0][tok][dim]); });
-      store_block<16, D>(page + code_block_bytes(16, D), true,
-                         [&](int tok, int dim) { return (uint32_t)__bfloat16_as_ushort(xs[1][tok][dim]); });
-    } else {
-      double err[4] = {0.0, 0.0, 0.0, 0.0};  // this thread's share of the error report
-      auto add_err = [&](int r, float x, double xh) {
-        const double dx = (double)x - xh;
-        err[2 * r] += dx * dx;
-        err[2 * r + 1] += (double)x * (double)x;
-      };
-      if (a.fmt != 0) {
-        if constexpr (KB == 8 && VB == 8) {
-          const float sc[2] = {a.fp8_scales[h], a.fp8_scales[H + h]};
-          auto code = [&](int r, int tok, int dim) -> uint32_t {
-            const float x = __bfloat162float(xs[r][tok][dim]);
-            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(__fdiv_rn(x, sc[r]), __NV_SATFINITE, __NV_E4M3);
-            add_err(r, x, (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3))) * sc[r]);
-            return (uint32_t)c;
+      cp_async_commit();
+    };
+    double err[4] = {0.0, 0.0, 0.0, 0.0};  // this thread's share of the error report
+    int groups = 0;
+    stage(item, 0);
+    for (int it = item, buf = 0; it < ng; it += gridDim.x, buf ^= 1, ++groups) {
+      if (it + (int)gridDim.x < ng) {
+        stage(it + (int)gridDim.x, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      const int g = g0 + it;
+      uint8_t* page = a.pages + ((int64_t)(b * H + h) * a.max_pages + g) * a.page_bytes;
+      auto& xs = xsb[buf];
+      __syncthreads();
+      if constexpr (kBf16Layer) {
+        emit_bf16<D, RS>(page, xs[0], false);
+        emit_bf16<D, RS>(page + code_block_bytes(16, D), xs[1], true);
+      } else {
+        auto add_err = [&](int r, float x, double xh) {
+          const double dx = (double)x - xh;
+          err[2 * r] += dx * dx;
+          err[2 * r + 1] += (double)x * (double)x;
+        };
+        if (a.fmt != 0) {
+          if constexpr (KB == 8 && VB == 8) {
+            const float sc[2] = {a.fp8_scales[h], a.fp8_scales[H + h]};
+            auto code = [&](int r, int tok, int dim) -> uint32_t {
+              const float x = __bfloat162float(xs[r][tok][dim]);
+              const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(__fdiv_rn(x, sc[r]), __NV_SATFINITE, __NV_E4M3);
+              add_err(r, x, (double)__half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3))) * sc[r]);
+              return (uint32_t)c;
+            };
+            store_block<8, D>(page, false, [&](int tok, int dim) { return code(0, tok, dim); });
+            store_block<8, D>(page + code_block_bytes(8, D), true, [&](int tok, int dim) { return code(1, tok, dim); });
+          }
+        } else {
+          const bool per_token_keys = a.key_mode != 0;
+          const int nk = per_token_keys ? kPageTokens : D;  // key scale/zero pairs
+          uint8_t* vblk = page + code_block_bytes(KB, D);
+          __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
+          __half* kzero = kscale + nk;
+          __half* vscale = kzero + nk;
+          __half* vzero = vscale + kPageTokens;
+          auto keep = [&](int r, int i, const QParams& q) {
+            qzr[r][i] = make_float2(q.z, q.r);  // r = 0 for a constant set
+            qzs[r][i] = make_double2((double)q.z, (double)__half2float(q.s_h));
           };
-          store_block<8, D>(page, false, [&](int tok, int dim) { return code(0, tok, dim); });
-          store_block<8, D>(page + code_block_bytes(8, D), true, [&](int tok, int dim) { return code(1, tok, dim); });
-        }
-      } else {
-        const bool per_token_keys = a.key_mode != 0;
-        const int nk = per_token_keys ? kPageTokens : D;  // key scale/zero pairs
-        uint8_t* vblk = page + code_block_bytes(KB, D);
-        __half* kscale = reinterpret_cast<__half*>(vblk + code_block_bytes(VB, D));
-        __half* kzero = kscale + nk;
-        __half* vscale = kzero + nk;
-        __half* vzero = vscale + kPageTokens;
-        auto keep = [&](int r, int i, const QParams& q) {
-          pz[r][i] = q.z;
-          pr[r][i] = q.r;  // 0 for a constant set
-          ps[r][i] = __half2float(q.s_h);
-        };
-        // one warp per token over the head dimension: row r of xs (0 keys, 1 values)
-        auto quantize_tokens = [&](int r, int qmax, __half* sdst, __half* zdst) {
-          const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-          for (int t = warp; t < kPageTokens; t += kThreads / 32) {
-            float mn = __bfloat162float(xs[r][t][lane]), mx = mn;
+          // per-token sets (values; keys in per-token mode): four threads per token,
+          // thread u taking the bf16 pairs u, u + 4, ... of the row
+          auto token_params = [&](int r, int qmax, __half* sdst, __half* zdst) {
+            const int tok = threadIdx.x >> 2, u = threadIdx.x & 3;
+            const __nv_bfloat162* row = reinterpret_cast<const __nv_bfloat162*>(&xs[r][tok][0]);
+            __nv_bfloat162 mn = row[u], mx = mn;
 #pragma unroll
-            for (int k = 1; k < D / 32; ++k) {
-              const float x = __bfloat162float(xs[r][t][lane + 32 * k]);
-              mn = fminf(mn, x);
-              mx = fmaxf(mx, x);
+            for (int k = 1; k < D / 8; ++k) {
+              mn = __hmin2(mn, row[u + 4 * k]);
+              mx = __hmax2(mx, row[u + 4 * k]);
             }
+            float fmn = fminf(__low2float(mn), __high2float(mn)), fmx = fmaxf(__low2float(mx), __high2float(mx));
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            for (int o = 1; o < 4; o <<= 1) {
+              fmn = fminf(fmn, __shfl_xor_sync(0xffffffffu, fmn, o));
+              fmx = fmaxf(fmx, __shfl_xor_sync(0xffffffffu, fmx, o));
             }
-            if (lane == 0) {
-              const QParams q = make_qparams(mn, mx, qmax);
-              sdst[t] = q.s_h;
-              zdst[t] = q.z_h;
-              keep(r, t, q);
+            if (u == 0) {
+              const QParams q = make_qparams(fmn, fmx, qmax);
+              sdst[tok] = q.s_h;
+              zdst[tok] = q.z_h;
+              keep(r, tok, q);
+            }
+          };
+          token_params(1, (1 << VB) - 1, vscale, vzero);
+          if (per_token_keys) {
+            token_params(0, (1 << KB) - 1, kscale, kzero);
+          } else {
+            // keys per channel: thread (split, pair) scans 32/KS tokens of one channel
+            // pair; the splits are then combined, one thread per channel
+            const int pi = threadIdx.x % KP, sp = threadIdx.x / KP;
+            const __nv_bfloat162* col = reinterpret_cast<const __nv_bfloat162*>(&xs[0][sp * (kPageTokens / KS)][0]) + pi;
+            __nv_bfloat162 mn = col[0], mx = mn;
+#pragma unroll
+            for (int k = 1; k < kPageTokens / KS; ++k) {
+              mn = __hmin2(mn, col[k * (RS / 2)]);
+              mx = __hmax2(mx, col[k * (RS / 2)]);
+            }
+            kpart[sp][0][pi] = mn;
+            kpart[sp][1][pi] = mx;
+            __syncthreads();
+            for (int d = threadIdx.x; d < D; d += kThreads) {
+              float fmn = 0.0f, fmx = 0.0f;
+#pragma unroll
+              for (int k = 0; k < KS; ++k) {
+                const __nv_bfloat162 m0 = kpart[k][0][d >> 1], m1 = kpart[k][1][d >> 1];
+                const float x0 = (d & 1) ? __high2float(m0) : __low2float(m0);
+                const float x1 = (d & 1) ? __high2float(m1) : __low2float(m1);
+                fmn = k ? fminf(fmn, x0) : x0;
+                fmx = k ? fmaxf(fmx, x1) : x1;
+              }
+              const QParams q = make_qparams(fmn, fmx, (1 << KB) - 1);
+              const int slot = kmeta_slot<D>(d);
+              kscale[slot] = q.s_h;
+              kzero[slot] = q.z_h;
+              keep(0, d, q);
             }
           }
-        };
-        if (per_token_keys) quantize_tokens(0, (1 << KB) - 1, kscale, kzero);
-        // keys (per-channel mode): one thread per channel, over the group's 32 tokens
-        for (int d = threadIdx.x; d < (per_token_keys ? 0 : D); d += kThreads) {
-          float mn = __bfloat162float(xs[0][0][d]), mx = mn;
-#pragma unroll 8
-          for (int t = 1; t < kPageTokens; ++t) {
-            const float x = __bfloat162float(xs[0][t][d]);
-            mn = fminf(mn, x);
-            mx = fmaxf(mx, x);
-          }
-          const QParams q = make_qparams(mn, mx, (1 << KB) - 1);
-          const int slot = kmeta_slot<D>(d);
-          kscale[slot] = q.s_h;
-          kzero[slot] = q.z_h;
-          keep(0, d, q);
+          __syncthreads();
+          // codes, each element quantized as it is packed, and its error report terms
+          double ek[2] = {0.0, 0.0}, ev[2] = {0.0, 0.0};
+          if (per_token_keys) emit_codes<KB, D, RS, 1>(page, xs[0], QTab{qzr[0], qzs[0]}, ek);
+          else emit_codes<KB, D, RS, 0>(page, xs[0], QTab{qzr[0], qzs[0]}, ek);
+          emit_codes<VB, D, RS, 2>(vblk, xs[1], QTab{qzr[1], qzs[1]}, ev);
+          err[0] += ek[0];
+          err[1] += ek[1];
+          err[2] += ev[0];
+          err[3] += ev[1];
         }
-        quantize_tokens(1, (1 << VB) - 1, vscale, vzero);
-        __syncthreads();
-        // codes, each element quantized as it is packed, and its error report terms
-        emit_block<0, KB, D, RS>(page, per_token_keys, xs[0], pz[0], pr[0], ps[0], err);
-        emit_block<1, VB, D, RS>(vblk, true, xs[1], pz[1], pr[1], ps[1], err);
       }
-      // this flush's error sums: warp shuffles, then one fp64 atomic per sum into
+      __syncthreads();  // the staged rows and the parameter tables are reused
+    }
+    if constexpr (!kBf16Layer) {
+      // this CTA's error sums: warp shuffles, then one fp64 atomic per sum into
       // one of the layer's bins
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
@@ -349,7 +471,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams a) {
         for (int w = 0; w < kThreads / 32; ++w) v += red[w][threadIdx.x];
         atomicAdd(&bin[threadIdx.x], v);
       }
-      if (bin && threadIdx.x == 4) atomicAdd(&bin[4], (double)(kPageTokens * D));
+      if (bin && threadIdx.x == 4) atomicAdd(&bin[4], (double)groups * (kPageTokens * D));
     }
   }
 

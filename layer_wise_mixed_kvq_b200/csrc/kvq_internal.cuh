@@ -187,6 +187,9 @@ int choose_chunk(int sm_count, int64_t total_pages, int64_t max_pages_per_seq, i
 // Overhead units per segment for the tensor-core kernel's balanced slices
 // (KVQ_SEG_OVERHEAD_UNITS overrides the default).
 int seg_overhead_units();
+// Completed 32-token groups of one sequence-head per append CTA in multi-token
+// appends (KVQ_APPEND_GROUPS_PER_CTA overrides).
+int append_groups_per_cta();
 // Message returned by kvq_last_error() on this thread.
 void set_last_error(const std::string& msg);
 // KVQ_DECODE_KERNEL=simt: the CUDA-core decode kernel instead of the tensor-core one.
