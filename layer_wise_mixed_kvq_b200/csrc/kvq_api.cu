@@ -174,6 +174,15 @@ int append_groups_per_cta() {
   return v;
 }
 
+int64_t early_l2_bytes() {
+  static const int64_t v = [] {
+    const char* e = std::getenv("KVQ_EARLY_L2_MB");
+    const int64_t mb = e ? std::atoll(e) : 48;
+    return (mb < 0 ? 0 : (mb > 96 ? 96 : mb)) << 20;
+  }();
+  return v;
+}
+
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_p, int64_t stride) {
   const int64_t target_ctas = (int64_t)sm_count * 3;
   int64_t chunk = std::max<int64_t>(8, (total_pages + target_ctas - 1) / target_ctas);
@@ -550,6 +559,7 @@ static kvq_status decode_params(kvq_cache* c, int layer, const void* Q, int batc
     for (int b = 0; b < batch; ++b) p.hlen[b] = (int32_t)lens[b];
     const int w = stream_written_layer(c, stream);
     p.early = (w != layer && w != -2) ? 1 : 0;
+    p.early_l2_bytes = kvq::early_l2_bytes();
   }
   if (append) {
     p.append = 1;
@@ -571,7 +581,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* Q, int batch, fl
   if (!Q || !out) return fail(KVQ_EINVAL, "Q or out is null");
   if (!aligned16(Q) || !aligned16(out)) return fail(KVQ_EINVAL, "Q and out must be 16-byte aligned");
   const kvq::LayerState& L = c->layers[layer];
-  kvq::DecodeParams p;
+  kvq::DecodeParams p{};
   st = decode_params(c, layer, Q, batch, out, stream, false, L.host_len, p);
   if (st != KVQ_OK) return st;
   int splits = 1;
@@ -603,7 +613,7 @@ kvq_status kvq_decode_step(kvq_cache* c, int layer, const void* K, const void* V
     st = kvq_append(c, layer, K, V, KVQ_BF16, ones.data(), batch, stream);
     return st != KVQ_OK ? st : kvq_decode_attn(c, layer, Q, batch, out, stream);
   }
-  kvq::DecodeParams p;
+  kvq::DecodeParams p{};
   st = decode_params(c, layer, Q, batch, out, stream, true, L.host_len, p);
   if (st != KVQ_OK) return st;
   p.k_new = static_cast<const __nv_bfloat16*>(K);

@@ -120,14 +120,35 @@ __device__ __forceinline__ void load_tile(uint32_t (&a)[4], const __nv_bfloat16 
   else ldsm_x4(a, &xs[16 * tt + r + 8 * (m & 1)][16 * dt + 8 * (m >> 1)]);
 }
 
-// One element's code, as the bits of the fp32 number 1.5 * 2^23 + code: for y in
-// [0, qmax] the single rounding of the addition is rint(y), round-half-even.
-// The clamp to [0, qmax] first gives clamp(rint(y), 0, qmax) for every y
-// (fmaxf also maps a NaN to 0), and a zero reciprocal (constant set) gives 0.
+// Two elements' codes, as the bits of the fp32 numbers 1.5 * 2^23 + code: for y
+// in [0, qmax] the single rounding of the addition is rint(y), round-half-even.
+// y = (x - z) * (1/s), x - z formed as x + (-z) (the same IEEE result), clamped
+// to [0, qmax] first, which gives clamp(rint(y), 0, qmax) for every y (fmaxf
+// also maps a NaN to 0); a zero reciprocal (constant set) gives 0. Two elements
+// per packed fp32 operation, each with an explicit rounding mode.
 constexpr uint32_t kRintBias = 0x4B400000u;  // bits of 1.5 * 2^23
-__device__ __forceinline__ uint32_t code_bits(float x, float z, float r, float qmax) {
-  const float y = fminf(fmaxf(__fmul_rn(__fsub_rn(x, z), r), 0.0f), qmax);
-  return __float_as_uint(__fadd_rn(y, 12582912.0f));
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "add.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mul.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ uint2 code_bits2(float2 x, float2 nz, float2 r, float qmax) {
+  float2 y = mul2_rn(add2_rn(x, nz), r);
+  y.x = fminf(fmaxf(y.x, 0.0f), qmax);
+  y.y = fminf(fmaxf(y.y, 0.0f), qmax);
+  const float2 m = add2_rn(y, make_float2(12582912.0f, 12582912.0f));
+  return make_uint2(__float_as_uint(m.x), __float_as_uint(m.y));
 }
 
 // Error report terms of one element: (x - x_hat)^2 and x^2 in fp64, with
@@ -144,8 +165,9 @@ __device__ __forceinline__ void add_error(double (&e)[2], float x, uint32_t bits
 // Quantizer parameters of one index (a channel or a token): z and 1/s in fp32
 // for the code, z and s in fp64 for the error report.
 struct QTab {
-  const float2* zr;
-  const double2* zs;
+  const float* nz;     // -z
+  const float* r;      // 1/s, 0 for a constant set
+  const double2* zs;   // z, s
 };
 
 // Integer code block of BITS-bit codes. Lane l's 16-byte vector vi holds tiles
@@ -160,72 +182,72 @@ __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*x
   constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
   constexpr float qmax = (float)((1 << BITS) - 1);
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  // parameters of the element pair (p, 0), (p, 1) of a tile: index h = p>>1
+  // (MODE 0, 2: indices i0 + 8h, +1) or h = p&1 (MODE 1: one token for both)
+  struct Pair {
+    float2 nz, r;
+    double2 zs0, zs1;
+  };
+  auto load_pair = [&](int i, bool one) {
+    Pair pr;
+    if (one) {
+      pr.nz = make_float2(q.nz[i], q.nz[i]);
+      pr.r = make_float2(q.r[i], q.r[i]);
+      pr.zs0 = pr.zs1 = q.zs[i];
+    } else {
+      pr.nz = *reinterpret_cast<const float2*>(q.nz + i);
+      pr.r = *reinterpret_cast<const float2*>(q.r + i);
+      pr.zs0 = q.zs[i];
+      pr.zs1 = q.zs[i + 1];
+    }
+    return pr;
+  };
   for (int v = threadIdx.x; v < kVectors; v += kThreads) {
     const int vi = v >> 5;
     uint32_t w[4] = {0u, 0u, 0u, 0u};
-    // one element: quantize, add its error terms, add its code into its field
-    auto put = [&](int i, int p, int j, float x, float2 zr, double2 zs) {
-      const uint32_t bits = code_bits(x, zr.x, zr.y, qmax);
-      add_error(e, x, bits, zs);
+    // one element pair: quantize, add the error terms, add the codes into their fields
+    auto put = [&](int i, int p, uint32_t a, const Pair& pr) {
+      const float2 x = make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+      const uint2 bits = code_bits2(x, pr.nz, pr.r, qmax);
+      add_error(e, x.x, bits.x, pr.zs0);
+      add_error(e, x.y, bits.y, pr.zs1);
       // (bits - bias) << shift is the code in place; words only gain disjoint fields
-      if constexpr (BITS == 4) w[i] += (bits - kRintBias) << (4 * (p + 4 * j));
-      else if constexpr (BITS == 2) w[i >> 1] += (bits - kRintBias) << (2 * (4 * (i & 1) + p + 8 * j));
-      else w[2 * i + (p >> 1)] += (bits - kRintBias) << (8 * (2 * (p & 1) + j));
-    };
-    auto elem = [](const uint32_t (&a)[4], int p, int j) {
-      return __uint_as_float(j ? (a[p] & 0xFFFF0000u) : (a[p] << 16));
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t c = (j ? bits.y : bits.x) - kRintBias;
+        if constexpr (BITS == 4) w[i] += c << (4 * (p + 4 * j));
+        else if constexpr (BITS == 2) w[i >> 1] += c << (2 * (4 * (i & 1) + p + 8 * j));
+        else w[2 * i + (p >> 1)] += c << (8 * (2 * (p & 1) + j));
+      }
     };
     if constexpr (MODE == 0) {
       // parameters by channel 16dt + 2t + j + 8(p>>1): shared by both token halves
 #pragma unroll
       for (int d2 = 0; d2 < TPV / 2; ++d2) {
         const int dt = vi * (TPV / 2) + d2;
-        float2 zr[2][2];
-        double2 zs[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            zr[h][j] = q.zr[16 * dt + 2 * t + j + 8 * h];
-            zs[h][j] = q.zs[16 * dt + 2 * t + j + 8 * h];
-          }
+        const Pair pr[2] = {load_pair(16 * dt + 2 * t, false), load_pair(16 * dt + 2 * t + 8, false)};
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
           uint32_t a[4];
           load_tile<RS>(a, xs, false, dt, tt, lane);
 #pragma unroll
-          for (int p = 0; p < 4; ++p)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) put(2 * d2 + tt, p, j, elem(a, p, j), zr[p >> 1][j], zs[p >> 1][j]);
+          for (int p = 0; p < 4; ++p) put(2 * d2 + tt, p, a[p], pr[p >> 1]);
         }
       }
     } else {
-      // parameters by token: 16tt + g + 8(p&1) (keys, MODE 1) or 16tt + 2t + j + 8(p>>1)
-      // (values), shared by every tile row of a token half
+      // parameters by token 16tt + g + 8(p&1) (keys, MODE 1) or 16tt + 2t + j + 8(p>>1)
+      // (values): shared by every tile row of a token half
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
-        float2 zr[2][2];
-        double2 zs[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int i = MODE == 1 ? 16 * tt + g + 8 * h : 16 * tt + 2 * t + j + 8 * h;
-            zr[h][j] = q.zr[i];
-            zs[h][j] = q.zs[i];
-          }
+        const Pair pr[2] = {MODE == 1 ? load_pair(16 * tt + g, true) : load_pair(16 * tt + 2 * t, false),
+                            MODE == 1 ? load_pair(16 * tt + g + 8, true) : load_pair(16 * tt + 2 * t + 8, false)};
 #pragma unroll
         for (int d2 = 0; d2 < TPV / 2; ++d2) {
           const int dt = vi * (TPV / 2) + d2;
           uint32_t a[4];
           load_tile<RS>(a, xs, MODE == 2, dt, tt, lane);
 #pragma unroll
-          for (int p = 0; p < 4; ++p)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int h = MODE == 1 ? (p & 1) : (p >> 1), jj = MODE == 1 ? 0 : j;
-              put(2 * d2 + tt, p, j, elem(a, p, j), zr[h][jj], zs[h][jj]);
-            }
+          for (int p = 0; p < 4; ++p) put(2 * d2 + tt, p, a[p], pr[MODE == 1 ? (p & 1) : (p >> 1)]);
         }
       }
     }
@@ -247,7 +269,7 @@ __device__ __forceinline__ void emit_bf16(uint8_t* blk, const __nv_bfloat16 (*xs
 }
 
 template <int KB, int VB, int D, bool F32IN>
-__global__ void __launch_bounds__(kThreads, (KB == 2 || VB == 2) ? 3 : 4) append_kernel(AppendParams a) {
+__global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
   pdl_enter();
   constexpr bool kBf16Layer = (KB == 16);
   constexpr int RS = D + 8;          // bf16 row stride of the staged rows (16-byte rows, staggered banks)
@@ -255,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, (KB == 2 || VB == 2) ? 3 : 4) append
   const int b = blockIdx.z, h = blockIdx.y, item = blockIdx.x;
   const int H = a.n_kv_heads;
   __shared__ __align__(16) __nv_bfloat16 xsb[2][2][kPageTokens][RS];  // two groups' key and value rows
-  __shared__ __align__(16) float2 qzr[2][NP];   // quantizer z, 1/s by index: keys, values
+  __shared__ __align__(16) float qnz[2][NP];    // quantizer -z by index: keys, values
+  __shared__ __align__(16) float qr[2][NP];     // 1/s (0 for a constant set)
   __shared__ __align__(16) double2 qzs[2][NP];  // z, s in fp64 (error report)
   constexpr int KP = D / 2, KS = kThreads / KP;  // key channel pairs, token splits of the key pass
   __shared__ __nv_bfloat162 kpart[KS][2][KP];   // per-split min, max of each key channel pair
@@ -377,7 +400,8 @@ __global__ void __launch_bounds__(kThreads, (KB == 2 || VB == 2) ? 3 : 4) append
           __half* vscale = kzero + nk;
           __half* vzero = vscale + kPageTokens;
           auto keep = [&](int r, int i, const QParams& q) {
-            qzr[r][i] = make_float2(q.z, q.r);  // r = 0 for a constant set
+            qnz[r][i] = -q.z;
+            qr[r][i] = q.r;  // 0 for a constant set
             qzs[r][i] = make_double2((double)q.z, (double)__half2float(q.s_h));
           };
           // per-token sets (values; keys in per-token mode): four threads per token,
@@ -441,9 +465,10 @@ __global__ void __launch_bounds__(kThreads, (KB == 2 || VB == 2) ? 3 : 4) append
           __syncthreads();
           // codes, each element quantized as it is packed, and its error report terms
           double ek[2] = {0.0, 0.0}, ev[2] = {0.0, 0.0};
-          if (per_token_keys) emit_codes<KB, D, RS, 1>(page, xs[0], QTab{qzr[0], qzs[0]}, ek);
-          else emit_codes<KB, D, RS, 0>(page, xs[0], QTab{qzr[0], qzs[0]}, ek);
-          emit_codes<VB, D, RS, 2>(vblk, xs[1], QTab{qzr[1], qzs[1]}, ev);
+          const QTab tk{qnz[0], qr[0], qzs[0]}, tv{qnz[1], qr[1], qzs[1]};
+          if (per_token_keys) emit_codes<KB, D, RS, 1>(page, xs[0], tk, ek);
+          else emit_codes<KB, D, RS, 0>(page, xs[0], tk, ek);
+          emit_codes<VB, D, RS, 2>(vblk, xs[1], tv, ev);
           err[0] += ek[0];
           err[1] += ek[1];
           err[2] += ev[0];
