@@ -174,15 +174,6 @@ int append_groups_per_cta() {
   return v;
 }
 
-int64_t early_l2_bytes() {
-  static const int64_t v = [] {
-    const char* e = std::getenv("KVQ_EARLY_L2_MB");
-    const int64_t mb = e ? std::atoll(e) : 48;
-    return (mb < 0 ? 0 : (mb > 96 ? 96 : mb)) << 20;
-  }();
-  return v;
-}
-
 int choose_chunk(int sm_count, int64_t total_pages, int64_t max_p, int64_t stride) {
   const int64_t target_ctas = (int64_t)sm_count * 3;
   int64_t chunk = std::max<int64_t>(8, (total_pages + target_ctas - 1) / target_ctas);
@@ -559,7 +550,6 @@ static kvq_status decode_params(kvq_cache* c, int layer, const void* Q, int batc
     for (int b = 0; b < batch; ++b) p.hlen[b] = (int32_t)lens[b];
     const int w = stream_written_layer(c, stream);
     p.early = (w != layer && w != -2) ? 1 : 0;
-    p.early_l2_bytes = kvq::early_l2_bytes();
   }
   if (append) {
     p.append = 1;

@@ -1649,25 +1649,7 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
     if (lane == 0 && work)
       for (int r = 0; r < C::R && !pdone; ++r) grab(r);
   };
-  if (p.host_units && p.early) {
-    issue_first();
-    // While the preceding kernel finishes, also bring the slice's pages into L2
-    // (up to p.early_l2_bytes over the whole grid, in slice order) so that the HBM
-    // reads of this launch start under that kernel's tail.
-    if (threadIdx.x == 0 && work) {
-      int64_t budget = (p.early_l2_bytes / (int64_t)gridDim.x) & ~(int64_t)15;
-      PageWalk w;
-      w.a = w.e = u0;
-      w.k0 = w.n = w.ord0 = 0;
-      w.base = nullptr;
-      for (int o = 0; budget > 0 && walk_to(w, o, p, ustart, slen, B, u1); o = w.ord0 + w.n) {
-        const uint8_t* src = w.base + (int64_t)w.k0 * p.page_bytes;
-        const int64_t bytes = min((int64_t)w.n * p.page_bytes, budget);
-        for (int64_t off = 0; off < bytes; off += 32768) prefetch_l2(src + off, (uint32_t)min((int64_t)32768, bytes - off));
-        budget -= bytes;
-      }
-    }
-  }
+  if (p.host_units && p.early) issue_first();
   if (p.host_units) pdl_enter();
   if (!(p.host_units && p.early)) issue_first();
   if (!work) return;  // no copy was issued

@@ -128,9 +128,6 @@ struct DecodeParams {
   // written by it)
   int host_units;
   int early;
-  // with `early`: bytes of the launch's pages (whole grid, in slice order) also
-  // prefetched into L2 before that wait
-  int64_t early_l2_bytes;
   int32_t hlen[kHostLens];
 };
 
@@ -193,8 +190,6 @@ int seg_overhead_units();
 // Completed 32-token groups of one sequence-head per append CTA in multi-token
 // appends (KVQ_APPEND_GROUPS_PER_CTA overrides).
 int append_groups_per_cta();
-// Early L2 prefetch budget of a decode launch in bytes (KVQ_EARLY_L2_MB overrides).
-int64_t early_l2_bytes();
 // Message returned by kvq_last_error() on this thread.
 void set_last_error(const std::string& msg);
 // KVQ_DECODE_KERNEL=simt: the CUDA-core decode kernel instead of the tensor-core one.
