@@ -79,8 +79,9 @@ def kernel_source_hash():
 
 
 def traffic_from_profile(workload):
-    """DRAM bytes per decode launch from the committed ncu summary, only if its
-    counters were taken on the current kernel source (else None)."""
+    """The committed ncu DRAM counters of one decode launch of the workload's
+    shapes, only if they were taken on the current kernel source (else None):
+    the entry's traffic_ratio is DRAM bytes / algorithmic bytes of that launch."""
     path = os.path.join(PROFILES, "decode_traffic.json")
     if not os.path.exists(path):
         return None
@@ -89,7 +90,7 @@ def traffic_from_profile(workload):
     e = d.get(workload)
     if not e or e.get("counters_taken_at") != kernel_source_hash():
         return None
-    return e.get("dram_bytes_per_launch")
+    return e
 
 
 # --------------------------------------------------------------- clocks --
@@ -367,13 +368,18 @@ def measure(w, args, world, full):
     ms_per_step = max_ms / args.steps
     value = total_bytes / (max_ms / 1e3) / 1e9
     launch_us = local_ms * 1e3 / (args.steps * NL)
-    traffic = traffic_from_profile(w.name)
+    # DRAM traffic of a launch: the captured launch's bytes per algorithmic byte
+    # times this run's algorithmic bytes per launch (the capture ran a 2-layer
+    # stack of the same shapes; the traffic grows with the units processed)
+    prof = traffic_from_profile(w.name)
+    traffic = prof["traffic_ratio"] * bytes_per_step / NL if prof else None
     res = {
         "value": value, "unit": "GB/s", "ms_per_step": ms_per_step, "decode_steps_per_s": 1e3 / ms_per_step,
         "tokens_per_s": B * world * 1e3 / ms_per_step, "bytes_per_step": bytes_per_step,
         "append_prefill_tokens_per_s": append["tokens_per_s"], "append": append,
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
-                     "frac": value / world / peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "frac": value / world / peak, "traffic": traffic,
+                     "traffic_ratio": prof["traffic_ratio"] if prof else None, "peak_kind": peak_kind,
                      "avg_launch_us": launch_us, "algorithmic_bytes_per_launch": bytes_per_step / NL,
                      "kernel": "fused decode step (decode_mma_kernel / decode_warp_kernel with the one-token "
                                "append): every launch of the timed region, average duration = region / launches"},
@@ -492,7 +498,7 @@ def run_gpu(args, w):
             per_config[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "decode_steps_per_s",
                                                   "append_prefill_tokens_per_s", "bytes_per_step", "gpu_launches")}
             per_config[name]["roofline"] = {k: r["roofline"][k] for k in ("achieved", "frac", "traffic",
-                                                                          "avg_launch_us")}
+                                                                          "traffic_ratio", "avg_launch_us")}
             per_config[name]["append_roofline_frac"] = r["append"]["roofline"]["frac"]
             per_config[name]["clocks"] = r["clocks"]
             per_config[name]["config"] = workload_config(synth.WORKLOADS[name],
