@@ -1871,89 +1871,63 @@ __global__ void __launch_bounds__(kThreads, TOK ? Cfg<KB, VB, D, PT, F8>::MINB_T
       }
       __syncthreads();
       if (s_last) {
-        // The slices' records, every load in flight at once: their maxima and sums
-        // into the (now free) merge area, then the accumulators in batches of 8,
-        // four channels per thread, each weighted by 2^(m_c - M). An empty slice,
-        // or a record with no scores (m = -inf), has weight 0 and is read from this
-        // CTA's own record in its place.
+        // The slices' records, four channels per thread, 4, 8 or 16 records per
+        // round with all their loads in flight at once (maximum, sum and
+        // accumulators), each weighted by 2^(m_c - M); rounds are joined by online
+        // rescaling. An empty slice (or a padding entry of a round) has weight 0 and
+        // is read from this CTA's own record in its place.
         const int nrec = c_hi - c_lo + 1;
         const int64_t rec_floats = split_record_floats(G, D);
-        auto record = [&](int c) {
-          const int slot = (sl.lo(c) >= sg.start) ? 0 : 1;
-          return p.partials + ((int64_t)c * 2 + slot) * rec_floats;
-        };
-        if (nrec > (kWarps + 1) * D / 2) {
-          // more records than the merge area holds maxima and sums for (a segment
-          // spread over hundreds of CTAs): one pass, online rescaling
-          for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += kThreads) {
-            const int gg = (4 * i4) / D, d = (4 * i4) % D;
-            float M = -INFINITY, L = 0.f;
-            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int c = c_lo; c <= c_hi; ++c) {
-              if (sl.empty(c)) continue;
-              const float* r = record(c);
-              const float mc = __ldcg(r + G * D + gg), lc = __ldcg(r + G * D + G + gg);
-              const float4 oc = __ldcg(reinterpret_cast<const float4*>(r + gg * D + d));
-              const float Mn = fmaxf(M, mc);
-              const float fa = (M == -INFINITY) ? 0.f : exp2f(M - Mn);
-              const float fb = (mc == -INFINITY) ? 0.f : exp2f(mc - Mn);
-              L = L * fa + lc * fb;
-              O.x = O.x * fa + oc.x * fb;
-              O.y = O.y * fa + oc.y * fb;
-              O.z = O.z * fa + oc.z * fb;
-              O.w = O.w * fa + oc.w * fb;
-              M = Mn;
-            }
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            *reinterpret_cast<float4*>(outp + gg * D + d) = make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
-          }
-        } else {
-          float* rm = mo;              // [nrec][G] maxima
-          float* rl = mo + nrec * G;   // [nrec][G] sums
-          for (int i = threadIdx.x; i < nrec * G; i += kThreads) {
-            const int c = c_lo + i / G, gg = i % G;
-            float m = -INFINITY, l = 0.f;
-            if (!sl.empty(c)) {
-              const float* r = record(c);
-              m = __ldcg(r + G * D + gg);
-              l = __ldcg(r + G * D + G + gg);
-            }
-            rm[i] = m;
-            rl[i] = l;
-          }
-          __syncthreads();
-          for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += kThreads) {
-            const int gg = (4 * i4) / D, d = (4 * i4) % D;
-            float M = -INFINITY;
-            for (int k = 0; k < nrec; ++k) M = fmaxf(M, rm[k * G + gg]);
-            float L = 0.f;
-            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (M != -INFINITY) {
-              for (int k0 = 0; k0 < nrec; k0 += 8) {
-                float w[8];
-                float4 oc[8];
+        for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += kThreads) {
+          const int gg = (4 * i4) / D, d = (4 * i4) % D;
+          float M = -INFINITY, L = 0.f;
+          float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+          // one round of R records starting at record k0
+          auto merge_round = [&](auto rounds, int k0) {
+            constexpr int R = decltype(rounds)::value;
+            float mc[R], lc[R];
+            float4 oc[R];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const int k = k0 + j;
-                  const float mc = k < nrec ? rm[k * G + gg] : -INFINITY;
-                  w[j] = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-                  const float* r = (mc == -INFINITY) ? part : record(c_lo + k);
-                  oc[j] = __ldcg(reinterpret_cast<const float4*>(r + gg * D + d));
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const int k = k0 + j;
-                  if (k < nrec) L = fmaf(w[j], rl[k * G + gg], L);
-                  O.x = fmaf(w[j], oc[j].x, O.x);
-                  O.y = fmaf(w[j], oc[j].y, O.y);
-                  O.z = fmaf(w[j], oc[j].z, O.z);
-                  O.w = fmaf(w[j], oc[j].w, O.w);
-                }
-              }
+            for (int j = 0; j < R; ++j) {
+              const int c = c_lo + k0 + j;
+              const bool valid = k0 + j < nrec && !sl.empty(c);
+              const float* r =
+                  valid ? p.partials + ((int64_t)c * 2 + ((sl.lo(c) >= sg.start) ? 0 : 1)) * rec_floats : part;
+              const float m = __ldcg(r + G * D + gg);
+              mc[j] = valid ? m : -INFINITY;
+              lc[j] = __ldcg(r + G * D + G + gg);
+              oc[j] = __ldcg(reinterpret_cast<const float4*>(r + gg * D + d));
             }
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            *reinterpret_cast<float4*>(outp + gg * D + d) = make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+            float Mn = M;
+#pragma unroll
+            for (int j = 0; j < R; ++j) Mn = fmaxf(Mn, mc[j]);
+            if (Mn == -INFINITY) return;
+            const float fa = (M == -INFINITY) ? 0.f : exp2f(M - Mn);
+            L *= fa;
+            O.x *= fa;
+            O.y *= fa;
+            O.z *= fa;
+            O.w *= fa;
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+              const float w = (mc[j] == -INFINITY) ? 0.f : exp2f(mc[j] - Mn);
+              L = fmaf(w, lc[j], L);
+              O.x = fmaf(w, oc[j].x, O.x);
+              O.y = fmaf(w, oc[j].y, O.y);
+              O.z = fmaf(w, oc[j].z, O.z);
+              O.w = fmaf(w, oc[j].w, O.w);
+            }
+            M = Mn;
+          };
+          if (nrec <= 4) {
+            merge_round(std::integral_constant<int, 4>{}, 0);
+          } else if (nrec <= 8) {
+            merge_round(std::integral_constant<int, 8>{}, 0);
+          } else {
+            for (int k0 = 0; k0 < nrec; k0 += 16) merge_round(std::integral_constant<int, 16>{}, k0);
           }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          *reinterpret_cast<float4*>(outp + gg * D + d) = make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
         }
       }
     }
