@@ -226,6 +226,24 @@ def test_split_segments_odd_gqa(kvq, oracle, G):
         P.close()
 
 
+@pytest.mark.parametrize("pair,G", [((4, 4), 4), ((8, 8), 4), ((4, 4), 7), ((16, 16), 1)])
+def test_one_segment_over_the_whole_grid(kvq, oracle, pair, G):
+    # a single (sequence, KV head) long enough that every CTA of the persistent
+    # grid takes a slice of it: the last CTA merges hundreds of split records
+    # (rounds of 16 with online rescaling between rounds)
+    rng = np.random.default_rng(70 + G + pair[0])
+    T = 24000 + 17
+    P = Pair(kvq, oracle, pair, 1, G, 1, 128, T + 8)
+    try:
+        K, V = _inputs(rng, T, 1, 128)
+        P.append(K, V, [T])
+        kvq.kvq_set_decode_mode(P.cache, 0)  # shared split
+        got, ref = P.attend(_q(rng, 1, G, 128))
+        _check_attention(got, ref, f"{pair} G={G}")
+    finally:
+        P.close()
+
+
 def test_tiny_k8v4_workload(kvq, oracle):
     """The 1-layer K8V4 workload: batch 1, 2 = 2 heads, D 64, 256 tokens + 1."""
     w = synth.WORKLOADS["tiny_k8v4"]
