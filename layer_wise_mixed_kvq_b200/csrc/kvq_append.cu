@@ -143,12 +143,26 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
-__device__ __forceinline__ uint2 code_bits2(float2 x, float2 nz, float2 r, float qmax) {
-  float2 y = mul2_rn(add2_rn(x, nz), r);
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, C, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mov.b64 C, {%6, %7};\n\tfma.rn.f32x2 D, A, B, C;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+// m: the two sums 1.5 * 2^23 + code (as floats); u: x - z (rounded, as used for y)
+struct CodePair {
+  float2 m, u;
+};
+__device__ __forceinline__ CodePair code_pair(float2 x, float2 nz, float2 r, float qmax) {
+  CodePair cp;
+  cp.u = add2_rn(x, nz);
+  float2 y = mul2_rn(cp.u, r);
   y.x = fminf(fmaxf(y.x, 0.0f), qmax);
   y.y = fminf(fmaxf(y.y, 0.0f), qmax);
-  const float2 m = add2_rn(y, make_float2(12582912.0f, 12582912.0f));
-  return make_uint2(__float_as_uint(m.x), __float_as_uint(m.y));
+  cp.m = add2_rn(y, make_float2(12582912.0f, 12582912.0f));
+  return cp;
 }
 
 // Error report terms of one element: (x - x_hat)^2 and x^2 in fp64, with
@@ -162,11 +176,27 @@ __device__ __forceinline__ void add_error(double (&e)[2], float x, uint32_t bits
   e[1] = fma(xd, xd, e[1]);
 }
 
+// Error report terms in fp32 for a pair of elements, for groups whose
+// magnitudes lie in [2^-40, 2^40): dx = (x - z) - code * s with x - z the
+// rounded u of the code computation and one rounding of the fused
+// multiply-add, dx^2 and x^2 accumulated in fp32 over one 16-byte vector (at
+// most 32 elements per thread) and then added to the fp64 sums. Each term is
+// within a few fp32 roundings of the fp64 one (x^2 is exact in fp32 for a bf16
+// x in that range), so a layer's sums stay within ~1e-6 relative of the exact
+// ones; outside that range the fp64 terms above are used.
+__device__ __forceinline__ void add_error2(float2 (&acc)[2], float2 x, const CodePair& cp, float2 ns) {
+  const float2 c = add2_rn(cp.m, make_float2(-12582912.0f, -12582912.0f));  // the codes, exactly
+  const float2 dx = fma2_rn(c, ns, cp.u);
+  acc[0] = fma2_rn(dx, dx, acc[0]);
+  acc[1] = fma2_rn(x, x, acc[1]);
+}
+
 // Quantizer parameters of one index (a channel or a token): z and 1/s in fp32
-// for the code, z and s in fp64 for the error report.
+// for the code; -s in fp32 and z, s in fp64 for the error report.
 struct QTab {
   const float* nz;     // -z
   const float* r;      // 1/s, 0 for a constant set
+  const float* ns;     // -s
   const double2* zs;   // z, s
 };
 
@@ -175,8 +205,9 @@ struct QTab {
 // of tile f goes to nibble p + 4j of word f (4-bit), to bits 2(4u + p + 8j) of
 // word f/2 with u = f%2 (2-bit), or to byte 2(p&1) + j of word 2f + p/2 (8-bit).
 // MODE 0: keys, one parameter set per channel; 1: keys, one per token;
-// 2: values, one per token. e: this thread's error terms of the block.
-template <int BITS, int D, int RS, int MODE>
+// 2: values, one per token. e: this thread's error terms of the block, formed
+// in fp32 (F32ERR) or fp64.
+template <int BITS, int D, int RS, int MODE, bool F32ERR>
 __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*xs)[RS], QTab q, double (&e)[2]) {
   constexpr int TPV = 16 / BITS;  // tiles per 16-byte vector
   constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
@@ -185,7 +216,7 @@ __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*x
   // parameters of the element pair (p, 0), (p, 1) of a tile: index h = p>>1
   // (MODE 0, 2: indices i0 + 8h, +1) or h = p&1 (MODE 1: one token for both)
   struct Pair {
-    float2 nz, r;
+    float2 nz, r, ns;
     double2 zs0, zs1;
   };
   auto load_pair = [&](int i, bool one) {
@@ -193,24 +224,35 @@ __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*x
     if (one) {
       pr.nz = make_float2(q.nz[i], q.nz[i]);
       pr.r = make_float2(q.r[i], q.r[i]);
-      pr.zs0 = pr.zs1 = q.zs[i];
+      if constexpr (F32ERR) pr.ns = make_float2(q.ns[i], q.ns[i]);
+      else pr.zs0 = pr.zs1 = q.zs[i];
     } else {
       pr.nz = *reinterpret_cast<const float2*>(q.nz + i);
       pr.r = *reinterpret_cast<const float2*>(q.r + i);
-      pr.zs0 = q.zs[i];
-      pr.zs1 = q.zs[i + 1];
+      if constexpr (F32ERR) {
+        pr.ns = *reinterpret_cast<const float2*>(q.ns + i);
+      } else {
+        pr.zs0 = q.zs[i];
+        pr.zs1 = q.zs[i + 1];
+      }
     }
     return pr;
   };
   for (int v = threadIdx.x; v < kVectors; v += kThreads) {
     const int vi = v >> 5;
     uint32_t w[4] = {0u, 0u, 0u, 0u};
+    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // F32ERR: dx^2, x^2 of this vector
     // one element pair: quantize, add the error terms, add the codes into their fields
     auto put = [&](int i, int p, uint32_t a, const Pair& pr) {
       const float2 x = make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
-      const uint2 bits = code_bits2(x, pr.nz, pr.r, qmax);
-      add_error(e, x.x, bits.x, pr.zs0);
-      add_error(e, x.y, bits.y, pr.zs1);
+      const CodePair cp = code_pair(x, pr.nz, pr.r, qmax);
+      const uint2 bits = make_uint2(__float_as_uint(cp.m.x), __float_as_uint(cp.m.y));
+      if constexpr (F32ERR) {
+        add_error2(acc, x, cp, pr.ns);
+      } else {
+        add_error(e, x.x, bits.x, pr.zs0);
+        add_error(e, x.y, bits.y, pr.zs1);
+      }
       // (bits - bias) << shift is the code in place; words only gain disjoint fields
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -252,6 +294,10 @@ __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*x
       }
     }
     reinterpret_cast<uint4*>(blk)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+    if constexpr (F32ERR) {
+      e[0] += (double)acc[0].x + (double)acc[0].y;
+      e[1] += (double)acc[1].x + (double)acc[1].y;
+    }
   }
 }
 
@@ -279,6 +325,8 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
   __shared__ __align__(16) __nv_bfloat16 xsb[2][2][kPageTokens][RS];  // two groups' key and value rows
   __shared__ __align__(16) float qnz[2][NP];    // quantizer -z by index: keys, values
   __shared__ __align__(16) float qr[2][NP];     // 1/s (0 for a constant set)
+  __shared__ __align__(16) float qns[2][NP];    // -s
+  __shared__ unsigned s_amax;                   // largest |min| or |max| of the group's sets (float bits)
   __shared__ __align__(16) double2 qzs[2][NP];  // z, s in fp64 (error report)
   constexpr int KP = D / 2, KS = kThreads / KP;  // key channel pairs, token splits of the key pass
   __shared__ __nv_bfloat162 kpart[KS][2][KP];   // per-split min, max of each key channel pair
@@ -369,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
       const int g = g0 + it;
       uint8_t* page = a.pages + ((int64_t)(b * H + h) * a.max_pages + g) * a.page_bytes;
       auto& xs = xsb[buf];
+      if (threadIdx.x == 0) s_amax = 0u;
       __syncthreads();
       if constexpr (kBf16Layer) {
         emit_bf16<D, RS>(page, xs[0], false);
@@ -399,8 +448,10 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
           __half* kzero = kscale + nk;
           __half* vscale = kzero + nk;
           __half* vzero = vscale + kPageTokens;
-          auto keep = [&](int r, int i, const QParams& q) {
+          auto keep = [&](int r, int i, const QParams& q, float mn, float mx) {
+            atomicMax(&s_amax, __float_as_uint(fmaxf(fabsf(mn), fabsf(mx))));  // bits order = value order
             qnz[r][i] = -q.z;
+            qns[r][i] = -__half2float(q.s_h);
             qr[r][i] = q.r;  // 0 for a constant set
             qzs[r][i] = make_double2((double)q.z, (double)__half2float(q.s_h));
           };
@@ -425,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
               const QParams q = make_qparams(fmn, fmx, qmax);
               sdst[tok] = q.s_h;
               zdst[tok] = q.z_h;
-              keep(r, tok, q);
+              keep(r, tok, q, fmn, fmx);
             }
           };
           token_params(1, (1 << VB) - 1, vscale, vzero);
@@ -459,16 +510,23 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
               const int slot = kmeta_slot<D>(d);
               kscale[slot] = q.s_h;
               kzero[slot] = q.z_h;
-              keep(0, d, q);
+              keep(0, d, q, fmn, fmx);
             }
           }
           __syncthreads();
           // codes, each element quantized as it is packed, and its error report terms
           double ek[2] = {0.0, 0.0}, ev[2] = {0.0, 0.0};
-          const QTab tk{qnz[0], qr[0], qzs[0]}, tv{qnz[1], qr[1], qzs[1]};
-          if (per_token_keys) emit_codes<KB, D, RS, 1>(page, xs[0], tk, ek);
-          else emit_codes<KB, D, RS, 0>(page, xs[0], tk, ek);
-          emit_codes<VB, D, RS, 2>(vblk, xs[1], tv, ev);
+          const QTab tk{qnz[0], qr[0], qns[0], qzs[0]}, tv{qnz[1], qr[1], qns[1], qzs[1]};
+          const float amax = __uint_as_float(s_amax);
+          if (amax >= 0x1p-40f && amax < 0x1p40f) {
+            if (per_token_keys) emit_codes<KB, D, RS, 1, true>(page, xs[0], tk, ek);
+            else emit_codes<KB, D, RS, 0, true>(page, xs[0], tk, ek);
+            emit_codes<VB, D, RS, 2, true>(vblk, xs[1], tv, ev);
+          } else {
+            if (per_token_keys) emit_codes<KB, D, RS, 1, false>(page, xs[0], tk, ek);
+            else emit_codes<KB, D, RS, 0, false>(page, xs[0], tk, ek);
+            emit_codes<VB, D, RS, 2, false>(vblk, xs[1], tv, ev);
+          }
           err[0] += ek[0];
           err[1] += ek[1];
           err[2] += ev[0];

@@ -1,6 +1,7 @@
 """GPU parity of the per-layer quantization error report (kvq_layer_error)
-with the oracle's: same element counts, sums within fp64 summation-order
-rounding."""
+with the oracle's: same element counts, sums within the rounding of the GPU's
+per-element terms (fp32 in the append kernel for groups of moderate magnitude,
+fp64 otherwise and in the fused step's flush) and of the summation order."""
 
 import numpy as np
 import pytest
@@ -12,8 +13,11 @@ pytestmark = pytest.mark.gpu
 
 
 def _same_report(got, want):
+    # the append kernel forms each element's terms in fp32 (a few roundings,
+    # summed in fp32 over at most 32 elements, then in fp64): ~1e-6 relative
+    # at most on the layer sums, held here to 1e-5
     assert got[4] == want[4]
-    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-9, atol=0)
+    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-5, atol=0)
 
 
 @pytest.mark.parametrize("pair", [(2, 2), (4, 8), (8, 4), (4, 4, 1), (2, 8, 1), (8, 8, 0, 1), (16, 16)])
