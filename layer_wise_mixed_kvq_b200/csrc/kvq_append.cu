@@ -122,10 +122,10 @@ __device__ __forceinline__ void load_tile(uint32_t (&a)[4], const __nv_bfloat16 
 
 // Two elements' codes, as the bits of the fp32 numbers 1.5 * 2^23 + code: for y
 // in [0, qmax] the single rounding of the addition is rint(y), round-half-even.
-// y = (x - z) * (1/s), x - z formed as x + (-z) (the same IEEE result), clamped
-// to [0, qmax] first, which gives clamp(rint(y), 0, qmax) for every y (fmaxf
-// also maps a NaN to 0); a zero reciprocal (constant set) gives 0. Two elements
-// per packed fp32 operation, each with an explicit rounding mode.
+// y = (x - z) * (1/s), x - z formed as x + (-z) (the same IEEE result); with
+// CLAMP, y is clamped to [0, qmax] first, which gives clamp(rint(y), 0, qmax) for
+// every y (fmaxf also maps a NaN to 0); a zero reciprocal (constant set) gives
+// 0. Two elements per packed fp32 operation, each with an explicit rounding mode.
 constexpr uint32_t kRintBias = 0x4B400000u;  // bits of 1.5 * 2^23
 __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
   float2 d;
@@ -155,13 +155,25 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
 struct CodePair {
   float2 m, u;
 };
+// Without CLAMP (a group none of whose sets had z or s clamped to fp16's
+// range) y already lies in [0, qmax + 2^-14] for every element of its set (z <=
+// min, s >= (max - z) / qmax rounded up), so rint(y) is in [0, qmax] without the
+// clamp. There the bias is added by two scalar additions: a packed addition
+// that directly consumes the packed product measured as a single rounding of
+// both on B200 (codes off by one in ~0.04% of elements), while __fadd_rn stays
+// its own operation.
+template <bool CLAMP>
 __device__ __forceinline__ CodePair code_pair(float2 x, float2 nz, float2 r, float qmax) {
   CodePair cp;
   cp.u = add2_rn(x, nz);
   float2 y = mul2_rn(cp.u, r);
-  y.x = fminf(fmaxf(y.x, 0.0f), qmax);
-  y.y = fminf(fmaxf(y.y, 0.0f), qmax);
-  cp.m = add2_rn(y, make_float2(12582912.0f, 12582912.0f));
+  if constexpr (CLAMP) {
+    y.x = fminf(fmaxf(y.x, 0.0f), qmax);
+    y.y = fminf(fmaxf(y.y, 0.0f), qmax);
+    cp.m = add2_rn(y, make_float2(12582912.0f, 12582912.0f));
+  } else {
+    cp.m = make_float2(__fadd_rn(y.x, 12582912.0f), __fadd_rn(y.y, 12582912.0f));
+  }
   return cp;
 }
 
@@ -206,8 +218,8 @@ struct QTab {
 // word f/2 with u = f%2 (2-bit), or to byte 2(p&1) + j of word 2f + p/2 (8-bit).
 // MODE 0: keys, one parameter set per channel; 1: keys, one per token;
 // 2: values, one per token. e: this thread's error terms of the block, formed
-// in fp32 (F32ERR) or fp64.
-template <int BITS, int D, int RS, int MODE, bool F32ERR>
+// in fp32 (F32ERR) or fp64. CLAMP: see code_pair.
+template <int BITS, int D, int RS, int MODE, bool F32ERR, bool CLAMP>
 __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*xs)[RS], QTab q, double (&e)[2]) {
   constexpr int TPV = 16 / BITS;  // tiles per 16-byte vector
   constexpr int kVectors = (int)(code_block_bytes(BITS, D) / 16);
@@ -245,7 +257,7 @@ __device__ __forceinline__ void emit_codes(uint8_t* blk, const __nv_bfloat16 (*x
     // one element pair: quantize, add the error terms, add the codes into their fields
     auto put = [&](int i, int p, uint32_t a, const Pair& pr) {
       const float2 x = make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
-      const CodePair cp = code_pair(x, pr.nz, pr.r, qmax);
+      const CodePair cp = code_pair<CLAMP>(x, pr.nz, pr.r, qmax);
       const uint2 bits = make_uint2(__float_as_uint(cp.m.x), __float_as_uint(cp.m.y));
       if constexpr (F32ERR) {
         add_error2(acc, x, cp, pr.ns);
@@ -327,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
   __shared__ __align__(16) float qr[2][NP];     // 1/s (0 for a constant set)
   __shared__ __align__(16) float qns[2][NP];    // -s
   __shared__ unsigned s_amax;                   // largest |min| or |max| of the group's sets (float bits)
+  __shared__ int s_clamp;                       // a set of the group had z or s clamped to fp16's range
   __shared__ __align__(16) double2 qzs[2][NP];  // z, s in fp64 (error report)
   constexpr int KP = D / 2, KS = kThreads / KP;  // key channel pairs, token splits of the key pass
   __shared__ __nv_bfloat162 kpart[KS][2][KP];   // per-split min, max of each key channel pair
@@ -417,7 +430,10 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
       const int g = g0 + it;
       uint8_t* page = a.pages + ((int64_t)(b * H + h) * a.max_pages + g) * a.page_bytes;
       auto& xs = xsb[buf];
-      if (threadIdx.x == 0) s_amax = 0u;
+      if (threadIdx.x == 0) {
+        s_amax = 0u;
+        s_clamp = 0;
+      }
       __syncthreads();
       if constexpr (kBf16Layer) {
         emit_bf16<D, RS>(page, xs[0], false);
@@ -450,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
           __half* vzero = vscale + kPageTokens;
           auto keep = [&](int r, int i, const QParams& q, float mn, float mx) {
             atomicMax(&s_amax, __float_as_uint(fmaxf(fabsf(mn), fabsf(mx))));  // bits order = value order
+            if (q.z > mn || __half2float(q.s_h) >= 65504.0f) atomicOr(&s_clamp, 1);
             qnz[r][i] = -q.z;
             qns[r][i] = -__half2float(q.s_h);
             qr[r][i] = q.r;  // 0 for a constant set
@@ -518,14 +535,18 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
           double ek[2] = {0.0, 0.0}, ev[2] = {0.0, 0.0};
           const QTab tk{qnz[0], qr[0], qns[0], qzs[0]}, tv{qnz[1], qr[1], qns[1], qzs[1]};
           const float amax = __uint_as_float(s_amax);
-          if (amax >= 0x1p-40f && amax < 0x1p40f) {
-            if (per_token_keys) emit_codes<KB, D, RS, 1, true>(page, xs[0], tk, ek);
-            else emit_codes<KB, D, RS, 0, true>(page, xs[0], tk, ek);
-            emit_codes<VB, D, RS, 2, true>(vblk, xs[1], tv, ev);
+          if (amax >= 0x1p-40f && amax < 0x1p40f && !s_clamp) {
+            if (per_token_keys) emit_codes<KB, D, RS, 1, true, false>(page, xs[0], tk, ek);
+            else emit_codes<KB, D, RS, 0, true, false>(page, xs[0], tk, ek);
+            emit_codes<VB, D, RS, 2, true, false>(vblk, xs[1], tv, ev);
+          } else if (amax >= 0x1p-40f && amax < 0x1p40f) {
+            if (per_token_keys) emit_codes<KB, D, RS, 1, true, true>(page, xs[0], tk, ek);
+            else emit_codes<KB, D, RS, 0, true, true>(page, xs[0], tk, ek);
+            emit_codes<VB, D, RS, 2, true, true>(vblk, xs[1], tv, ev);
           } else {
-            if (per_token_keys) emit_codes<KB, D, RS, 1, false>(page, xs[0], tk, ek);
-            else emit_codes<KB, D, RS, 0, false>(page, xs[0], tk, ek);
-            emit_codes<VB, D, RS, 2, false>(vblk, xs[1], tv, ev);
+            if (per_token_keys) emit_codes<KB, D, RS, 1, false, true>(page, xs[0], tk, ek);
+            else emit_codes<KB, D, RS, 0, false, true>(page, xs[0], tk, ek);
+            emit_codes<VB, D, RS, 2, false, true>(vblk, xs[1], tv, ev);
           }
           err[0] += ek[0];
           err[1] += ek[1];

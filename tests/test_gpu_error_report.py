@@ -45,3 +45,22 @@ def test_error_report_matches_oracle(kvq, oracle, pair, D):
         assert kvq.kvq_layer_error(P.cache, 0) == (0.0, 0.0, 0.0, 0.0, 0)
     finally:
         P.close()
+
+
+@pytest.mark.parametrize("scale", [1e13, 1e-13, 3e4])
+@pytest.mark.parametrize("pair", [(4, 4), (8, 2), (2, 8, 1)])
+def test_error_report_at_extreme_magnitudes(kvq, oracle, pair, scale):
+    # groups with magnitudes outside [2^-40, 2^40) take the fp64 terms; 3e4
+    # (beyond fp16's range after the zero point) takes the clamping path
+    rng = np.random.default_rng(hash((pair, scale, "err-x")) % 2**32)
+    batch, hkv, D = 2, 2, 64
+    P = Pair(kvq, oracle, pair, batch, hkv * 4, hkv, D, 200)
+    try:
+        K, V = _inputs(rng, 160, hkv, D)
+        K = torch.from_numpy(K * scale).to(torch.bfloat16).float().numpy()
+        V = torch.from_numpy(V * scale).to(torch.bfloat16).float().numpy()
+        P.append(K, V, [96, 64])
+        P.check_pages()
+        _same_report(kvq.kvq_layer_error(P.cache, 0), P.ref.error())
+    finally:
+        P.close()
