@@ -188,14 +188,16 @@ __device__ __forceinline__ void add_error(double (&e)[2], float x, uint32_t bits
   e[1] = fma(xd, xd, e[1]);
 }
 
-// Error report terms in fp32 for a pair of elements, for groups whose
-// magnitudes lie in [2^-40, 2^40): dx = (x - z) - code * s with x - z the
-// rounded u of the code computation and one rounding of the fused
-// multiply-add, dx^2 and x^2 accumulated in fp32 over one 16-byte vector (at
-// most 32 elements per thread) and then added to the fp64 sums. Each term is
-// within a few fp32 roundings of the fp64 one (x^2 is exact in fp32 for a bf16
-// x in that range), so a layer's sums stay within ~1e-6 relative of the exact
-// ones; outside that range the fp64 terms above are used.
+// Error report terms in fp32 for a pair of elements, for groups whose largest
+// magnitude lies in [2^-14, 2^40) (fp16's normal range and above, so z and s
+// resolve the data): dx = (x - z) - code * s with x - z the rounded u of the
+// code computation and one rounding of the fused multiply-add, dx^2 and x^2
+// accumulated in fp32 over one 16-byte vector (at most 32 elements per thread)
+// and then added to the fp64 sums. x^2 is exact in fp32 for a bf16 x there; the
+// rounding of u (|u| <= (qmax + 1) s) moves a dx by at most 2^-24 |u|, so a
+// layer's sum of dx^2 stays within about 2^-23 (qmax + 1) * 3 (below 1e-4 for
+// 8-bit codes, far less in practice) of the exact one. Outside that range the
+// fp64 terms above are used.
 __device__ __forceinline__ void add_error2(float2 (&acc)[2], float2 x, const CodePair& cp, float2 ns) {
   const float2 c = add2_rn(cp.m, make_float2(-12582912.0f, -12582912.0f));  // the codes, exactly
   const float2 dx = fma2_rn(c, ns, cp.u);
@@ -535,11 +537,11 @@ __global__ void __launch_bounds__(kThreads, 4) append_kernel(AppendParams a) {
           double ek[2] = {0.0, 0.0}, ev[2] = {0.0, 0.0};
           const QTab tk{qnz[0], qr[0], qns[0], qzs[0]}, tv{qnz[1], qr[1], qns[1], qzs[1]};
           const float amax = __uint_as_float(s_amax);
-          if (amax >= 0x1p-40f && amax < 0x1p40f && !s_clamp) {
+          if (amax >= 0x1p-14f && amax < 0x1p40f && !s_clamp) {
             if (per_token_keys) emit_codes<KB, D, RS, 1, true, false>(page, xs[0], tk, ek);
             else emit_codes<KB, D, RS, 0, true, false>(page, xs[0], tk, ek);
             emit_codes<VB, D, RS, 2, true, false>(vblk, xs[1], tv, ev);
-          } else if (amax >= 0x1p-40f && amax < 0x1p40f) {
+          } else if (amax >= 0x1p-14f && amax < 0x1p40f) {
             if (per_token_keys) emit_codes<KB, D, RS, 1, true, true>(page, xs[0], tk, ek);
             else emit_codes<KB, D, RS, 0, true, true>(page, xs[0], tk, ek);
             emit_codes<VB, D, RS, 2, true, true>(vblk, xs[1], tv, ev);

@@ -34,11 +34,12 @@ def _step(P, kvq, rng, batch, hkv, D, G, seqs=None):
 
 
 def _same_report(got, want):
-    # the append kernel forms each element's terms in fp32 (a few roundings,
-    # summed in fp32 over at most 32 elements, then in fp64): ~1e-6 relative
-    # at most on the layer sums, held here to 1e-5
+    # the append kernel forms each element's terms in fp32 for groups of
+    # moderate magnitude: a dx moves by at most 2^-24 |x - z| with |x - z| <=
+    # (qmax + 1) s, i.e. at most about 2^-23 * 256 * 3 < 1e-4 relative on the
+    # sum of dx^2 for 8-bit codes (fp32 summation over <= 32 terms adds ~2e-6)
     assert got[4] == want[4]
-    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-5, atol=0)
+    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-4, atol=0)
 
 
 @pytest.mark.parametrize("pair", [(2, 2), (2, 4), (4, 2), (4, 4), (4, 8), (8, 2), (8, 8), (16, 16),

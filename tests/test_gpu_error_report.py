@@ -13,11 +13,12 @@ pytestmark = pytest.mark.gpu
 
 
 def _same_report(got, want):
-    # the append kernel forms each element's terms in fp32 (a few roundings,
-    # summed in fp32 over at most 32 elements, then in fp64): ~1e-6 relative
-    # at most on the layer sums, held here to 1e-5
+    # the append kernel forms each element's terms in fp32 for groups of
+    # moderate magnitude: a dx moves by at most 2^-24 |x - z| with |x - z| <=
+    # (qmax + 1) s, i.e. at most about 2^-23 * 256 * 3 < 1e-4 relative on the
+    # sum of dx^2 for 8-bit codes (fp32 summation over <= 32 terms adds ~2e-6)
     assert got[4] == want[4]
-    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-5, atol=0)
+    np.testing.assert_allclose(got[:4], want[:4], rtol=1e-4, atol=0)
 
 
 @pytest.mark.parametrize("pair", [(2, 2), (4, 8), (8, 4), (4, 4, 1), (2, 8, 1), (8, 8, 0, 1), (16, 16)])
@@ -50,8 +51,9 @@ def test_error_report_matches_oracle(kvq, oracle, pair, D):
 @pytest.mark.parametrize("scale", [1e13, 1e-13, 3e4])
 @pytest.mark.parametrize("pair", [(4, 4), (8, 2), (2, 8, 1)])
 def test_error_report_at_extreme_magnitudes(kvq, oracle, pair, scale):
-    # groups with magnitudes outside [2^-40, 2^40) take the fp64 terms; 3e4
-    # (beyond fp16's range after the zero point) takes the clamping path
+    # groups with magnitudes outside [2^-14, 2^40) take the fp64 terms (1e-13:
+    # below fp16's resolution, where z and s are coarse next to the data); 3e4
+    # (beyond fp16's range) takes the clamping path
     rng = np.random.default_rng(hash((pair, scale, "err-x")) % 2**32)
     batch, hkv, D = 2, 2, 64
     P = Pair(kvq, oracle, pair, batch, hkv * 4, hkv, D, 200)
