@@ -475,8 +475,14 @@ __device__ __forceinline__ void tile_frags_f8(const uint32_t (&w)[TileWords<8>::
 template <int D>
 __device__ __forceinline__ void softmax_update(WarpState<D>& st, float (&sc)[8]) {
   float mx = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])), fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  // the row maximum is needed only when some score passes the reference by more
+  // than kTau: one vote decides (a row's lanes share st.m, so the result is the
+  // same as reducing every time)
+  if (!__any_sync(0xffffffffu, mx > st.m + kTau)) mx = st.m;
+  else {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  }
   if (mx > st.m + kTau) {
     const float alpha = ex2(st.m - mx);  // 0 when st.m = -inf
 #pragma unroll
@@ -501,9 +507,14 @@ __device__ __forceinline__ void softmax_update(WarpState<D>& st, float (&sc)[8])
 template <int D>
 __device__ __forceinline__ void tok_softmax_update(TokState<D>& st, float (&sc)[4]) {
   float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+  // the head's maximum over the page is needed only when some score passes the
+  // reference by more than kTau: one vote decides (a head's lanes share st.m)
+  if (!__any_sync(0xffffffffu, mx > st.m + kTau)) mx = st.m;
+  else {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+  }
   if (mx > st.m + kTau) {
     const float alpha = ex2(st.m - mx);
 #pragma unroll
