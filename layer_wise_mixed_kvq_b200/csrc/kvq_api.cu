@@ -539,6 +539,7 @@ static kvq_status decode_params(kvq_cache* c, int layer, const void* Q, int batc
   p.fmt = L.fmt;
   p.fp8_scales = L.fp8_scales;
   p.warp_split = choose_warp_split(c, p.gqa, batch, max_p + (append ? 1 : 0), total_pages) ? 1 : 0;
+  p.warp_pairs = max_p >= 4 ? 1 : 0;  // halving a warp's pages pays from a few pages on
   // The lengths travel in the parameters unless a captured graph may replay this
   // launch (frozen parameters) or replays have moved the device lengths past the
   // host's view. Then the page copies may start under the preceding kernel's

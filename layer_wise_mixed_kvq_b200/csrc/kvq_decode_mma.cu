@@ -78,6 +78,10 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
@@ -1970,6 +1974,13 @@ struct WarpCfg {
   static constexpr int QBUF_OFF = WSCR_OFF + kWarps * C::WSCR_STRIDE;
   static constexpr int QSLOT = 4 * D * 2;                                            // [4][D] bf16 per warp
   static constexpr int SMEM = QBUF_OFF + kWarps * QSLOT;
+  // warp pairs: per pair three barriers (length handed over, state dumped, dump read),
+  // the handed-over length, and the second warp's state [32 lanes][D/4 + 3] floats
+  static constexpr int DUMP_FLOATS = D / 4 + 3;
+  static constexpr int PBAR_OFF = SMEM;
+  static constexpr int T0_OFF = PBAR_OFF + (kWarps / 2) * 3 * 8;
+  static constexpr int DUMP_OFF = (T0_OFF + (kWarps / 2) * 4 + 15) / 16 * 16;
+  static constexpr int SMEM_PAIR = DUMP_OFF + (kWarps / 2) * 32 * DUMP_FLOATS * 4;
 };
 
 // AP (kvq_decode_step): before attending segment (b, h) the warp appends its new
@@ -1977,7 +1988,12 @@ struct WarpCfg {
 // next page, which the warp then attends from global memory -- and the last of
 // sequence b's H warps to have read the old length publishes the new one (the
 // acquire-release increment orders every read before that write).
-template <int KB, int VB, int D, bool PT, bool F8, bool AP = false>
+//
+// PAIR: warps 2i and 2i + 1 share a segment -- the first takes its even pages,
+// the tail and the window, the second its odd pages -- and the first merges the
+// second's state from shared memory before the window and the output. The pair
+// syncs on three mbarriers, every wait bounded like the ring's.
+template <int KB, int VB, int D, bool PT, bool F8, bool AP = false, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
     decode_warp_kernel(const __grid_constant__ DecodeParams p) {
   pdl_enter();
@@ -1993,25 +2009,42 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
   uint64_t* qbar = bars + C::R;
   float* wscr = reinterpret_cast<float*>(smem + WC::WSCR_OFF + warp * C::WSCR_STRIDE);
   __nv_bfloat16* qslot = reinterpret_cast<__nv_bfloat16*>(smem + WC::QBUF_OFF + warp * WC::QSLOT);
+  constexpr int SPW = PAIR ? 2 : 1;  // warps per segment
+  const int half = PAIR ? (warp & 1) : 0;
+  uint64_t* pbar = reinterpret_cast<uint64_t*>(smem + WC::PBAR_OFF) + (warp >> 1) * 3;
+  int* t0slot = reinterpret_cast<int*>(smem + WC::T0_OFF) + (warp >> 1);
+  float* dump = reinterpret_cast<float*>(smem + WC::DUMP_OFF) + (warp >> 1) * 32 * WC::DUMP_FLOATS +
+                lane * WC::DUMP_FLOATS;
   if (lane == 0) {
     for (int r = 0; r <= C::R; ++r) mbar_init(&bars[r], 1);
+    if (PAIR && half == 0)
+      for (int r = 0; r < 3; ++r) mbar_init(&pbar[r], 1);
     mbar_init_fence();
   }
-  __syncwarp();
+  if constexpr (PAIR) __syncthreads();  // the pair barriers exist before either warp uses them
+  else __syncwarp();
 
   const int S = p.batch * H;
-  const int stride = (int)gridDim.x * kWarps;
+  const int stride = (int)gridDim.x * kWarps / SPW;
   const uint32_t qbytes = (uint32_t)(G * D * 2);
   const uint64_t pol = l2_evict_first_policy();
   bool ok = true;
   int issued = 0, consumed = 0, nq = 0;
-  for (int s = blockIdx.x * kWarps + warp; s < S && ok; s += stride, ++nq) {
+  for (int s = (blockIdx.x * kWarps + warp) / SPW; s < S && ok; s += stride, ++nq) {
     const int b = s / H, h = s % H;
-    int T, P;              // tokens attended; pages read through the ring
+    int T, P;              // tokens attended; pages of the segment (before the new token)
     bool flushed = false;  // AP: page P, just written, is attended too
     if constexpr (AP) {
       int t0 = 0;
-      if (lane == 0) {
+      if (PAIR && half == 1) {
+        // the first warp of the pair read the length and appended the token
+        const bool got = mbar_wait(&pbar[0], (uint32_t)(nq & 1));
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        t0 = *t0slot;
+      } else if (lane == 0) {
         t0 = p.step_len[b];
         if (atomic_add_acq_rel(&p.append_ctr[b], 1) == H - 1) {
           p.append_ctr[b] = 0;
@@ -2019,32 +2052,39 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
         }
       }
       t0 = __shfl_sync(0xffffffffu, t0, 0);
+      if (PAIR && half == 0 && lane == 0) {
+        *t0slot = t0;
+        mbar_arrive(&pbar[0]);
+      }
       P = t0 / kPageTokens;
       if (t0 < p.max_tokens) {
         T = t0 + 1;
-        flushed = append_token<KB, VB, D, PT, F8>(p, s, h, t0, wscr, lane);
+        if (half == 0) flushed = append_token<KB, VB, D, PT, F8>(p, s, h, t0, wscr, lane);
       } else {
         T = t0;  // a full sequence is left unchanged and the cache's error flag raised
-        if (lane == 0 && p.err) atomicExch(p.err, 2);
+        if (half == 0 && lane == 0 && p.err) atomicExch(p.err, 2);
       }
     } else {
       T = p.len[b];
       P = T / kPageTokens;
     }
     const int W = T % kPageTokens;
-    const uint8_t* base = p.pages + ((int64_t)s * p.max_pages) * p.page_bytes;
+    // this warp's pages: half, half + SPW, ... (all of them without pairs)
+    const int Pn = P > half ? (P - half + SPW - 1) / SPW : 0;
+    const uint8_t* base = p.pages + ((int64_t)s * p.max_pages + half) * p.page_bytes;
+    const int64_t pstride = (int64_t)SPW * p.page_bytes;
     const __nv_bfloat16* win = p.window + ((int64_t)s * 2) * kPageTokens * D;
-    int next = 0;  // next page of this segment to copy
+    int next = 0;  // next of this warp's pages to copy
     if (lane == 0) {
       fence_proxy_async();  // the slot's previous rows were read through the generic proxy
       mbar_expect_tx(qbar, qbytes);
       bulk_load(qslot, p.Q + (int64_t)s * G * D, qbytes, qbar);
-      for (; next < P && next < C::R; ++next) {
+      for (; next < Pn && next < C::R; ++next) {
         const int stage = (issued + next) % C::R;
         mbar_expect_tx(&bars[stage], C::PB);
-        bulk_load_once(ring + stage * C::STAGE, base + (int64_t)next * p.page_bytes, C::PB, &bars[stage], pol);
+        bulk_load_once(ring + stage * C::STAGE, base + (int64_t)next * pstride, C::PB, &bars[stage], pol);
       }
-      if (W > 0) {
+      if (W > 0 && half == 0) {
         prefetch_l2(win, (uint32_t)(W * D * 2));
         prefetch_l2(win + kPageTokens * D, (uint32_t)(W * D * 2));
       }
@@ -2074,7 +2114,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
       else if constexpr (PT) attend_qpage_tok_pt<KB, VB, D>(page, st, tops, wscr, lane);
       else attend_qpage_tok<KB, VB, D>(page, st, tops, wscr, lane);
     };
-    for (int k = 0; k < P; ++k) {
+    for (int k = 0; k < Pn; ++k) {
       const int stage = consumed % C::R;
       const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / C::R) & 1));
       if (!__all_sync(0xffffffffu, arrived)) {
@@ -2084,11 +2124,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
       attend_page(ring + stage * C::STAGE);
       ++consumed;
       __syncwarp();
-      if (next < P) {
+      if (next < Pn) {
         if (lane == 0) {
           fence_proxy_async();
           mbar_expect_tx(&bars[stage], C::PB);
-          bulk_load_once(ring + stage * C::STAGE, base + (int64_t)next * p.page_bytes, C::PB, &bars[stage], pol);
+          bulk_load_once(ring + stage * C::STAGE, base + (int64_t)next * pstride, C::PB, &bars[stage], pol);
         }
         ++next;
         ++issued;
@@ -2096,8 +2136,49 @@ __global__ void __launch_bounds__(kThreads, Cfg<KB, VB, D, PT, F8>::MINB_TOK)
     }
     if (!ok) break;
     // the page this warp has just written (generic loads: it never went through the async proxy)
-    if (flushed) attend_page(base + (int64_t)P * p.page_bytes);
+    if (flushed) attend_page(p.pages + ((int64_t)s * p.max_pages + P) * p.page_bytes);
     to_true_units<VB, true, F8>(st, F8 ? p.fp8_scales[H + h] : 1.f);
+    if constexpr (PAIR) {
+      constexpr int NT = D / 16;
+      if (half == 1) {
+        // hand this warp's state over once the first warp has read the previous one
+        bool got = nq == 0 || mbar_wait(&pbar[2], (uint32_t)((nq - 1) & 1));
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dump[4 * j + k] = st.o[j][k];
+        dump[4 * NT] = st.m;
+        dump[4 * NT + 1] = st.l;
+        dump[4 * NT + 2] = st.vz;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pbar[1]);
+        __syncwarp();  // every lane has read the query slot before the next segment's copy lands
+        continue;
+      }
+      // merge the second warp's state (same lane layout; heads share st.m per lane)
+      const bool got = mbar_wait(&pbar[1], (uint32_t)(nq & 1));
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      const float m1 = dump[4 * NT];
+      const float M = fmaxf(st.m, m1);
+      const float f0 = (st.m == -INFINITY) ? 0.f : ex2(st.m - M);
+      const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st.o[j][k] = st.o[j][k] * f0 + dump[4 * j + k] * f1;
+      st.l = st.l * f0 + dump[4 * NT + 1] * f1;
+      st.vz = st.vz * f0 + dump[4 * NT + 2] * f1;
+      st.m = M;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pbar[2]);
+    }
     if (W > 0) {
       if constexpr (!C::kBf16) load_qbp();
       attend_window_tok<D>(win, W, st, qb, p.scale_log2, lane);
@@ -2138,19 +2219,33 @@ template <int KB, int VB, int D, bool PT, bool F8, bool AP>
 cudaError_t launch_warp(const DecodeParams& p, cudaStream_t s) {
   using WC = WarpCfg<KB, VB, D, PT, F8>;
   static bool configured = false;
-  static int occ = 0;
+  static int occ = 0, occ_pair = 0;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8, AP>,
+    cudaError_t e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8, AP, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_warp_kernel<KB, VB, D, PT, F8, AP>, kThreads,
-                                                      WC::SMEM);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_warp_kernel<KB, VB, D, PT, F8, AP, false>,
+                                                      kThreads, WC::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_warp_kernel<KB, VB, D, PT, F8, AP, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, WC::SMEM_PAIR);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_pair, decode_warp_kernel<KB, VB, D, PT, F8, AP, true>,
+                                                      kThreads, WC::SMEM_PAIR);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int64_t ctas = ((int64_t)p.batch * p.n_kv_heads + kWarps - 1) / kWarps;
+  const int64_t segs = (int64_t)p.batch * p.n_kv_heads;
+  if (p.warp_pairs) {
+    // two warps per segment when the pairs fit one resident wave too
+    const int64_t ctas = (2 * segs + kWarps - 1) / kWarps;
+    if (ctas >= 1 && ctas <= (int64_t)occ_pair * p.sm_count)
+      return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8, AP, true>, dim3((unsigned)ctas), dim3(kThreads),
+                        (size_t)WC::SMEM_PAIR, s, p);
+  }
+  const int64_t ctas = (segs + kWarps - 1) / kWarps;
   if (ctas < 1 || ctas > (int64_t)occ * p.sm_count) return cudaErrorNotSupported;
-  return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8, AP>, dim3((unsigned)ctas), dim3(kThreads),
+  return launch_pdl(decode_warp_kernel<KB, VB, D, PT, F8, AP, false>, dim3((unsigned)ctas), dim3(kThreads),
                     (size_t)WC::SMEM, s, p);
 }
 

@@ -110,6 +110,8 @@ struct DecodeParams {
   int* err;              // set to nonzero if a bounded wait gave up (may be null)
   int warp_split;        // tensor-core kernel, G <= 4: one warp per segment (if the segments fit the
                          // resident warps) instead of CTAs sharing each segment's pages
+  int warp_pairs;        // warp split: two warps per segment (alternate pages, merged in shared
+                         // memory) when the pairs also fit the resident warps
   // fused decode step (kvq_decode_step): the warp that owns segment (b, h)'s tail
   // unit first appends that segment's new token; the same buffers as above, writable
   int append;
