@@ -474,16 +474,20 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* K, const void* V, kvq
   return KVQ_OK;
 }
 
-// One warp per (sequence, KV head) segment, or CTAs sharing each segment's pages.
-// Automatic: the split a cost model predicts faster, fitted to both kernels' times
-// on B200 (K4V2..K8V8 pages, batch 16 and 64, 5 to 128 pages per sequence): the
-// warp split takes about 5 + 1.0 us per page of the longest sequence, the shared
-// split about 11.5 + 0.01 us per segment + 0.15 us per page per SM.
+// One warp (or warp pair) per (sequence, KV head) segment, or CTAs sharing each
+// segment's pages. Automatic: the split a cost model predicts faster, fitted to
+// both kernels' times on B200 (K4V2..K8V8 pages, batch 8 to 128, 5 to 128 pages
+// per sequence): the warp split takes about 5 + 1.0 us per page a warp reads of
+// the longest sequence (half its pages with warp pairs), the shared split about
+// 11.5 + 0.01 us per segment + 0.15 us per page per SM.
 static bool choose_warp_split(const kvq_cache* c, int gqa, int batch, int64_t max_p, int64_t total_pages) {
   if (gqa > 4 || c->warp_pages == 0) return false;
   if (c->warp_pages > 0) return max_p <= c->warp_pages;
   const double segs = (double)batch * c->n_kv_heads;
-  const double t_warp = 5.0 + 1.0 * (double)max_p;
+  // warp pairs (two warps per segment, from 4 pages on, while 2 warps per segment fit
+  // about 12 resident warps per SM) halve a warp's pages
+  const bool pairs = max_p >= 4 && 2.0 * segs <= 12.0 * c->sm_count;
+  const double t_warp = 5.0 + 1.0 * (double)max_p / (pairs ? 2.0 : 1.0);
   const double t_shared = 11.5 + 0.01 * segs + 0.15 * (double)total_pages / c->sm_count;
   return t_warp < t_shared;
 }
